@@ -1,0 +1,175 @@
+/*
+ * pa.h -- C ABI of the B200 (sm_100a) paged-KV grouped-query attention engine.
+ *
+ * The engine computes, for a batch of variable-length requests whose keys and
+ * values live in a shared page pool,
+ *
+ *     O = softmax(scale * Q K^T + causal mask) V,   LSE = ln sum exp(scale * Q K^T)
+ *
+ * in one launch sequence that covers decode (one query token per request),
+ * causal paged prefill and mixed batches of both.
+ *
+ * Sources for the contract:
+ *  - "integrate PrimTS FMHA kernels" (TensorRT-LLM PR #17399), section
+ *    "Unified page-table metadata": an int32 row-strided page table [B, C]
+ *    plus live int32 seq_lens[B]; logical page p of request b is
+ *    page_table[b][p]; columns past ceil(seq_lens[b] / page_size) are never
+ *    read.  Section "Planning, preprocessing, and workspace ownership": one
+ *    plan per active batch size, geometry and capacity fixed in the plan,
+ *    request metadata bound at run time; only a split counter is reset per
+ *    run.  Section "Integration and supported scope": page sizes
+ *    16/32/64/128, head dims 64/128/256, GQA ratio up to 32, fail closed on
+ *    anything else.
+ *  - "Unified Triton kernel that doesn't distinguish between prefill +
+ *    decode" (vLLM PR #16828): varlen packed queries addressed by cu_q_lens
+ *    (like flash_attn_varlen_func), GQA query heads packed along the query
+ *    dimension, causal mask applied by select to -inf.
+ *  - "[Perf][FA4] Warm up dense (paged) FA4 attention kernels" (vLLM PR
+ *    #48156), review thread: split-KV decode (num_splits > 1, 0 = automatic)
+ *    and CUDA-graph (FULL) decode, hence pa_run must be capturable.
+ *
+ * Conventions of every entry point:
+ *  - Pointers named as device pointers must point to memory of the current
+ *    CUDA device; they are owned by the caller and only read or written during
+ *    the stream work that pa_run enqueues.
+ *  - Integer return codes: PA_OK (0) on success, otherwise a PA_ERR_* value;
+ *    pa_last_error() then describes the failure (thread-local string, valid
+ *    until the next call on the same thread).
+ *  - A plan is not safe for concurrent use from several streams or threads:
+ *    its workspace is shared by all runs.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *pa_stream_t;
+
+typedef struct pa_plan pa_plan; /* opaque; owns the device workspace */
+
+enum {
+    PA_OK = 0,
+    PA_ERR_INVALID = 1,     /* NULL or misaligned pointer, bad argument value */
+    PA_ERR_UNSUPPORTED = 2, /* geometry outside the supported envelope */
+    PA_ERR_CUDA = 3         /* a CUDA runtime call or launch failed */
+};
+
+/* Bits of the sticky device status word (pa_get_status).  The kernels never
+ * trap and never wait on the host; they record bad request data here and
+ * carry on with a defined fallback for the affected rows. */
+enum {
+    PA_STATUS_BAD_PAGE = 1u << 0,     /* a live page id < 0 or >= num_pages: that
+                                         page reads as zeros, outputs of the request
+                                         are unspecified */
+    PA_STATUS_Q_GT_KV = 1u << 1,      /* q_b > seq_lens[b]: rows that see no key get
+                                         O = 0, LSE = -inf */
+    PA_STATUS_KV_GT_CAPACITY = 1u << 2, /* seq_lens[b] > capacity * page_size or < 0:
+                                         clamped into [0, capacity * page_size] */
+    PA_STATUS_BAD_CU_Q = 1u << 3,     /* cu_q_lens decreasing or cu_q_lens[0] != 0:
+                                         the request is treated as having no tokens */
+    PA_STATUS_TIMEOUT = 1u << 4       /* an internal pipeline wait ran out (never
+                                         expected); the launch returned early */
+};
+
+/*
+ * pa_create_plan -- validate a geometry and allocate the plan's workspace.
+ *
+ *   batch       B, number of requests each pa_run covers (> 0)
+ *   heads_q     Hq, query heads (> 0, multiple of heads_kv)
+ *   heads_kv    Hkv, KV heads (> 0); GQA ratio G = Hq / Hkv must be <= 32
+ *   head_dim    D in {64, 128, 256}
+ *   page_size   ps in {16, 32, 64, 128}
+ *   capacity    C, columns of the page table (> 0); C * ps bounds seq_lens
+ *
+ * Allocates the workspace (work list, split partials, status word) on the
+ * current device with cudaMalloc.  Returns NULL on error (pa_last_error()
+ * says why: unsupported geometry, non-positive argument, CUDA failure).
+ * The softmax scale defaults to 1/sqrt(head_dim).
+ */
+PA_API pa_plan *pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int page_size,
+                        int capacity);
+
+/*
+ * pa_run -- enqueue one attention pass on `stream`.
+ *
+ *   q          device, bf16 [T, Hq, D], row-major; T = cu_q_lens[B]
+ *   k_pool     device, bf16 [P, ps, Hkv, D], row-major page pool of keys
+ *   v_pool     device, bf16 [P, ps, Hkv, D], row-major page pool of values
+ *   page_table device, int32 [B, C], row stride C; page_table[b][p] is the
+ *              physical page holding keys p*ps .. p*ps+ps-1 of request b.
+ *              Columns at or past ceil(seq_lens[b] / ps) are never read.
+ *   seq_lens   device, int32 [B]; seq_lens[b] = KV length of request b,
+ *              including this step's query tokens (0 <= seq_lens[b] <= C*ps)
+ *   cu_q_lens  device, int32 [B+1], cu_q_lens[0] = 0, nondecreasing; request b
+ *              owns query rows cu_q_lens[b] .. cu_q_lens[b+1]-1.  NULL means
+ *              one query token per request (pure decode, T = B).
+ *   out        device, bf16 [T, Hq, D]; row (t, h) = attention of query t,
+ *              head h over the keys it may see (round to nearest even)
+ *   lse        device, fp32 [T, Hq], natural-log log-sum-exp of the scaled
+ *              scores of each row; may be NULL
+ *
+ * Query i (0-based within request b, q_b = cu_q_lens[b+1] - cu_q_lens[b])
+ * sees keys j < seq_lens[b] - q_b + i + 1 (causal mask aligned to the end of
+ * the request's KV; decode sees every key).  Query head h reads KV head
+ * h / G.  All pointers must be 16-byte aligned.
+ *
+ * Enqueues at most three kernels (scheduler, attention, split merge); does
+ * not allocate, does not synchronise and reads no device data on the host,
+ * so it can be captured in a CUDA graph.  Returns PA_OK, PA_ERR_INVALID
+ * (NULL or misaligned pointer) or PA_ERR_CUDA (launch failure).  Problems in
+ * the device-side request data are recorded in the status word instead.
+ */
+PA_API int pa_run(pa_plan *plan, const void *q, const void *k_pool, const void *v_pool,
+           const int32_t *page_table, const int32_t *seq_lens, const int32_t *cu_q_lens,
+           void *out, float *lse, pa_stream_t stream);
+
+/* pa_destroy -- free the workspace and the plan.  NULL is a no-op.  The
+ * caller must make sure no enqueued pa_run on the plan is still pending. */
+PA_API void pa_destroy(pa_plan *plan);
+
+/* Description of the last error on this thread ("" if none). */
+PA_API const char *pa_last_error(void);
+
+/* Softmax scale applied to Q K^T (finite, > 0).  Default 1/sqrt(head_dim). */
+PA_API int pa_set_scale(pa_plan *plan, float scale);
+
+/* Number of pages P in the pools (the page-pool bound, cf. the PrimTS PR's
+ * "page-pool bound" of the active layer).  With P > 0 every live page id is
+ * checked against [0, P) and out-of-range pages read as zeros (status bit
+ * PA_STATUS_BAD_PAGE).  0 (default) trusts the table: negative ids still read
+ * as zeros, but ids >= the real pool size are undefined behaviour. */
+PA_API int pa_set_num_pages(pa_plan *plan, int num_pages);
+
+/* KV splits for requests whose packed query rows fit one 128-row tile
+ * (decode-like requests): 0 = automatic (default), 1 = never split,
+ * n > 1 = split every such request into min(n, its KV tiles) chunks.
+ * May reallocate the workspace; call it outside graph capture. */
+PA_API int pa_set_num_splits(pa_plan *plan, int num_splits);
+
+/* Synchronise `stream`, copy the sticky status word (PA_STATUS_* bits) to
+ * *status and, if clear != 0, reset it to 0.  Not capturable. */
+PA_API int pa_get_status(pa_plan *plan, pa_stream_t stream, uint32_t *status, int clear);
+
+/* Bytes of device workspace the plan holds. */
+PA_API size_t pa_workspace_bytes(const pa_plan *plan);
+
+/* Largest number of KV splits this plan can use for one request. */
+PA_API int pa_max_splits(const pa_plan *plan);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

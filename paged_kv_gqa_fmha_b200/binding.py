@@ -1,0 +1,190 @@
+"""ctypes binding of the C ABI in ``include/pa.h``.
+
+Argument marshalling only: tensors are checked for dtype, shape, device and
+contiguity, then their device pointers and the current CUDA stream are passed
+to ``libpa_b200.so``.  Every step of the attention runs in the library's
+kernels; there is no other implementation behind this module, and it raises if
+the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpa_b200.so")
+
+PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA = 0, 1, 2, 3
+STATUS_BAD_PAGE = 1 << 0
+STATUS_Q_GT_KV = 1 << 1
+STATUS_KV_GT_CAPACITY = 1 << 2
+STATUS_BAD_CU_Q = 1 << 3
+STATUS_TIMEOUT = 1 << 4
+
+EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_scale",
+           "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
+           "pa_max_splits")
+
+_lib = None
+
+
+class PAError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__("%s (code %d)" % (msg, code))
+        self.code = code
+
+
+def load_library(path: str = LIB_PATH):
+    """Load ``libpa_b200.so`` and declare the C signatures."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError("paged_kv_gqa_fmha_b200: CUDA library %s is missing; build it with "
+                           "`python -m paged_kv_gqa_fmha_b200._build`" % path)
+    lib = ctypes.CDLL(path)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.pa_create_plan.argtypes = [I, I, I, I, I, I]
+    lib.pa_create_plan.restype = P
+    lib.pa_run.argtypes = [P, P, P, P, P, P, P, P, P, P]
+    lib.pa_run.restype = I
+    lib.pa_destroy.argtypes = [P]
+    lib.pa_destroy.restype = None
+    lib.pa_last_error.argtypes = []
+    lib.pa_last_error.restype = ctypes.c_char_p
+    lib.pa_set_scale.argtypes = [P, F]
+    lib.pa_set_scale.restype = I
+    lib.pa_set_num_pages.argtypes = [P, I]
+    lib.pa_set_num_pages.restype = I
+    lib.pa_set_num_splits.argtypes = [P, I]
+    lib.pa_set_num_splits.restype = I
+    lib.pa_get_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32), I]
+    lib.pa_get_status.restype = I
+    lib.pa_workspace_bytes.argtypes = [P]
+    lib.pa_workspace_bytes.restype = ctypes.c_size_t
+    lib.pa_max_splits.argtypes = [P]
+    lib.pa_max_splits.restype = I
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def last_error() -> str:
+    return load_library().pa_last_error().decode()
+
+
+def _check(rc):
+    if rc != PA_OK:
+        raise PAError(rc, last_error())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class Plan:
+    """One geometry (batch, heads, head_dim, page size, capacity): owns the
+    device workspace; ``run`` binds the request metadata of each call."""
+
+    def __init__(self, batch, heads_q, heads_kv, head_dim, page_size, capacity,
+                 scale: Optional[float] = None, num_pages: int = 0, num_splits: int = 0):
+        self._lib = load_library()
+        self._h = self._lib.pa_create_plan(batch, heads_q, heads_kv, head_dim, page_size,
+                                           capacity)
+        if not self._h:
+            raise PAError(PA_ERR_INVALID, last_error())
+        self.batch, self.heads_q, self.heads_kv = batch, heads_q, heads_kv
+        self.head_dim, self.page_size, self.capacity = head_dim, page_size, capacity
+        if scale is not None:
+            _check(self._lib.pa_set_scale(self._h, float(scale)))
+        if num_pages:
+            _check(self._lib.pa_set_num_pages(self._h, int(num_pages)))
+        if num_splits:
+            _check(self._lib.pa_set_num_splits(self._h, int(num_splits)))
+
+    def set_num_pages(self, n: int):
+        _check(self._lib.pa_set_num_pages(self._h, int(n)))
+
+    def set_num_splits(self, n: int):
+        _check(self._lib.pa_set_num_splits(self._h, int(n)))
+
+    def set_scale(self, s: float):
+        _check(self._lib.pa_set_scale(self._h, float(s)))
+
+    @property
+    def workspace_bytes(self) -> int:
+        return int(self._lib.pa_workspace_bytes(self._h))
+
+    @property
+    def max_splits(self) -> int:
+        return int(self._lib.pa_max_splits(self._h))
+
+    def run(self, q, k_pool, v_pool, page_table, seq_lens, cu_q_lens=None, out=None, lse=None,
+            want_lse=True, stream=None):
+        """Enqueue one pass on ``stream`` (default: torch's current stream).
+        Returns (out, lse); lse is None if ``want_lse`` is False and no ``lse``
+        tensor was given."""
+        B, Hq, Hkv, D = self.batch, self.heads_q, self.heads_kv, self.head_dim
+        dev = q.device
+        if dev.type != "cuda":
+            raise ValueError("tensors must be on a CUDA device")
+        for name, t, dt in (("q", q, torch.bfloat16), ("k_pool", k_pool, torch.bfloat16),
+                            ("v_pool", v_pool, torch.bfloat16),
+                            ("page_table", page_table, torch.int32),
+                            ("seq_lens", seq_lens, torch.int32)):
+            if t.dtype != dt or t.device != dev or not t.is_contiguous():
+                raise ValueError("%s must be a contiguous %s tensor on %s" % (name, dt, dev))
+        if q.dim() != 3 or q.shape[1] != Hq or q.shape[2] != D:
+            raise ValueError("q must be [T, %d, %d], got %s" % (Hq, D, tuple(q.shape)))
+        if k_pool.dim() != 4 or tuple(k_pool.shape[1:]) != (self.page_size, Hkv, D):
+            raise ValueError("k_pool must be [P, %d, %d, %d], got %s"
+                             % (self.page_size, Hkv, D, tuple(k_pool.shape)))
+        if v_pool.shape != k_pool.shape:
+            raise ValueError("v_pool shape %s != k_pool shape %s"
+                             % (tuple(v_pool.shape), tuple(k_pool.shape)))
+        if tuple(page_table.shape) != (B, self.capacity):
+            raise ValueError("page_table must be [%d, %d]" % (B, self.capacity))
+        if tuple(seq_lens.shape) != (B,):
+            raise ValueError("seq_lens must be [%d]" % B)
+        if cu_q_lens is not None:
+            if (cu_q_lens.dtype != torch.int32 or tuple(cu_q_lens.shape) != (B + 1,)
+                    or cu_q_lens.device != dev or not cu_q_lens.is_contiguous()):
+                raise ValueError("cu_q_lens must be a contiguous int32 [%d] tensor" % (B + 1))
+        elif q.shape[0] != B:
+            raise ValueError("without cu_q_lens, q must hold one token per request")
+        T = q.shape[0]
+        if out is None:
+            out = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=dev)
+        if lse is None and want_lse:
+            lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+        if stream is None:
+            stream = torch.cuda.current_stream(dev).cuda_stream
+        elif isinstance(stream, torch.cuda.Stream):
+            stream = stream.cuda_stream
+        _check(self._lib.pa_run(self._h, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table),
+                                _ptr(seq_lens), _ptr(cu_q_lens), _ptr(out), _ptr(lse),
+                                ctypes.c_void_p(stream)))
+        return out, lse
+
+    def status(self, clear: bool = True, stream=None) -> int:
+        """Synchronise and read (then clear) the sticky device status word."""
+        if stream is None:
+            stream = torch.cuda.current_stream().cuda_stream
+        v = ctypes.c_uint32(0)
+        _check(self._lib.pa_get_status(self._h, ctypes.c_void_p(stream), ctypes.byref(v),
+                                       1 if clear else 0))
+        return int(v.value)
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.pa_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

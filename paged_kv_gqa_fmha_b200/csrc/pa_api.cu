@@ -1,0 +1,414 @@
+// pa_api.cu -- the C ABI declared in include/pa.h.
+//
+// Host side only: argument validation, plan / workspace ownership, TMA tensor
+// maps for the q tensor and the two page pools, and the three launches.  No
+// host <-> device synchronisation happens in pa_run, so it can be captured in
+// a CUDA graph (decode is run as FULL CUDA graphs in the FA4 warm-up PR, vLLM
+// #48156; PrimTS tests generation CUDA-graph replay, TensorRT-LLM #17399).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/pa.h"
+#include "pa_kernels.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+void set_err(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+struct pa_plan {
+  int B, Hq, Hkv, D, ps, C, G;
+  int device, n_sm;
+  float scale;
+  int num_pages;
+  int num_splits;   // 0 auto, 1 off, n forced
+  int S_max;
+  int max_items;
+  int tpb, box_h, BN;
+  // workspace
+  void* ws;
+  size_t ws_bytes;
+  pa::WsHeader* hdr;
+  int4* req_info;
+  pa::WorkItem* items;
+  float* part_lse;
+  float* part_o;
+  // tensor-map cache
+  const void* tm_ptr[3];
+  int tm_num_pages;
+  CUtensorMap tm_q, tm_k, tm_v;
+};
+
+namespace {
+
+int kv_tile(int D) { return D == 256 ? 64 : 128; }
+
+int auto_smax(int B, int Hkv, int n_sm) {
+  const long units = (long)B * Hkv;
+  long s = (4L * n_sm + units - 1) / units;
+  if (s > pa::kMaxSplits) s = pa::kMaxSplits;
+  if (s < 1) s = 1;
+  return (int)s;
+}
+
+// (Re)allocate the workspace for the plan's current S_max.
+int alloc_workspace(pa_plan* p) {
+  const int G = p->G;
+  const long blocks_per_req = (long)(((long)p->C * p->ps + p->tpb - 1) / p->tpb);
+  long per_req = blocks_per_req > p->S_max ? blocks_per_req : p->S_max;
+  const long max_items = (long)p->B * p->Hkv * per_req;
+  if (max_items > (1L << 30)) {
+    set_err("pa: work list would need %ld items (batch * heads_kv * capacity too large)",
+            max_items);
+    return PA_ERR_UNSUPPORTED;
+  }
+  (void)G;
+  const size_t n_part_rows = p->S_max > 1 ? (size_t)p->B * p->Hkv * p->S_max * pa::kBM : 0;
+  size_t off = 0;
+  const size_t o_hdr = off; off = align_up(off + sizeof(pa::WsHeader), 256);
+  const size_t o_req = off; off = align_up(off + sizeof(int4) * (size_t)p->B, 256);
+  const size_t o_items = off; off = align_up(off + sizeof(pa::WorkItem) * (size_t)max_items, 256);
+  const size_t o_plse = off; off = align_up(off + sizeof(float) * n_part_rows, 256);
+  const size_t o_po = off; off = align_up(off + sizeof(float) * n_part_rows * p->D, 256);
+  void* ws = nullptr;
+  cudaError_t e = cudaMalloc(&ws, off);
+  if (e != cudaSuccess) {
+    set_err("pa: cudaMalloc of %zu workspace bytes failed: %s", off, cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  e = cudaMemset(ws, 0, o_req);
+  if (e != cudaSuccess) {
+    cudaFree(ws);
+    set_err("pa: cudaMemset failed: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  if (p->ws) cudaFree(p->ws);
+  p->ws = ws;
+  p->ws_bytes = off;
+  char* c = static_cast<char*>(ws);
+  p->hdr = reinterpret_cast<pa::WsHeader*>(c + o_hdr);
+  p->req_info = reinterpret_cast<int4*>(c + o_req);
+  p->items = reinterpret_cast<pa::WorkItem*>(c + o_items);
+  p->part_lse = reinterpret_cast<float*>(c + o_plse);
+  p->part_o = reinterpret_cast<float*>(c + o_po);
+  p->max_items = (int)max_items;
+  return PA_OK;
+}
+
+template <int D>
+cudaError_t set_smem_attr() {
+  return cudaFuncSetAttribute(pa::pa_attention_kernel<D>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              pa::TileCfg<D>::SMEM_BYTES);
+}
+
+int encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
+           const cuuint64_t* strides, const cuuint32_t* box, const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    set_err("pa: cuTensorMapEncodeTiled is not available from the driver");
+    return PA_ERR_CUDA;
+  }
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_err("pa: cuTensorMapEncodeTiled(%s) failed with %d", what, (int)r);
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+int build_maps(pa_plan* p, const void* q, const void* k, const void* v) {
+  if (p->tm_ptr[0] == q && p->tm_ptr[1] == k && p->tm_ptr[2] == v &&
+      p->tm_num_pages == p->num_pages)
+    return PA_OK;
+  const cuuint64_t e = 2;  // bytes per bf16
+  // q [T, Hq, D]: dims (D, Hq, T bound); box (64, G, tokens per block).
+  // T is only known on the device; every coordinate the kernel issues stays
+  // below cu_q_lens[B], and B * C * ps bounds T for valid inputs.
+  {
+    cuuint64_t tb = (cuuint64_t)p->B * p->C * p->ps;
+    cuuint64_t dims[3] = {(cuuint64_t)p->D, (cuuint64_t)p->Hq, tb};
+    cuuint64_t str[2] = {(cuuint64_t)p->D * e, (cuuint64_t)p->Hq * p->D * e};
+    cuuint32_t box[3] = {64, (cuuint32_t)p->G, (cuuint32_t)p->tpb};
+    int rc = encode(&p->tm_q, q, 3, dims, str, box, "q");
+    if (rc) return rc;
+  }
+  // pools [P, ps, Hkv, D]: dims (D, Hkv, ps, P); box (64, 1, box_h, 1).
+  {
+    cuuint64_t P = p->num_pages > 0 ? (cuuint64_t)p->num_pages : (cuuint64_t)0x7fffffff;
+    cuuint64_t dims[4] = {(cuuint64_t)p->D, (cuuint64_t)p->Hkv, (cuuint64_t)p->ps, P};
+    cuuint64_t str[3] = {(cuuint64_t)p->D * e, (cuuint64_t)p->Hkv * p->D * e,
+                         (cuuint64_t)p->ps * p->Hkv * p->D * e};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)p->box_h, 1};
+    int rc = encode(&p->tm_k, k, 4, dims, str, box, "k_pool");
+    if (rc) return rc;
+    rc = encode(&p->tm_v, v, 4, dims, str, box, "v_pool");
+    if (rc) return rc;
+  }
+  p->tm_ptr[0] = q;
+  p->tm_ptr[1] = k;
+  p->tm_ptr[2] = v;
+  p->tm_num_pages = p->num_pages;
+  return PA_OK;
+}
+
+bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_last_error(void) { return g_err; }
+
+pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int page_size,
+                        int capacity) {
+  g_err[0] = 0;
+  if (batch <= 0 || heads_q <= 0 || heads_kv <= 0 || head_dim <= 0 || page_size <= 0 ||
+      capacity <= 0) {
+    set_err("pa_create_plan: every argument must be > 0 (batch=%d heads_q=%d heads_kv=%d "
+            "head_dim=%d page_size=%d capacity=%d)",
+            batch, heads_q, heads_kv, head_dim, page_size, capacity);
+    return nullptr;
+  }
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) {
+    set_err("pa_create_plan: unsupported head_dim %d (supported: 64, 128, 256)", head_dim);
+    return nullptr;
+  }
+  if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128) {
+    set_err("pa_create_plan: unsupported page_size %d (supported: 16, 32, 64, 128)", page_size);
+    return nullptr;
+  }
+  if (heads_q % heads_kv != 0) {
+    set_err("pa_create_plan: heads_q %d is not a multiple of heads_kv %d", heads_q, heads_kv);
+    return nullptr;
+  }
+  const int G = heads_q / heads_kv;
+  if (G > 32) {
+    set_err("pa_create_plan: GQA ratio %d exceeds 32", G);
+    return nullptr;
+  }
+  if ((long)capacity * page_size > (1L << 30)) {
+    set_err("pa_create_plan: capacity * page_size too large");
+    return nullptr;
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  int n_sm = 0, major = 0;
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) {
+    set_err("pa_create_plan: no usable CUDA device: %s", cudaGetErrorString(e));
+    return nullptr;
+  }
+  if (major != 10) {
+    set_err("pa_create_plan: device %d has compute capability %d.x; this library is built "
+            "for sm_100a only", dev, major);
+    return nullptr;
+  }
+  if (head_dim == 64) e = set_smem_attr<64>();
+  else if (head_dim == 128) e = set_smem_attr<128>();
+  else e = set_smem_attr<256>();
+  if (e != cudaSuccess) {
+    set_err("pa_create_plan: cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
+    return nullptr;
+  }
+  pa_plan* p = new pa_plan();
+  p->B = batch; p->Hq = heads_q; p->Hkv = heads_kv; p->D = head_dim; p->ps = page_size;
+  p->C = capacity; p->G = G; p->device = dev; p->n_sm = n_sm;
+  p->scale = 1.0f / std::sqrt((float)head_dim);
+  p->num_pages = 0;
+  p->num_splits = 0;
+  p->BN = kv_tile(head_dim);
+  p->tpb = pa::kBM / G;
+  p->box_h = page_size < p->BN ? page_size : p->BN;
+  p->S_max = auto_smax(batch, heads_kv, n_sm);
+  p->ws = nullptr;
+  p->tm_ptr[0] = p->tm_ptr[1] = p->tm_ptr[2] = nullptr;
+  p->tm_num_pages = -1;
+  if (alloc_workspace(p) != PA_OK) {
+    delete p;
+    return nullptr;
+  }
+  return p;
+}
+
+void pa_destroy(pa_plan* p) {
+  if (!p) return;
+  if (p->ws) cudaFree(p->ws);
+  delete p;
+}
+
+int pa_set_scale(pa_plan* p, float scale) {
+  if (!p) { set_err("pa_set_scale: NULL plan"); return PA_ERR_INVALID; }
+  if (!(scale > 0.f) || !std::isfinite(scale)) {
+    set_err("pa_set_scale: scale must be finite and > 0");
+    return PA_ERR_INVALID;
+  }
+  p->scale = scale;
+  return PA_OK;
+}
+
+int pa_set_num_pages(pa_plan* p, int num_pages) {
+  if (!p) { set_err("pa_set_num_pages: NULL plan"); return PA_ERR_INVALID; }
+  if (num_pages < 0) { set_err("pa_set_num_pages: negative page count"); return PA_ERR_INVALID; }
+  p->num_pages = num_pages;
+  return PA_OK;
+}
+
+int pa_set_num_splits(pa_plan* p, int num_splits) {
+  if (!p) { set_err("pa_set_num_splits: NULL plan"); return PA_ERR_INVALID; }
+  if (num_splits < 0 || num_splits > pa::kMaxSplits) {
+    set_err("pa_set_num_splits: %d outside [0, %d]", num_splits, pa::kMaxSplits);
+    return PA_ERR_INVALID;
+  }
+  int want = num_splits == 0 ? auto_smax(p->B, p->Hkv, p->n_sm) : num_splits;
+  if (want != p->S_max) {
+    const int old = p->S_max;
+    p->S_max = want;
+    int rc = alloc_workspace(p);
+    if (rc != PA_OK) {
+      p->S_max = old;
+      return rc;
+    }
+  }
+  p->num_splits = num_splits;
+  return PA_OK;
+}
+
+size_t pa_workspace_bytes(const pa_plan* p) { return p ? p->ws_bytes : 0; }
+
+int pa_max_splits(const pa_plan* p) { return p ? p->S_max : 0; }
+
+int pa_get_status(pa_plan* p, pa_stream_t stream, uint32_t* status, int clear) {
+  if (!p || !status) { set_err("pa_get_status: NULL argument"); return PA_ERR_INVALID; }
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess) e = cudaMemcpy(status, &p->hdr->status, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && clear) e = cudaMemset(&p->hdr->status, 0, sizeof(uint32_t));
+  if (e != cudaSuccess) {
+    set_err("pa_get_status: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
+           const int32_t* page_table, const int32_t* seq_lens, const int32_t* cu_q_lens,
+           void* out, float* lse, pa_stream_t stream) {
+  if (!p) { set_err("pa_run: NULL plan"); return PA_ERR_INVALID; }
+  if (!q || !k_pool || !v_pool || !page_table || !seq_lens || !out) {
+    set_err("pa_run: NULL pointer (q, k_pool, v_pool, page_table, seq_lens and out are required)");
+    return PA_ERR_INVALID;
+  }
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) ||
+      !aligned16(page_table) || !aligned16(seq_lens) || (cu_q_lens && !aligned16(cu_q_lens)) ||
+      (lse && !aligned16(lse))) {
+    set_err("pa_run: every pointer must be 16-byte aligned");
+    return PA_ERR_INVALID;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) {
+    set_err("pa_run: current device %d is not the plan's device %d", dev, p->device);
+    return PA_ERR_INVALID;
+  }
+  int rc = build_maps(p, q, k_pool, v_pool);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  pa::SchedParams sp;
+  sp.seq_lens = seq_lens;
+  sp.cu_q_lens = cu_q_lens;
+  sp.items = p->items;
+  sp.req_info = p->req_info;
+  sp.hdr = p->hdr;
+  sp.max_items = p->max_items;
+  sp.B = p->B; sp.Hkv = p->Hkv; sp.G = p->G; sp.C = p->C; sp.ps = p->ps; sp.BN = p->BN;
+  sp.tpb = p->tpb;
+  sp.S_max = p->num_splits == 1 ? 1 : p->S_max;
+  sp.forced_splits = p->num_splits > 1 ? p->num_splits : 0;
+  sp.n_ctas = p->n_sm;
+  pa::pa_schedule_kernel<<<1, pa::kCostBuckets, 0, st>>>(sp);
+
+  pa::AttnParams ap;
+  ap.q = static_cast<const uint16_t*>(q);
+  ap.page_table = page_table;
+  ap.cu_q_lens = cu_q_lens;
+  ap.out = static_cast<uint16_t*>(out);
+  ap.lse = lse;
+  ap.items = p->items;
+  ap.hdr = p->hdr;
+  ap.part_o = p->part_o;
+  ap.part_lse = p->part_lse;
+  ap.status = &p->hdr->status;
+  ap.B = p->B; ap.Hq = p->Hq; ap.Hkv = p->Hkv; ap.G = p->G; ap.C = p->C; ap.ps = p->ps;
+  ap.num_pages = p->num_pages;
+  ap.S_max = p->S_max;
+  ap.tpb = p->tpb;
+  ap.box_h = p->box_h;
+  ap.scale_log2 = p->scale * 1.4426950408889634f;
+  const dim3 grid(p->n_sm), block(pa::kThreads);
+  switch (p->D) {
+    case 64:
+      pa::pa_attention_kernel<64><<<grid, block, pa::TileCfg<64>::SMEM_BYTES, st>>>(p->tm_q, p->tm_k, p->tm_v, ap);
+      break;
+    case 128:
+      pa::pa_attention_kernel<128><<<grid, block, pa::TileCfg<128>::SMEM_BYTES, st>>>(p->tm_q, p->tm_k, p->tm_v, ap);
+      break;
+    default:
+      pa::pa_attention_kernel<256><<<grid, block, pa::TileCfg<256>::SMEM_BYTES, st>>>(p->tm_q, p->tm_k, p->tm_v, ap);
+      break;
+  }
+  if (sp.S_max > 1) {
+    pa::MergeParams mp;
+    mp.req_info = p->req_info;
+    mp.part_o = p->part_o;
+    mp.part_lse = p->part_lse;
+    mp.out = static_cast<uint16_t*>(out);
+    mp.lse = lse;
+    mp.B = p->B; mp.Hq = p->Hq; mp.Hkv = p->Hkv; mp.G = p->G; mp.D = p->D; mp.S_max = p->S_max;
+    pa::pa_merge_kernel<<<p->B * p->Hkv, 128, 0, st>>>(mp);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_err("pa_run: launch failed: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+}  // extern "C"

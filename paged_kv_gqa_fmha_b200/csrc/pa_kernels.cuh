@@ -1,0 +1,816 @@
+// pa_kernels.cuh -- device kernels of the paged-KV GQA attention engine (sm_100a).
+//
+// Three kernels run per pa_run, in stream order:
+//   1. pa_schedule_kernel: reads seq_lens / cu_q_lens on the device and writes
+//      a work list (one item per (request, KV head, 128-row query block, KV
+//      split)), longest first, plus per-request split counts.
+//   2. pa_attention_kernel<D>: persistent, one CTA per SM, warp-specialised:
+//        warps 0-3  softmax / correction / epilogue (one thread per query row)
+//        warp  4    producer: page-table-driven TMA gathers of K and V pages,
+//                   Q tiles by TMA (or plain loads for partial blocks)
+//        warp  5    MMA issuer: tcgen05 S = Q K^T and O += P V, TMEM accumulators
+//   3. pa_merge_kernel: log-sum-exp merge of split-KV partial states.
+//
+// Sources: page-table contract and page-pool bound from "integrate PrimTS FMHA
+// kernels" (TensorRT-LLM PR #17399, "Unified page-table metadata"); GQA
+// packing of query heads along M, varlen queries and the mask by select from
+// "Unified Triton kernel that doesn't distinguish between prefill + decode"
+// (vLLM PR #16828); 128-row query tiles and split-KV decode with num_splits
+// (0 = automatic) from "[Perf][FA4] Warm up dense (paged) FA4 attention
+// kernels" (vLLM PR #48156, review thread on q_stage and is_split_kv).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "sm100.cuh"
+
+namespace pa {
+
+// One unit of attention work.  Rows of the query block are packed token-major:
+// row r <-> (token q_tok0 + r / G, query head kvh * G + r % G).
+struct WorkItem {
+  int b, kvh, split, n_splits;
+  int q_tok0, n_tok;     // query tokens of the block (local to the request)
+  int kv_lo, kv_hi;      // keys [kv_lo, kv_hi) processed by this item
+  int kv_len, q_len;     // request lengths after validation
+  int t_base, pad;       // cu_q_lens[b]
+};
+static_assert(sizeof(WorkItem) == 48, "work item layout");
+
+// Device status bits (mirror of PA_STATUS_* in pa.h).
+constexpr unsigned kStatusBadPage = 1u << 0;
+constexpr unsigned kStatusQgtKv = 1u << 1;
+constexpr unsigned kStatusKvGtCap = 1u << 2;
+constexpr unsigned kStatusBadCuQ = 1u << 3;
+constexpr unsigned kStatusTimeout = 1u << 4;
+
+struct WsHeader {
+  unsigned status;
+  int n_items;
+  int pad[62];
+};
+
+constexpr int kBM = 128;              // query rows per tile (tcgen05 M)
+constexpr int kThreads = 192;         // 6 warps
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kCostBuckets = 1024;
+constexpr int kMaxSplits = 64;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows > 2^8
+
+template <int D>
+struct TileCfg {
+  static constexpr int BN = (D == 256) ? 64 : 128;   // keys per KV tile
+  static constexpr int DCH = D / 64;                  // 128-byte column chunks per row
+  static constexpr int Q_CHUNK = kBM * 128;           // bytes of one Q column chunk
+  static constexpr int Q_BYTES = kBM * D * 2;
+  static constexpr int SLOT_CHUNK = BN * 128;         // bytes of one K/V column chunk
+  static constexpr int SLOT_BYTES = BN * D * 2;
+  static constexpr int NSLOT = (D == 64) ? 12 : (D == 128 ? 6 : 5);
+  static constexpr int O_COL = 2 * BN;                // TMEM: S0 [0,BN), S1 [BN,2BN), O
+  static constexpr int TMEM_COLS = 512;
+  // barriers: q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full[2], p_full[2],
+  //           pv_done[2], o_empty, drain
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = 2 + NSLOT,
+                       B_SFULL = 2 + 2 * NSLOT, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
+                       B_OEMPTY = B_PVDONE + 2, B_DRAIN = B_OEMPTY + 1, NBAR = B_DRAIN + 1;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + NSLOT * SLOT_BYTES + BAR_BYTES;
+  static_assert(NBAR * 8 + 16 <= BAR_BYTES, "barrier area");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(O_COL + D <= TMEM_COLS, "TMEM columns");
+};
+
+struct AttnParams {
+  const uint16_t* q;          // bf16 [T, Hq, D]
+  const int* page_table;      // [B, C]
+  const int* cu_q_lens;       // [B+1] or nullptr
+  uint16_t* out;              // bf16 [T, Hq, D]
+  float* lse;                 // [T, Hq] or nullptr
+  const WorkItem* items;
+  const WsHeader* hdr;
+  float* part_o;              // [B*Hkv*S_max*128, D]
+  float* part_lse;            // [B*Hkv*S_max*128]
+  unsigned* status;
+  int B, Hq, Hkv, G, C, ps, num_pages, S_max, tpb, box_h;
+  float scale_log2;
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+__device__ __forceinline__ int item_tiles(const WorkItem& w, int BN) {
+  return w.kv_hi > w.kv_lo ? ceil_div(w.kv_hi - w.kv_lo, BN) : 0;
+}
+
+// Order in which K and V tiles of an item are loaded and consumed:
+// K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1).  S for tile j+1 is issued
+// before P*V of tile j so the tensor core works while softmax runs.
+__device__ __forceinline__ void kv_sequence(int s, int n, int& j, bool& is_v) {
+  if (s == 0) { j = 0; is_v = false; }
+  else if (s == 2 * n - 1) { j = n - 1; is_v = true; }
+  else if (s & 1) { j = (s + 1) >> 1; is_v = false; }
+  else { j = (s >> 1) - 1; is_v = true; }
+}
+
+// mbar_wait executed by every lane of a warp, with a warp-uniform result: a
+// lane that gives up makes the whole warp give up, so no lane is left behind
+// at a later warp-collective instruction.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
+// Wait without the abort shortcut, for draining in-flight copies at exit.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > 100000000ull) return;  // 100 ms
+  }
+}
+
+// =========================================================================== scheduler
+struct SchedParams {
+  const int* seq_lens;
+  const int* cu_q_lens;
+  WorkItem* items;
+  int4* req_info;      // [B] {n_splits, q_len, t_base, kv_len}
+  WsHeader* hdr;
+  int max_items;
+  int B, Hkv, G, C, ps, BN, tpb, S_max, forced_splits, n_ctas;
+};
+
+struct ReqInfo {
+  int q_len, t_base, kv_len;
+  unsigned flags;
+};
+
+__device__ __forceinline__ ReqInfo read_request(const SchedParams& p, int b) {
+  ReqInfo r;
+  r.flags = 0;
+  if (p.cu_q_lens) {
+    const int a = p.cu_q_lens[b], e = p.cu_q_lens[b + 1];
+    if (a < 0 || e < a || (b == 0 && a != 0)) {
+      r.flags |= kStatusBadCuQ;
+      r.q_len = 0;
+      r.t_base = a < 0 ? 0 : a;
+    } else {
+      r.q_len = e - a;
+      r.t_base = a;
+    }
+  } else {
+    r.q_len = 1;
+    r.t_base = b;
+  }
+  const int cap = p.C * p.ps;
+  int kv = p.seq_lens[b];
+  if (kv < 0) { r.flags |= kStatusKvGtCap; kv = 0; }
+  if (kv > cap) { r.flags |= kStatusKvGtCap; kv = cap; }
+  r.kv_len = kv;
+  if (r.q_len > kv) r.flags |= kStatusQgtKv;
+  if (r.q_len > cap) r.q_len = cap;   // keeps the work list within its bound
+  return r;
+}
+
+// Keys visible to the last row of query block [q0, q0 + n): the causal limit
+// aligned to the end of the request's KV, clamped to [0, kv_len].
+__device__ __forceinline__ int block_kv_hi(const ReqInfo& r, int q0, int n) {
+  int hi = q0 + n + (r.kv_len - r.q_len);
+  return hi < 0 ? 0 : (hi > r.kv_len ? r.kv_len : hi);
+}
+
+__device__ __forceinline__ int n_qblocks(const ReqInfo& r, int tpb) {
+  return r.q_len > 0 ? (r.q_len + tpb - 1) / tpb : 0;
+}
+
+// Split count and tiles per split of a request whose rows fit one query block.
+__device__ __forceinline__ void split_plan(const SchedParams& p, const ReqInfo& r, int chunk,
+                                           int& n_splits, int& per) {
+  const int tiles = ceil_div(block_kv_hi(r, 0, r.q_len), p.BN);
+  n_splits = 1;
+  per = tiles > 0 ? tiles : 1;
+  if (n_qblocks(r, p.tpb) != 1 || p.S_max <= 1 || tiles <= 1) return;
+  int s = p.forced_splits > 0 ? p.forced_splits : ceil_div(tiles, chunk);
+  if (s > p.S_max) s = p.S_max;
+  if (s > tiles) s = tiles;
+  if (s < 1) s = 1;
+  per = ceil_div(tiles, s);
+  n_splits = ceil_div(tiles, per);
+}
+
+__device__ __forceinline__ int cost_bucket(int tiles) {
+  return tiles < kCostBuckets ? tiles : kCostBuckets - 1;
+}
+
+__global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
+  __shared__ int hist[kCostBuckets];
+  __shared__ int cursor[kCostBuckets];
+  __shared__ unsigned long long total_tiles;
+  __shared__ int s_chunk;
+  __shared__ unsigned s_flags;
+  __shared__ int warp_sums[32];
+  const int tid = threadIdx.x;
+  for (int i = tid; i < kCostBuckets; i += blockDim.x) hist[i] = 0;
+  if (tid == 0) { total_tiles = 0; s_flags = 0; }
+  __syncthreads();
+
+  // Pass A: validate requests, count the KV tiles of all work.
+  unsigned long long my_tiles = 0;
+  unsigned my_flags = 0;
+  for (int b = tid; b < p.B; b += blockDim.x) {
+    const ReqInfo r = read_request(p, b);
+    my_flags |= r.flags;
+    const int nb = n_qblocks(r, p.tpb);
+    for (int m = 0; m < nb; ++m) {
+      const int q0 = m * p.tpb;
+      const int n = min(p.tpb, r.q_len - q0);
+      my_tiles += (unsigned long long)p.Hkv * ceil_div(block_kv_hi(r, q0, n), p.BN);
+    }
+  }
+  atomicAdd(&total_tiles, my_tiles);
+  if (my_flags) atomicOr(&s_flags, my_flags);
+  __syncthreads();
+  if (tid == 0) {
+    // tiles per split so that the whole launch is about two waves of CTAs
+    const unsigned long long target = (unsigned long long)p.n_ctas * 2ull;
+    unsigned long long c = (total_tiles + target - 1) / target;
+    s_chunk = (int)(c < 4 ? 4 : (c > (1ull << 30) ? (1ull << 30) : c));
+    if (s_flags) atomicOr(&p.hdr->status, s_flags);
+  }
+  __syncthreads();
+  const int chunk = s_chunk;
+
+  // Pass B: histogram of item costs (KV tiles per item).
+  for (int b = tid; b < p.B; b += blockDim.x) {
+    const ReqInfo r = read_request(p, b);
+    int ns, per;
+    split_plan(p, r, chunk, ns, per);
+    const int nb = n_qblocks(r, p.tpb);
+    if (ns > 1) {
+      const int tiles = ceil_div(block_kv_hi(r, 0, r.q_len), p.BN);
+      for (int s = 0; s < ns; ++s) {
+        const int t = min(per, tiles - s * per);
+        atomicAdd(&hist[cost_bucket(t)], p.Hkv);
+      }
+    } else {
+      for (int m = 0; m < nb; ++m) {
+        const int q0 = m * p.tpb;
+        const int n = min(p.tpb, r.q_len - q0);
+        atomicAdd(&hist[cost_bucket(ceil_div(block_kv_hi(r, q0, n), p.BN))], p.Hkv);
+      }
+    }
+  }
+  __syncthreads();
+
+  // Exclusive scan over buckets in descending cost order (longest items first).
+  {
+    const int lane = tid & 31, warp = tid >> 5;
+    int v = 0;
+    const int bucket = kCostBuckets - 1 - tid;        // blockDim.x == kCostBuckets
+    if (tid < kCostBuckets) v = hist[bucket];
+    int x = v;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_sums[lane] = w;   // inclusive
+    }
+    __syncthreads();
+    const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+    if (tid < kCostBuckets) cursor[bucket] = before;
+    if (tid == blockDim.x - 1) {
+      const int total = warp_sums[(blockDim.x >> 5) - 1];
+      p.hdr->n_items = total < p.max_items ? total : p.max_items;
+    }
+  }
+  __syncthreads();
+
+  // Pass C: emit the items.
+  for (int b = tid; b < p.B; b += blockDim.x) {
+    const ReqInfo r = read_request(p, b);
+    int ns, per;
+    split_plan(p, r, chunk, ns, per);
+    p.req_info[b] = make_int4(ns, r.q_len, r.t_base, r.kv_len);
+    const int nb = n_qblocks(r, p.tpb);
+    WorkItem w;
+    w.b = b;
+    w.n_splits = ns;
+    w.kv_len = r.kv_len;
+    w.q_len = r.q_len;
+    w.t_base = r.t_base;
+    w.pad = 0;
+    if (ns > 1) {
+      const int hi = block_kv_hi(r, 0, r.q_len);
+      const int tiles = ceil_div(hi, p.BN);
+      for (int s = 0; s < ns; ++s) {
+        const int t = min(per, tiles - s * per);
+        w.split = s;
+        w.q_tok0 = 0;
+        w.n_tok = r.q_len;
+        w.kv_lo = s * per * p.BN;
+        w.kv_hi = min(hi, (s + 1) * per * p.BN);
+        for (int g = 0; g < p.Hkv; ++g) {
+          w.kvh = g;
+          const int pos = atomicAdd(&cursor[cost_bucket(t)], 1);
+          if (pos < p.max_items) p.items[pos] = w;
+        }
+      }
+    } else {
+      for (int m = 0; m < nb; ++m) {
+        const int q0 = m * p.tpb;
+        const int n = min(p.tpb, r.q_len - q0);
+        w.split = 0;
+        w.q_tok0 = q0;
+        w.n_tok = n;
+        w.kv_lo = 0;
+        w.kv_hi = block_kv_hi(r, q0, n);
+        const int t = ceil_div(w.kv_hi, p.BN);
+        for (int g = 0; g < p.Hkv; ++g) {
+          w.kvh = g;
+          const int pos = atomicAdd(&cursor[cost_bucket(t)], 1);
+          if (pos < p.max_items) p.items[pos] = w;
+        }
+      }
+    }
+  }
+}
+
+// =========================================================================== attention
+template <int D>
+__device__ __forceinline__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                              const CUtensorMap* tm_v, const AttnParams& p,
+                                              uint32_t sQ, uint32_t sKV, uint32_t bar0,
+                                              int n_items, volatile int* abort) {
+  using C = TileCfg<D>;
+  const int lane = threadIdx.x & 31;
+  const int G = p.G;
+  const int T = p.cu_q_lens ? p.cu_q_lens[p.B] : p.B;
+  uint32_t ld_idx = 0, q_cnt = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    const WorkItem w = p.items[it];
+    const int n = item_tiles(w, C::BN);
+    if (n == 0) continue;
+    // ---- Q tile
+    if (!warp_wait(bar0 + 8 * C::B_QEMPTY, (q_cnt & 1) ^ 1, abort)) { ok = false; break; }
+    const int t0 = w.t_base + w.q_tok0;
+    if (w.n_tok == p.tpb && t0 + p.tpb <= T) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar0 + 8 * C::B_QFULL, C::DCH * p.tpb * G * 128);
+        for (int c = 0; c < C::DCH; ++c)
+          tma_load_3d(sQ + c * C::Q_CHUNK, tm_q, bar0 + 8 * C::B_QFULL, c * 64, w.kvh * G, t0);
+      }
+    } else {
+      // Partial block: plain 16-byte loads of the live rows only, stored with the
+      // same 128-byte swizzle the TMA uses (16-byte unit u of row r lands at
+      // unit u ^ (r % 8) of that row).
+      const int rows = w.n_tok * G;
+      const int units = rows * (D / 8);
+      for (int u = lane; u < units; u += 32) {
+        const int r = u / (D / 8), c16 = u % (D / 8);
+        const int t = t0 + r / G, h = w.kvh * G + r % G;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)t * p.Hq + h) * D) + c16);
+        const uint32_t dst = sQ + (c16 >> 3) * C::Q_CHUNK + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y),
+                     "r"(v.z), "r"(v.w)
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar0 + 8 * C::B_QFULL);
+    }
+    ++q_cnt;
+    // ---- K / V tiles, gathered page by page
+    for (int s = 0; s < 2 * n; ++s) {
+      int j;
+      bool is_v;
+      kv_sequence(s, n, j, is_v);
+      const uint32_t slot = ld_idx % C::NSLOT;
+      if (!warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
+        ok = false;
+        break;
+      }
+      const int n0 = w.kv_lo + j * C::BN;
+      // every live row of the tile is loaded (rows past the item's causal limit
+      // included) so that no stale shared memory meets P * V
+      const int live = min(w.kv_len - n0, C::BN);
+      const int nbox = ceil_div(live, p.box_h);
+      const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
+      if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
+      __syncwarp();
+      if (lane < nbox) {
+        const int tok = n0 + lane * p.box_h;
+        const int col = tok / p.ps, row = tok - col * p.ps;
+        int page = p.page_table[(size_t)w.b * p.C + col];
+        if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
+          atomicOr(p.status, kStatusBadPage);
+          page = -1;   // out of the tensor map: the box reads as zeros
+        }
+        const CUtensorMap* tm = is_v ? tm_v : tm_k;
+        const uint32_t dst = sKV + slot * C::SLOT_BYTES + lane * p.box_h * 128;
+        for (int c = 0; c < C::DCH; ++c)
+          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, row, page);
+      }
+      ++ld_idx;
+    }
+  }
+  if (!ok || *abort) {
+    // wait (bounded) for our copies still in flight before the CTA exits
+    if (lane == 0) {
+      const uint32_t first = ld_idx > (uint32_t)C::NSLOT ? ld_idx - C::NSLOT : 0;
+      for (uint32_t k = first; k < ld_idx; ++k)
+        mbar_drain(bar0 + 8 * (C::B_KVFULL + k % C::NSLOT), (k / C::NSLOT) & 1);
+      if (q_cnt > 0) mbar_drain(bar0 + 8 * C::B_QFULL, (q_cnt - 1) & 1);
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint32_t sKV,
+                                         uint32_t bar0, uint32_t tmem, int n_items,
+                                         volatile int* abort) {
+  using C = TileCfg<D>;
+  constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, C::BN, false, false);
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, false, true);
+  uint32_t ld_idx = 0, g_base = 0, q_cnt = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    const WorkItem w = p.items[it];
+    const int n = item_tiles(w, C::BN);
+    if (n == 0) continue;
+    if (!mbar_wait(bar0 + 8 * C::B_QFULL, q_cnt & 1, abort)) { ok = false; break; }
+    tc_fence_after();
+    for (int s = 0; s < 2 * n; ++s) {
+      int j;
+      bool is_v;
+      kv_sequence(s, n, j, is_v);
+      const uint32_t slot = ld_idx % C::NSLOT;
+      if (!mbar_wait(bar0 + 8 * (C::B_KVFULL + slot), (ld_idx / C::NSLOT) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t slot_addr = sKV + slot * C::SLOT_BYTES;
+      const uint32_t g = g_base + j, sb = g & 1;
+      if (!is_v) {
+        // S[sb] = Q K^T: K-major A (Q) and B (K), 16 columns of D per MMA
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(sQ + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              smem_desc_sw128(slot_addr + (kk >> 2) * C::SLOT_CHUNK + (kk & 3) * 32, 16, 1024);
+          mma_ss(tmem + sb * C::BN, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar0 + 8 * (C::B_SFULL + sb));
+        tc_commit(bar0 + 8 * (C::B_KVEMPTY + slot));
+        if (j == n - 1) tc_commit(bar0 + 8 * C::B_QEMPTY);
+      } else {
+        if (!mbar_wait(bar0 + 8 * (C::B_PFULL + sb), (g >> 1) & 1, abort)) { ok = false; break; }
+        if (j == 0 && !mbar_wait(bar0 + 8 * C::B_OEMPTY, (q_cnt & 1) ^ 1, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // O += P V: A = P (bf16, packed two per TMEM column), B = V tile (MN-major:
+        // D contiguous), 16 keys per MMA
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(slot_addr + kk * 16 * 128, C::SLOT_CHUNK, 1024);
+          mma_ts(tmem + C::O_COL, tmem + sb * C::BN + kk * 8, bd, kIdescPV,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(bar0 + 8 * (C::B_PVDONE + sb));
+        tc_commit(bar0 + 8 * (C::B_KVEMPTY + slot));
+      }
+      ++ld_idx;
+    }
+    g_base += n;
+    ++q_cnt;
+  }
+  // all MMAs issued by this thread complete before TMEM is released
+  tc_commit(bar0 + 8 * C::B_DRAIN);
+  mbar_drain(bar0 + 8 * C::B_DRAIN, 0);
+}
+
+template <int D>
+__device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, uint32_t bar0,
+                                             uint32_t tmem, int n_items, volatile int* abort) {
+  using C = TileCfg<D>;
+  constexpr int BN = C::BN;
+  const int r = threadIdx.x;          // query row of the tile, 0..127
+  const int warp = r >> 5, lane = r & 31;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);   // this warp's lanes
+  const int G = p.G;
+  uint32_t g_base = 0, ld_base = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    const WorkItem w = p.items[it];
+    const int n = item_tiles(w, BN);
+    const int n_rows = w.n_tok * G;
+    const bool real = r < n_rows;
+    const bool warp_active = warp * 32 < n_rows;
+    const int t = w.t_base + w.q_tok0 + r / G;
+    const int h = w.kvh * G + r % G;
+    const bool split = w.n_splits > 1;
+    const size_t prow = ((((size_t)w.b * p.Hkv + w.kvh) * p.S_max + w.split) * kBM + r);
+    if (n == 0) {
+      // no key is visible to any row of the block: O = 0, LSE = -inf
+      if (real) {
+        if (split) {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D);
+          for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+          p.part_lse[prow] = -INFINITY;
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)t * p.Hq + h) * D);
+          for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+          if (p.lse) p.lse[(size_t)t * p.Hq + h] = -INFINITY;
+        }
+      }
+      continue;
+    }
+    // keys visible to this row: [kv_lo, lim)
+    const int i_r = w.q_tok0 + r / G;
+    const int lim = min(w.kv_hi, i_r + (w.kv_len - w.q_len) + 1);
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int j = 0; j < n && ok; ++j) {
+      const uint32_t g = g_base + j, sb = g & 1;
+      if (!warp_wait(bar0 + 8 * (C::B_SFULL + sb), (g >> 1) & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      const int n0 = w.kv_lo + j * BN;
+      if (warp_active) {
+        float s[BN];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(trow + sb * BN + c * 32, v);
+          tmem_ld_wait(v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(v[e]);
+        }
+        const int nvis = lim - n0;
+        if (nvis < BN) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c >= nvis) s[c] = -INFINITY;   // mask by select, never by add
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_run, mx * p.scale_log2);
+        const bool need = real && (m_new > m_run + kRescaleThreshold);
+        if (j > 0 && __any_sync(0xffffffffu, need && m_run != -INFINITY)) {
+          // O holds the sum up to tile g-1: wait for that P V, then rescale it
+          const uint32_t gp = g - 1;
+          if (!warp_wait(bar0 + 8 * (C::B_PVDONE + (gp & 1)), (gp >> 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(trow + C::O_COL + c * 32, v);
+            tmem_ld_wait(v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            tmem_st32(trow + C::O_COL + c * 32, v);
+          }
+          tmem_st_wait();
+        }
+        if (need) {
+          l_run *= ex2_approx(m_run - m_new);
+          m_run = m_new;
+        }
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        float rowsum = 0.f;
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_use));
+          const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_use));
+          rowsum += p0 + p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+        }
+        l_run += rowsum;
+        // P overwrites the first BN/2 columns of the S buffer it came from
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) tmem_st16(trow + sb * BN + c * 16, pk + c * 16);
+        tmem_st_wait();
+      }
+      if (j == n - 1) {
+        if (n0 + BN > w.kv_len) {
+          // Last tile of the request: rows at and past kv_len in the V tile are
+          // tail slots or rows never loaded; zero them so that 0 * garbage
+          // cannot reach O (P is 0 there, but 0 * NaN is NaN).
+          const uint32_t ldv = ld_base + 2 * n - 1;
+          const uint32_t slot = ldv % C::NSLOT;
+          if (!warp_wait(bar0 + 8 * (C::B_KVFULL + slot), (ldv / C::NSLOT) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          const int z0 = w.kv_len - n0;
+          const int units = (BN - z0) * C::DCH * 8;
+          const uint32_t base = sKV + slot * C::SLOT_BYTES;
+          for (int u = r; u < units; u += 128) {
+            const int row = z0 + u / (C::DCH * 8);
+            const int rem = u % (C::DCH * 8);
+            const uint32_t a = base + (rem >> 3) * C::SLOT_CHUNK + row * 128 + (rem & 7) * 16;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+          }
+          fence_proxy_async_smem();
+        }
+        // make sure the P V of the previous tile has completed before this
+        // tile's P is published (keeps pv_done phases unambiguous)
+        const uint32_t gp = g - 1;
+        if (!warp_wait(bar0 + 8 * (C::B_PVDONE + (gp & 1)), (gp >> 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar0 + 8 * (C::B_PFULL + sb));
+    }
+    if (!ok) break;
+    // ---- epilogue: O / l -> out (or the split partial), LSE
+    const uint32_t gl = g_base + n - 1;
+    if (!warp_wait(bar0 + 8 * (C::B_PVDONE + (gl & 1)), (gl >> 1) & 1, abort)) { ok = false; break; }
+    tc_fence_after();
+    if (warp_active) {
+      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+      const float lse_v = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(trow + C::O_COL + c * 32, v);
+        tmem_ld_wait(v);
+        if (real) {
+          if (split) {
+            float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv_l, __uint_as_float(v[4 * e + 1]) * inv_l,
+                                   __uint_as_float(v[4 * e + 2]) * inv_l,
+                                   __uint_as_float(v[4 * e + 3]) * inv_l);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)t * p.Hq + h) * D + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 q4;
+              q4.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * inv_l, __uint_as_float(v[8 * e + 1]) * inv_l);
+              q4.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * inv_l, __uint_as_float(v[8 * e + 3]) * inv_l);
+              q4.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * inv_l, __uint_as_float(v[8 * e + 5]) * inv_l);
+              q4.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * inv_l, __uint_as_float(v[8 * e + 7]) * inv_l);
+              dst[e] = q4;
+            }
+          }
+        }
+      }
+      if (real) {
+        if (split) p.part_lse[prow] = lse_v;
+        else if (p.lse) p.lse[(size_t)t * p.Hq + h] = lse_v;
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar0 + 8 * C::B_OEMPTY);
+    g_base += n;
+    ld_base += 2 * n;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    pa_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = TileCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;             // 1024-B aligned for SW128
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t sQ = base;
+  const uint32_t sKV = base + C::Q_BYTES;
+  const uint32_t bar0 = sKV + C::NSLOT * C::SLOT_BYTES;
+  uint8_t* bar_ptr = smem + C::Q_BYTES + C::NSLOT * C::SLOT_BYTES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NBAR);
+  volatile int* abort = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 4);
+
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(bar0 + 8 * C::B_QFULL, 1);
+    mbar_init(bar0 + 8 * C::B_QEMPTY, 1);
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(bar0 + 8 * (C::B_KVFULL + i), 1);
+      mbar_init(bar0 + 8 * (C::B_KVEMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar0 + 8 * (C::B_SFULL + i), 1);
+      mbar_init(bar0 + 8 * (C::B_PFULL + i), 4);
+      mbar_init(bar0 + 8 * (C::B_PVDONE + i), 1);
+    }
+    mbar_init(bar0 + 8 * C::B_OEMPTY, 4);
+    mbar_init(bar0 + 8 * C::B_DRAIN, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kProducerWarp && (threadIdx.x & 31) == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_items = p.hdr->n_items;
+
+  if (warp == kProducerWarp) {
+    producer_role<D>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bar0, n_items, abort);
+  } else if (warp == kMmaWarp) {
+    if ((threadIdx.x & 31) == 0) mma_role<D>(p, sQ, sKV, bar0, tmem, n_items, abort);
+    __syncwarp();
+  } else {
+    softmax_role<D>(p, sKV, bar0, tmem, n_items, abort);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort) atomicOr(p.status, kStatusTimeout);
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// =========================================================================== merge
+struct MergeParams {
+  const int4* req_info;  // {n_splits, q_len, t_base, kv_len}
+  const float* part_o;
+  const float* part_lse;
+  uint16_t* out;
+  float* lse;
+  int B, Hq, Hkv, G, D, S_max;
+};
+
+// out = sum_s exp(lse_s - L) O_s with L = ln sum_s exp(lse_s): the exact merge
+// of attention states over disjoint key ranges; empty splits (lse_s = -inf)
+// get weight 0.
+__global__ void __launch_bounds__(128) pa_merge_kernel(MergeParams p) {
+  const int bh = blockIdx.x;
+  const int b = bh / p.Hkv, kvh = bh % p.Hkv;
+  const int4 ri = p.req_info[b];
+  const int ns = ri.x;
+  if (ns <= 1) return;
+  const int n_rows = ri.y * p.G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = warp; r < n_rows; r += 4) {
+    const size_t base = (size_t)bh * p.S_max * kBM + r;   // + s * kBM
+    float l0 = lane < ns ? p.part_lse[base + (size_t)lane * kBM] : -INFINITY;
+    float l1 = lane + 32 < ns ? p.part_lse[base + (size_t)(lane + 32) * kBM] : -INFINITY;
+    float m = fmaxf(l0, l1);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float e = 0.f;
+    if (m != -INFINITY) {
+      e = (l0 == -INFINITY ? 0.f : expf(l0 - m)) + (l1 == -INFINITY ? 0.f : expf(l1 - m));
+    }
+    for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+    const float L = (m == -INFINITY) ? -INFINITY : m + logf(e);
+    const int t = ri.z + r / p.G;
+    const int h = kvh * p.G + r % p.G;
+    for (int d = lane * 4; d < p.D; d += 128) {
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      if (L != -INFINITY) {
+        for (int s = 0; s < ns; ++s) {
+          const float ls = p.part_lse[base + (size_t)s * kBM];
+          if (ls == -INFINITY) continue;
+          const float wgt = expf(ls - L);
+          const float4 o = *reinterpret_cast<const float4*>(p.part_o + (base + (size_t)s * kBM) * p.D + d);
+          a0 = fmaf(wgt, o.x, a0);
+          a1 = fmaf(wgt, o.y, a1);
+          a2 = fmaf(wgt, o.z, a2);
+          a3 = fmaf(wgt, o.w, a3);
+        }
+      }
+      uint2 pk;
+      pk.x = pack_bf16x2(a0, a1);
+      pk.y = pack_bf16x2(a2, a3);
+      *reinterpret_cast<uint2*>(p.out + ((size_t)t * p.Hq + h) * p.D + d) = pk;
+    }
+    if (lane == 0 && p.lse) p.lse[(size_t)t * p.Hq + h] = L;
+  }
+}
+
+}  // namespace pa

@@ -1,0 +1,253 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the fp64 CPU
+oracle on the same seeded inputs.  Bar: max |O - oracle| <= 1e-2 on bf16
+outputs and max |LSE - oracle| <= 1e-3 on the fp32 LSE (N(0,1) inputs)."""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_gqa_fmha_b200 import workloads as W
+from tests.gpu_common import (compare, gpu_run, make_plan, oracle_all, oracle_rows,
+                              sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def gen(spec, seed):
+    return W.generate(spec, seed, device="cuda")
+
+
+# ------------------------------------------------------------------ tiny decode (config 1)
+def test_tiny_decode_matches_oracle_and_golden():
+    w = gen(W.CONFIGS["tiny_decode"], W.default_seed("tiny_decode"))
+    # the golden fixture was drawn on the CPU generator: regenerate values there
+    wc = W.generate(W.CONFIGS["tiny_decode"], W.default_seed("tiny_decode"))
+    for key in ("q", "k_pool", "v_pool"):
+        w[key] = wc[key].cuda()
+    out, lse, _ = gpu_run(w, use_cu=False)
+    o_ref, l_ref = oracle_all(w)
+    compare(out, lse, o_ref, l_ref)
+    import os
+    g = np.array([float(x) for x in open(os.path.join(os.path.dirname(__file__), "golden",
+                                                      "tiny_decode.txt"))
+                  if not x.startswith("#")])
+    assert np.max(np.abs(lse.cpu().numpy().reshape(-1) - g[:8])) <= 1e-3
+    assert np.max(np.abs(out.float().cpu().numpy().reshape(-1) - g[8:])) <= 1e-2
+
+
+# ------------------------------------------------------------------ small geometries, all rows
+GEOMS = [  # (D, ps, G, Hkv, prefill)
+    (128, 16, 4, 2, False), (128, 16, 4, 2, True), (64, 16, 2, 2, True), (64, 64, 8, 1, False),
+    (256, 128, 32, 1, False), (256, 32, 2, 2, True), (128, 64, 1, 3, True), (128, 128, 16, 2, True),
+    (64, 32, 32, 1, True), (256, 16, 8, 1, True), (128, 32, 3, 2, True), (128, 16, 6, 1, False),
+]
+
+
+@pytest.mark.parametrize("D,ps,G,Hkv,prefill", GEOMS)
+def test_small_geometry_all_rows(D, ps, G, Hkv, prefill):
+    rng = np.random.default_rng(D * 7 + ps * 3 + G + Hkv + int(prefill))
+    spec = W.random_small(rng, D=D, ps=ps, G=G, Hkv=Hkv, B=int(rng.integers(1, 6)),
+                          max_kv=700, prefill=prefill)
+    w = gen(spec, 500 + D + ps + G)
+    out, lse, _ = gpu_run(w)
+    compare(out, lse, *oracle_all(w))
+
+
+def test_prefill_many_tiles_ragged():
+    """Several 128-row query blocks and KV tiles, with a ragged tail and chunked
+    prefill (kv > q)."""
+    spec = W.custom_spec("ragged", 32, 8, 128, 16, [300, 1, 77, 129], [300, 901, 500, 129])
+    w = gen(spec, 11)
+    out, lse, _ = gpu_run(w)
+    compare(out, lse, *oracle_all(w))
+
+
+def test_decode_without_cu_q_lens():
+    spec = W.custom_spec("dec", 32, 8, 128, 16, [1] * 9, [1, 15, 16, 17, 127, 128, 129, 600, 2048])
+    w = gen(spec, 12)
+    out, lse, _ = gpu_run(w, use_cu=False)
+    compare(out, lse, *oracle_all(w))
+
+
+# ------------------------------------------------------------------ split-KV (a8)
+@pytest.mark.parametrize("splits", [1, 2, 7, 0])
+def test_split_invariance(splits):
+    spec = W.custom_spec("split", 16, 2, 128, 32, [1, 1, 3, 1], [3000, 1200, 2500, 64])
+    w = gen(spec, 13)
+    plan = make_plan(w, num_splits=splits)
+    out, lse, _ = gpu_run(w, plan)
+    compare(out, lse, *oracle_all(w))
+    ref_plan = make_plan(w, num_splits=1)
+    out1, lse1, _ = gpu_run(w, ref_plan)
+    assert torch.max(torch.abs(out.float() - out1.float())).item() <= 1e-2
+    assert torch.max(torch.abs(lse - lse1)).item() <= 1e-3
+
+
+def test_split_long_gqa32_head_dim_256():
+    spec = W.custom_spec("split256", 64, 2, 256, 128, [1, 1], [20000, 7000])
+    w = gen(spec, 14)
+    for splits in (0, 5):
+        out, lse, _ = gpu_run(w, make_plan(w, num_splits=splits))
+        compare(out, lse, *oracle_all(w))
+
+
+# ------------------------------------------------------------------ invariants on the GPU path
+def test_page_permutation_invariance_gpu():
+    spec = W.custom_spec("perm", 16, 4, 64, 16, [1, 40, 1], [500, 300, 77])
+    w = gen(spec, 15)
+    out1, lse1, _ = gpu_run(w)
+    perm = torch.randperm(w["P"], generator=torch.Generator().manual_seed(3)).cuda()
+    k2 = torch.empty_like(w["k_pool"])
+    v2 = torch.empty_like(w["v_pool"])
+    k2[perm] = w["k_pool"]
+    v2[perm] = w["v_pool"]
+    t = w["page_table"].long()
+    t2 = torch.where(t >= 0, perm[t.clamp(min=0)], t).to(torch.int32)
+    out2, lse2, _ = gpu_run(w, k_pool=k2, v_pool=v2, page_table=t2)
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
+
+
+@pytest.mark.parametrize("fill", [-1, 2**31 - 1])
+def test_poisoned_tails_and_columns_gpu(fill):
+    """NaN in tail slots of the last live page and in every unused page; table
+    columns past the live pages set to -1 or INT32_MAX: output unchanged and
+    finite (pages never read, V tail sanitised)."""
+    spec = W.custom_spec("poison", 16, 2, 128, 16, [1, 20, 1, 5], [37, 100, 64, 5])
+    w = gen(spec, 16)
+    out1, lse1, _ = gpu_run(w)
+    k, v = w["k_pool"].clone(), w["v_pool"].clone()
+    table = w["page_table"].clone()
+    seq = w["seq_lens_cpu"].tolist()
+    live = set()
+    for b, kv in enumerate(seq):
+        n = -(-kv // 16)
+        pages = w["page_table_cpu"][b, :n].tolist()
+        live.update(pages)
+        tail = kv - (n - 1) * 16
+        k[pages[-1], tail:] = float("nan")
+        v[pages[-1], tail:] = float("nan")
+        table[b, n:] = fill
+    for p in range(w["P"]):
+        if p not in live:
+            k[p] = float("nan")
+            v[p] = float("nan")
+    plan = make_plan(w, num_pages=0)
+    out2, lse2, _ = gpu_run(w, plan, k_pool=k, v_pool=v, page_table=table)
+    assert torch.isfinite(out2.float()).all() and torch.isfinite(lse2).all()
+    assert torch.max(torch.abs(out1.float() - out2.float())).item() == 0.0
+    assert torch.max(torch.abs(lse1 - lse2)).item() == 0.0
+
+
+def test_metadata_mutation_between_runs_same_plan():
+    """One plan, new request metadata bound on every run."""
+    spec = W.custom_spec("mut", 16, 2, 128, 32, [1, 7, 1], [900, 400, 33])
+    w = gen(spec, 17)
+    plan = make_plan(w)
+    out, lse, _ = gpu_run(w, plan)
+    compare(out, lse, *oracle_all(w))
+    seq2 = torch.tensor([513, 7, 1], dtype=torch.int32)
+    w2 = dict(w)
+    w2["seq_lens"] = seq2.cuda()
+    w2["seq_lens_cpu"] = seq2
+    out2, lse2, _ = gpu_run(w2, plan)
+    compare(out2, lse2, *oracle_all(w2))
+
+
+def test_cuda_graph_replay_with_new_seq_lens():
+    spec = W.custom_spec("graph", 32, 8, 128, 16, [1] * 6, [100, 2000, 37, 64, 1500, 999])
+    w = gen(spec, 18)
+    plan = make_plan(w)
+    seq = w["seq_lens"].clone()
+    out = torch.empty_like(w["q"])
+    lse = torch.empty(w["T"], w["Hq"], device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        plan.run(w["q"], w["k_pool"], w["v_pool"], w["page_table"], seq, None, out=out, lse=lse)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        plan.run(w["q"], w["k_pool"], w["v_pool"], w["page_table"], seq, None, out=out, lse=lse)
+    for new in ([100, 2000, 37, 64, 1500, 999], [1, 1999, 38, 17, 1024, 1000]):
+        seq.copy_(torch.tensor(new, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        w2 = dict(w)
+        w2["seq_lens_cpu"] = torch.tensor(new, dtype=torch.int32)
+        w2["cu_q_lens_cpu"] = torch.arange(7, dtype=torch.int32)
+        compare(out, lse, *oracle_all(w2))
+
+
+def test_status_bits_for_bad_requests():
+    spec = W.custom_spec("bad", 8, 2, 64, 16, [1, 1], [40, 30])
+    w = gen(spec, 19)
+    plan = make_plan(w)
+    assert plan.status() == 0
+    gpu_run(w, plan)
+    assert plan.status() == 0
+    table = w["page_table"].clone()
+    table[0, 1] = w["P"] + 5                       # live column out of the pool
+    gpu_run(w, plan, page_table=table)
+    assert plan.status() & 1
+    seq = torch.tensor([40, 10**6], dtype=torch.int32, device="cuda")
+    gpu_run(w, plan, seq_lens=seq)
+    assert plan.status() & 4
+
+
+def test_rows_without_visible_keys_get_zero_and_minus_inf():
+    """q_b > kv_b (invalid): the first q_b - kv_b rows see no key."""
+    spec = W.custom_spec("qgt", 8, 2, 64, 16, [6, 3], [4, 40])
+    w = gen(spec, 20)
+    plan = make_plan(w)
+    out, lse, _ = gpu_run(w, plan)
+    assert plan.status() & 2
+    compare(out, lse, *oracle_all(w))
+
+
+def test_empty_requests():
+    spec = W.custom_spec("empty", 8, 2, 128, 16, [0, 5, 0, 1], [0, 5, 17, 1])
+    w = gen(spec, 21)
+    out, lse, _ = gpu_run(w)
+    compare(out, lse, *oracle_all(w))
+
+
+def test_zero_query_closed_form_gpu():
+    """q = 0: O is the mean of the visible V rows, LSE = ln(#visible keys)."""
+    spec = W.custom_spec("q0", 16, 4, 128, 16, [50, 1], [300, 200])
+    w = gen(spec, 22)
+    w["q"] = torch.zeros_like(w["q"])
+    out, lse, _ = gpu_run(w)
+    compare(out, lse, *oracle_all(w))
+    cu = w["cu_q_lens_cpu"]
+    n = np.array([300 - 50 + i + 1 for i in range(50)] + [200], dtype=np.float64)
+    assert np.max(np.abs(lse.cpu().numpy()[:, 0] - np.log(n))) < 1e-4
+
+
+def test_large_logits_gpu():
+    """q x 30: a very peaked softmax must neither overflow nor lose accuracy
+    beyond what bf16 allows.  With P rounded to bf16 (relative error <= 2^-9
+    per weight) and O rounded to bf16 (<= 2^-9 |O|), |O - O_ref| is bounded by
+    2^-8 max|V|; N(0,1) inputs with moderate logits stay far below that, but a
+    one-hot softmax reaches it."""
+    spec = W.custom_spec("big", 16, 4, 128, 32, [64, 1], [700, 900])
+    w = gen(spec, 23)
+    w["q"] = (w["q"].float() * 30.0).to(torch.bfloat16)
+    out, lse, _ = gpu_run(w)
+    o_ref, l_ref = oracle_all(w)
+    vmax = float(w["v_pool"].float().abs().max())
+    compare(out, lse, o_ref, l_ref, tol_o=2.0 ** -8 * vmax,
+            tol_l=1e-3 * max(1.0, float(np.max(np.abs(l_ref)))))
+
+
+# ------------------------------------------------------------------ full-size configs, sampled rows
+@pytest.mark.parametrize("name", ["llama8b_decode", "llama8b_causal_prefill", "unified_mixed",
+                                  "long_gqa32_decode"])
+def test_full_size_config_sampled_rows(name):
+    w = gen(W.CONFIGS[name], W.default_seed(name))
+    plan = make_plan(w)
+    out, lse, _ = gpu_run(w, plan, use_cu=not W.CONFIGS[name].decode_only)
+    assert plan.status() == 0
+    assert torch.isfinite(out.float()).all()
+    rt, rh = sample_rows(w, 48, seed=1)
+    o_ref, l_ref = oracle_rows(w, rt, rh)
+    o = out[torch.from_numpy(rt).long().cuda(), torch.from_numpy(rh).long().cuda()]
+    l = lse[torch.from_numpy(rt).long().cuda(), torch.from_numpy(rh).long().cuda()]
+    compare(o, l, o_ref, l_ref)
