@@ -168,6 +168,16 @@ PA_API size_t pa_workspace_bytes(const pa_plan *plan);
 /* Largest number of KV splits this plan can use for one request. */
 PA_API int pa_max_splits(const pa_plan *plan);
 
+/* Kernel timing for benchmarks.  pa_profile_start makes the next `max_runs`
+ * (1..4096) calls of pa_run record a CUDA event pair on their stream around
+ * the attention kernel.  pa_profile_read synchronises on those events, writes
+ * the summed attention-kernel time in milliseconds, the number of runs
+ * recorded and the number of kernels each pa_run launches, and turns the
+ * recording off.  While recording, pa_run must not be captured in a graph.
+ * The events are owned by the plan. */
+PA_API int pa_profile_start(pa_plan *plan, int max_runs);
+PA_API int pa_profile_read(pa_plan *plan, float *attn_ms, int *n_runs, int *launches_per_run);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,7 @@ STATUS_TIMEOUT = 1 << 4
 
 EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_scale",
            "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
-           "pa_max_splits")
+           "pa_max_splits", "pa_profile_start", "pa_profile_read")
 
 _lib = None
 
@@ -67,6 +67,10 @@ def load_library(path: str = LIB_PATH):
     lib.pa_workspace_bytes.restype = ctypes.c_size_t
     lib.pa_max_splits.argtypes = [P]
     lib.pa_max_splits.restype = I
+    lib.pa_profile_start.argtypes = [P, I]
+    lib.pa_profile_start.restype = I
+    lib.pa_profile_read.argtypes = [P, ctypes.POINTER(F), ctypes.POINTER(I), ctypes.POINTER(I)]
+    lib.pa_profile_read.restype = I
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -168,6 +172,17 @@ class Plan:
                                 _ptr(seq_lens), _ptr(cu_q_lens), _ptr(out), _ptr(lse),
                                 ctypes.c_void_p(stream)))
         return out, lse
+
+    def profile_start(self, max_runs: int):
+        """Record the attention kernel's duration in the next ``max_runs`` runs."""
+        _check(self._lib.pa_profile_start(self._h, int(max_runs)))
+
+    def profile_read(self):
+        """Returns (summed attention-kernel ms, runs recorded, kernels per run)."""
+        ms, n, k = ctypes.c_float(0), ctypes.c_int(0), ctypes.c_int(0)
+        _check(self._lib.pa_profile_read(self._h, ctypes.byref(ms), ctypes.byref(n),
+                                         ctypes.byref(k)))
+        return float(ms.value), int(n.value), int(k.value)
 
     def status(self, clear: bool = True, stream=None) -> int:
         """Synchronise and read (then clear) the sticky device status word."""

@@ -66,6 +66,9 @@ struct pa_plan {
   pa::WorkItem* items;
   float* part_lse;
   float* part_o;
+  // attention-kernel timing (pa_profile_*)
+  cudaEvent_t* prof_ev;
+  int prof_cap, prof_n, prof_on;
   // tensor-map cache
   const void* tm_ptr[3];
   int tm_num_pages;
@@ -259,6 +262,8 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->box_h = page_size < p->BN ? page_size : p->BN;
   p->S_max = auto_smax(batch, heads_kv, n_sm);
   p->ws = nullptr;
+  p->prof_ev = nullptr;
+  p->prof_cap = p->prof_n = p->prof_on = 0;
   p->tm_ptr[0] = p->tm_ptr[1] = p->tm_ptr[2] = nullptr;
   p->tm_num_pages = -1;
   if (alloc_workspace(p) != PA_OK) {
@@ -268,8 +273,18 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   return p;
 }
 
+static void free_profile_events(pa_plan* p) {
+  if (p->prof_ev) {
+    for (int i = 0; i < 2 * p->prof_cap; ++i) cudaEventDestroy(p->prof_ev[i]);
+    delete[] p->prof_ev;
+  }
+  p->prof_ev = nullptr;
+  p->prof_cap = p->prof_n = p->prof_on = 0;
+}
+
 void pa_destroy(pa_plan* p) {
   if (!p) return;
+  free_profile_events(p);
   if (p->ws) cudaFree(p->ws);
   delete p;
 }
@@ -382,6 +397,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.box_h = p->box_h;
   ap.scale_log2 = p->scale * 1.4426950408889634f;
   const dim3 grid(p->n_sm), block(pa::kThreads);
+  const bool prof = p->prof_on && p->prof_n < p->prof_cap;
+  if (prof) cudaEventRecord(p->prof_ev[2 * p->prof_n], st);
   switch (p->D) {
     case 64:
       pa::pa_attention_kernel<64><<<grid, block, pa::TileCfg<64>::SMEM_BYTES, st>>>(p->tm_q, p->tm_k, p->tm_v, ap);
@@ -392,6 +409,10 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     default:
       pa::pa_attention_kernel<256><<<grid, block, pa::TileCfg<256>::SMEM_BYTES, st>>>(p->tm_q, p->tm_k, p->tm_v, ap);
       break;
+  }
+  if (prof) {
+    cudaEventRecord(p->prof_ev[2 * p->prof_n + 1], st);
+    ++p->prof_n;
   }
   if (sp.S_max > 1) {
     pa::MergeParams mp;
@@ -408,6 +429,53 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     set_err("pa_run: launch failed: %s", cudaGetErrorString(e));
     return PA_ERR_CUDA;
   }
+  return PA_OK;
+}
+
+int pa_profile_start(pa_plan* p, int max_runs) {
+  if (!p) { set_err("pa_profile_start: NULL plan"); return PA_ERR_INVALID; }
+  if (max_runs < 1 || max_runs > 4096) {
+    set_err("pa_profile_start: max_runs %d outside [1, 4096]", max_runs);
+    return PA_ERR_INVALID;
+  }
+  if (p->prof_cap < max_runs) {
+    free_profile_events(p);
+    p->prof_ev = new cudaEvent_t[2 * max_runs];
+    for (int i = 0; i < 2 * max_runs; ++i) {
+      cudaError_t e = cudaEventCreate(&p->prof_ev[i]);
+      if (e != cudaSuccess) {
+        for (int k = 0; k < i; ++k) cudaEventDestroy(p->prof_ev[k]);
+        delete[] p->prof_ev;
+        p->prof_ev = nullptr;
+        set_err("pa_profile_start: cudaEventCreate failed: %s", cudaGetErrorString(e));
+        return PA_ERR_CUDA;
+      }
+    }
+    p->prof_cap = max_runs;
+  }
+  p->prof_n = 0;
+  p->prof_on = 1;
+  return PA_OK;
+}
+
+int pa_profile_read(pa_plan* p, float* attn_ms, int* n_runs, int* launches_per_run) {
+  if (!p || !attn_ms || !n_runs) { set_err("pa_profile_read: NULL argument"); return PA_ERR_INVALID; }
+  float total = 0.f;
+  for (int i = 0; i < p->prof_n; ++i) {
+    cudaError_t e = cudaEventSynchronize(p->prof_ev[2 * i + 1]);
+    float ms = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, p->prof_ev[2 * i], p->prof_ev[2 * i + 1]);
+    if (e != cudaSuccess) {
+      set_err("pa_profile_read: %s", cudaGetErrorString(e));
+      return PA_ERR_CUDA;
+    }
+    total += ms;
+  }
+  *attn_ms = total;
+  *n_runs = p->prof_n;
+  if (launches_per_run) *launches_per_run = (p->num_splits != 1 && p->S_max > 1) ? 3 : 2;
+  p->prof_on = 0;
+  p->prof_n = 0;
   return PA_OK;
 }
 
