@@ -178,6 +178,51 @@ PA_API int pa_max_splits(const pa_plan *plan);
 PA_API int pa_profile_start(pa_plan *plan, int max_runs);
 PA_API int pa_profile_read(pa_plan *plan, float *attn_ms, int *n_runs, int *launches_per_run);
 
+/*
+ * pa_run_noalloc -- the same attention pass as pa_run, for callers that cannot
+ * allocate device memory.  (The source pages have no counterpart: this entry
+ * point exists for integration, not for the method.)
+ *
+ * Some callers cannot call cudaMalloc at the point where they run attention:
+ * a region being captured into a CUDA graph in global capture mode (device
+ * allocation is not allowed there), an engine whose device memory is fully
+ * budgeted by its own allocator (a raw cudaMalloc would bypass its accounting
+ * and can fail late), or a loop where a synchronous allocation would stall
+ * the device.  pa_create_plan allocates a workspace, so such callers use this
+ * entry point instead: no plan, no cudaMalloc, no cudaFree, no allocating
+ * library routine.  The caller still passes every input and output.
+ *
+ * Scratch: the work list and the status word live in one file-scope device
+ * array of PA_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU which loads the
+ * library holds until the process exits.  A geometry whose worst-case work
+ * list does not fit (batch * heads_kv * ceil(capacity * page_size * G / 128)
+ * items of 48 bytes, plus 16 bytes per request and a 256-byte header) is
+ * rejected with PA_ERR_UNSUPPORTED and a message saying so.  KV splitting is
+ * not used on this path (each (request, KV head, query block) is one item),
+ * so there is no split merge and no partial-state storage.
+ *
+ * All calls share the array and it keeps the last call's contents; each call
+ * clears the header it relies on (status word, item count) on `stream` before
+ * its kernels run.  Calls whose work overlaps on the GPU (different streams,
+ * or several threads) race on the array and must be serialised by the caller.
+ *
+ * The first call on a device performs a one-time set-up on that device (it
+ * resolves the array's device address with cudaGetSymbolAddress and sets the
+ * kernel's shared-memory limit); make that first call before any stream
+ * capture.  Later calls only enqueue work.
+ *
+ * Arguments are those of pa_create_plan followed by those of pa_run, plus
+ *   num_pages  pool size P for page-id checks (0 = trust the table)
+ *   scale      softmax scale (> 0), or 0 for 1/sqrt(head_dim)
+ * Returns PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED or PA_ERR_CUDA.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (8u << 20)
+PA_API int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_size,
+                          int capacity, int num_pages, float scale, const void *q,
+                          const void *k_pool, const void *v_pool, const int32_t *page_table,
+                          const int32_t *seq_lens, const int32_t *cu_q_lens, void *out,
+                          float *lse, pa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,10 @@ STATUS_TIMEOUT = 1 << 4
 
 EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_scale",
            "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
-           "pa_max_splits", "pa_profile_start", "pa_profile_read")
+           "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc")
+
+# Size of the library's static scratch array used by pa_run_noalloc.
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _lib = None
 
@@ -71,6 +74,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_profile_start.restype = I
     lib.pa_profile_read.argtypes = [P, ctypes.POINTER(F), ctypes.POINTER(I), ctypes.POINTER(I)]
     lib.pa_profile_read.restype = I
+    lib.pa_run_noalloc.argtypes = [I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P]
+    lib.pa_run_noalloc.restype = I
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -203,3 +208,24 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def run_noalloc(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, out, lse, *, heads_kv,
+                page_size, capacity, num_pages=0, scale=0.0, stream=None):
+    """Call ``pa_run_noalloc``: the attention pass for callers that cannot
+    allocate device memory (the library's static scratch array replaces the
+    plan's workspace).  Every output tensor is passed in; nothing is allocated
+    here or in the library.  The first call on a device does a one-time set-up
+    there, so make it before any stream capture.  Calls that overlap on the GPU
+    race on the shared scratch."""
+    lib = load_library()
+    B = seq_lens.shape[0]
+    Hq, D = q.shape[1], q.shape[2]
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    elif isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    _check(lib.pa_run_noalloc(B, Hq, heads_kv, D, page_size, capacity, int(num_pages),
+                              float(scale), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                              _ptr(page_table), _ptr(seq_lens), _ptr(cu_q_lens), _ptr(out),
+                              _ptr(lse), ctypes.c_void_p(stream)))

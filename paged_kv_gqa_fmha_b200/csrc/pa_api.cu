@@ -12,6 +12,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
+#include <mutex>
 
 #include "../../include/pa.h"
 #include "pa_kernels.cuh"
@@ -476,6 +478,213 @@ int pa_profile_read(pa_plan* p, float* attn_ms, int* n_runs, int* launches_per_r
   if (launches_per_run) *launches_per_run = (p->num_splits != 1 && p->S_max > 1) ? 3 : 2;
   p->prof_on = 0;
   p->prof_n = 0;
+  return PA_OK;
+}
+
+
+// ---------------------------------------------------------------------------
+// pa_run_noalloc: the attention pass without any device allocation, for
+// callers that cannot call cudaMalloc (see include/pa.h).  Its scratch is the
+// file-scope array below.  Host code must not use the array's name as a
+// device address (it is a host-side stand-in): the device address comes from
+// cudaGetSymbolAddress, resolved once per device with that device current.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+struct NoallocDevice {
+  std::atomic<int> ready{0};
+  void* scratch = nullptr;
+  int n_sm = 0;
+};
+constexpr int kMaxDevices = 64;
+NoallocDevice g_noalloc_dev[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// One-time set-up of the current device; returns PA_OK or an error code.
+int noalloc_setup(int dev, NoallocDevice** out) {
+  if (dev < 0 || dev >= kMaxDevices) {
+    set_err("pa_run_noalloc: device %d out of range", dev);
+    return PA_ERR_INVALID;
+  }
+  NoallocDevice& d = g_noalloc_dev[dev];
+  if (!d.ready.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!d.ready.load(std::memory_order_relaxed)) {
+      int major = 0, n_sm = 0;
+      cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) {
+        set_err("pa_run_noalloc: device query failed: %s", cudaGetErrorString(e));
+        return PA_ERR_CUDA;
+      }
+      if (major != 10) {
+        set_err("pa_run_noalloc: device %d is not sm_100", dev);
+        return PA_ERR_UNSUPPORTED;
+      }
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+      if (e != cudaSuccess || ptr == nullptr) {
+        set_err("pa_run_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+        return PA_ERR_CUDA;
+      }
+      e = set_smem_attr<64>();
+      if (e == cudaSuccess) e = set_smem_attr<128>();
+      if (e == cudaSuccess) e = set_smem_attr<256>();
+      if (e != cudaSuccess) {
+        set_err("pa_run_noalloc: cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
+        return PA_ERR_CUDA;
+      }
+      d.scratch = ptr;
+      d.n_sm = n_sm;
+      d.ready.store(1, std::memory_order_release);
+    }
+  }
+  *out = &d;
+  return PA_OK;
+}
+
+}  // namespace
+
+int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_size,
+                   int capacity, int num_pages, float scale, const void* q, const void* k_pool,
+                   const void* v_pool, const int32_t* page_table, const int32_t* seq_lens,
+                   const int32_t* cu_q_lens, void* out, float* lse, pa_stream_t stream) {
+  g_err[0] = 0;
+  // geometry: the same envelope as pa_create_plan
+  if (batch <= 0 || heads_q <= 0 || heads_kv <= 0 || head_dim <= 0 || page_size <= 0 ||
+      capacity <= 0 || num_pages < 0) {
+    set_err("pa_run_noalloc: batch, heads, head_dim, page_size and capacity must be > 0 "
+            "and num_pages >= 0");
+    return PA_ERR_INVALID;
+  }
+  if ((head_dim != 64 && head_dim != 128 && head_dim != 256) ||
+      (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128) ||
+      heads_q % heads_kv != 0 || heads_q / heads_kv > 32) {
+    set_err("pa_run_noalloc: unsupported geometry (head_dim %d, page_size %d, heads %d/%d)",
+            head_dim, page_size, heads_q, heads_kv);
+    return PA_ERR_UNSUPPORTED;
+  }
+  if (!(scale >= 0.f) || !std::isfinite(scale)) {
+    set_err("pa_run_noalloc: scale must be finite and >= 0 (0 = 1/sqrt(head_dim))");
+    return PA_ERR_INVALID;
+  }
+  const int G = heads_q / heads_kv;
+  const int tpb = pa::kBM / G;
+  const int BN = kv_tile(head_dim);
+  const long blocks_per_req = ((long)capacity * page_size + tpb - 1) / tpb;
+  const long max_items = (long)batch * heads_kv * blocks_per_req;
+  const size_t o_req = align_up(sizeof(pa::WsHeader), 256);
+  const size_t o_items = align_up(o_req + sizeof(int4) * (size_t)batch, 256);
+  const size_t need = o_items + sizeof(pa::WorkItem) * (size_t)max_items;
+  if (max_items > (1L << 30) || need > (size_t)PA_NOALLOC_SCRATCH_BYTES) {
+    set_err("pa_run_noalloc: this geometry needs %zu bytes of scratch (%ld work items); the "
+            "static scratch holds %u bytes -- use pa_create_plan / pa_run instead",
+            need, max_items, (unsigned)PA_NOALLOC_SCRATCH_BYTES);
+    return PA_ERR_UNSUPPORTED;
+  }
+  if (!q || !k_pool || !v_pool || !page_table || !seq_lens || !out) {
+    set_err("pa_run_noalloc: NULL pointer (q, k_pool, v_pool, page_table, seq_lens and out "
+            "are required)");
+    return PA_ERR_INVALID;
+  }
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) ||
+      !aligned16(page_table) || !aligned16(seq_lens) || (cu_q_lens && !aligned16(cu_q_lens)) ||
+      (lse && !aligned16(lse))) {
+    set_err("pa_run_noalloc: every pointer must be 16-byte aligned");
+    return PA_ERR_INVALID;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_err("pa_run_noalloc: no current CUDA device");
+    return PA_ERR_CUDA;
+  }
+  NoallocDevice* nd = nullptr;
+  int rc = noalloc_setup(dev, &nd);
+  if (rc) return rc;
+
+  // tensor maps for this call, on the host stack
+  const int box_h = page_size < BN ? page_size : BN;
+  CUtensorMap tm_q, tm_k, tm_v;
+  {
+    const cuuint64_t e = 2;
+    cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)heads_q,
+                          (cuuint64_t)batch * capacity * page_size};
+    cuuint64_t str[2] = {(cuuint64_t)head_dim * e, (cuuint64_t)heads_q * head_dim * e};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)tpb};
+    rc = encode(&tm_q, q, 3, dims, str, box, "q");
+    if (rc) return rc;
+    cuuint64_t P = num_pages > 0 ? (cuuint64_t)num_pages : (cuuint64_t)0x7fffffff;
+    cuuint64_t kd[4] = {(cuuint64_t)head_dim, (cuuint64_t)heads_kv, (cuuint64_t)page_size, P};
+    cuuint64_t ks[3] = {(cuuint64_t)head_dim * e, (cuuint64_t)heads_kv * head_dim * e,
+                        (cuuint64_t)page_size * heads_kv * head_dim * e};
+    cuuint32_t kb[4] = {64, 1, (cuuint32_t)box_h, 1};
+    rc = encode(&tm_k, k_pool, 4, kd, ks, kb, "k_pool");
+    if (rc) return rc;
+    rc = encode(&tm_v, v_pool, 4, kd, ks, kb, "v_pool");
+    if (rc) return rc;
+  }
+
+  char* base = static_cast<char*>(nd->scratch);
+  pa::WsHeader* hdr = reinterpret_cast<pa::WsHeader*>(base);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the previous call's header must not leak into this one
+  cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(pa::WsHeader), st);
+  if (e != cudaSuccess) {
+    set_err("pa_run_noalloc: cudaMemsetAsync failed: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+
+  pa::SchedParams sp;
+  sp.seq_lens = seq_lens;
+  sp.cu_q_lens = cu_q_lens;
+  sp.items = reinterpret_cast<pa::WorkItem*>(base + o_items);
+  sp.req_info = reinterpret_cast<int4*>(base + o_req);
+  sp.hdr = hdr;
+  sp.max_items = (int)max_items;
+  sp.B = batch; sp.Hkv = heads_kv; sp.G = G; sp.C = capacity; sp.ps = page_size; sp.BN = BN;
+  sp.tpb = tpb;
+  sp.S_max = 1;             // no KV splits on this path
+  sp.forced_splits = 0;
+  sp.n_ctas = nd->n_sm;
+  pa::pa_schedule_kernel<<<1, pa::kCostBuckets, 0, st>>>(sp);
+
+  pa::AttnParams ap;
+  ap.q = static_cast<const uint16_t*>(q);
+  ap.page_table = page_table;
+  ap.cu_q_lens = cu_q_lens;
+  ap.out = static_cast<uint16_t*>(out);
+  ap.lse = lse;
+  ap.items = sp.items;
+  ap.hdr = hdr;
+  ap.part_o = nullptr;
+  ap.part_lse = nullptr;
+  ap.status = &hdr->status;
+  ap.B = batch; ap.Hq = heads_q; ap.Hkv = heads_kv; ap.G = G; ap.C = capacity; ap.ps = page_size;
+  ap.num_pages = num_pages;
+  ap.S_max = 1;
+  ap.tpb = tpb;
+  ap.box_h = box_h;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)head_dim);
+  ap.scale_log2 = sc * 1.4426950408889634f;
+  const dim3 grid(nd->n_sm), block(pa::kThreads);
+  switch (head_dim) {
+    case 64:
+      pa::pa_attention_kernel<64><<<grid, block, pa::TileCfg<64>::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, ap);
+      break;
+    case 128:
+      pa::pa_attention_kernel<128><<<grid, block, pa::TileCfg<128>::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, ap);
+      break;
+    default:
+      pa::pa_attention_kernel<256><<<grid, block, pa::TileCfg<256>::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, ap);
+      break;
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_err("pa_run_noalloc: launch failed: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
   return PA_OK;
 }
 
