@@ -196,7 +196,7 @@ PA_API int pa_profile_read(pa_plan *plan, float *attn_ms, int *n_runs, int *laun
  * array of PA_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU which loads the
  * library holds until the process exits.  A geometry whose worst-case work
  * list does not fit (batch * heads_kv * ceil(capacity * page_size * G / 128)
- * items of 48 bytes, plus 16 bytes per request and a 256-byte header) is
+ * items of 32 bytes, plus 40 bytes per request and a small header) is
  * rejected with PA_ERR_UNSUPPORTED and a message saying so.  KV splitting is
  * not used on this path (each (request, KV head, query block) is one item),
  * so there is no split merge and no partial-state storage.

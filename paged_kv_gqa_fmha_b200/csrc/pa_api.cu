@@ -65,7 +65,10 @@ struct pa_plan {
   size_t ws_bytes;
   pa::WsHeader* hdr;
   int4* req_info;
-  pa::WorkItem* items;
+  int4* req_aux;
+  int* unit_off;
+  int* split_list;
+  pa::PackedItem* items;
   float* part_lse;
   float* part_o;
   // attention-kernel timing (pa_profile_*)
@@ -105,7 +108,10 @@ int alloc_workspace(pa_plan* p) {
   size_t off = 0;
   const size_t o_hdr = off; off = align_up(off + sizeof(pa::WsHeader), 256);
   const size_t o_req = off; off = align_up(off + sizeof(int4) * (size_t)p->B, 256);
-  const size_t o_items = off; off = align_up(off + sizeof(pa::WorkItem) * (size_t)max_items, 256);
+  const size_t o_aux = off; off = align_up(off + sizeof(int4) * (size_t)p->B, 256);
+  const size_t o_uoff = off; off = align_up(off + sizeof(int) * (size_t)(p->B + 1), 256);
+  const size_t o_split = off; off = align_up(off + sizeof(int) * (size_t)p->B, 256);
+  const size_t o_items = off; off = align_up(off + sizeof(pa::PackedItem) * (size_t)max_items, 256);
   const size_t o_plse = off; off = align_up(off + sizeof(float) * n_part_rows, 256);
   const size_t o_po = off; off = align_up(off + sizeof(float) * n_part_rows * p->D, 256);
   void* ws = nullptr;
@@ -126,7 +132,10 @@ int alloc_workspace(pa_plan* p) {
   char* c = static_cast<char*>(ws);
   p->hdr = reinterpret_cast<pa::WsHeader*>(c + o_hdr);
   p->req_info = reinterpret_cast<int4*>(c + o_req);
-  p->items = reinterpret_cast<pa::WorkItem*>(c + o_items);
+  p->req_aux = reinterpret_cast<int4*>(c + o_aux);
+  p->unit_off = reinterpret_cast<int*>(c + o_uoff);
+  p->split_list = reinterpret_cast<int*>(c + o_split);
+  p->items = reinterpret_cast<pa::PackedItem*>(c + o_items);
   p->part_lse = reinterpret_cast<float*>(c + o_plse);
   p->part_o = reinterpret_cast<float*>(c + o_po);
   p->max_items = (int)max_items;
@@ -138,6 +147,50 @@ cudaError_t set_smem_attr() {
   return cudaFuncSetAttribute(pa::pa_attention_kernel<D>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               pa::TileCfg<D>::SMEM_BYTES);
+}
+
+// The attention kernel and the merge are programmatic dependents of the
+// kernel launched before them on the stream (their prologues overlap it; each
+// waits with griddepcontrol.wait before reading its results).
+template <int D>
+cudaError_t launch_attention(int n_sm, cudaStream_t st, const CUtensorMap& tq,
+                             const CUtensorMap& tk, const CUtensorMap& tv,
+                             const pa::AttnParams& ap) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_sm);
+  cfg.blockDim = dim3(pa::kThreads);
+  cfg.dynamicSmemBytes = pa::TileCfg<D>::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pa::pa_attention_kernel<D>, tq, tk, tv, ap);
+}
+
+cudaError_t launch_attention_d(int D, int n_sm, cudaStream_t st, const CUtensorMap& tq,
+                               const CUtensorMap& tk, const CUtensorMap& tv,
+                               const pa::AttnParams& ap) {
+  switch (D) {
+    case 64: return launch_attention<64>(n_sm, st, tq, tk, tv, ap);
+    case 128: return launch_attention<128>(n_sm, st, tq, tk, tv, ap);
+    default: return launch_attention<256>(n_sm, st, tq, tk, tv, ap);
+  }
+}
+
+cudaError_t launch_merge(int n_sm, cudaStream_t st, const pa::MergeParams& mp) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * n_sm);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pa::pa_merge_kernel, mp);
 }
 
 int encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
@@ -372,6 +425,9 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.cu_q_lens = cu_q_lens;
   sp.items = p->items;
   sp.req_info = p->req_info;
+  sp.req_aux = p->req_aux;
+  sp.unit_off = p->unit_off;
+  sp.split_list = p->split_list;
   sp.hdr = p->hdr;
   sp.max_items = p->max_items;
   sp.B = p->B; sp.Hkv = p->Hkv; sp.G = p->G; sp.C = p->C; sp.ps = p->ps; sp.BN = p->BN;
@@ -398,33 +454,28 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.tpb = p->tpb;
   ap.box_h = p->box_h;
   ap.scale_log2 = p->scale * 1.4426950408889634f;
-  const dim3 grid(p->n_sm), block(pa::kThreads);
   const bool prof = p->prof_on && p->prof_n < p->prof_cap;
   if (prof) cudaEventRecord(p->prof_ev[2 * p->prof_n], st);
-  switch (p->D) {
-    case 64:
-      pa::pa_attention_kernel<64><<<grid, block, pa::TileCfg<64>::SMEM_BYTES, st>>>(p->tm_q, p->tm_k, p->tm_v, ap);
-      break;
-    case 128:
-      pa::pa_attention_kernel<128><<<grid, block, pa::TileCfg<128>::SMEM_BYTES, st>>>(p->tm_q, p->tm_k, p->tm_v, ap);
-      break;
-    default:
-      pa::pa_attention_kernel<256><<<grid, block, pa::TileCfg<256>::SMEM_BYTES, st>>>(p->tm_q, p->tm_k, p->tm_v, ap);
-      break;
-  }
+  cudaError_t le = launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, ap);
   if (prof) {
     cudaEventRecord(p->prof_ev[2 * p->prof_n + 1], st);
     ++p->prof_n;
   }
-  if (sp.S_max > 1) {
+  if (le == cudaSuccess && sp.S_max > 1) {
     pa::MergeParams mp;
     mp.req_info = p->req_info;
+    mp.split_list = p->split_list;
+    mp.hdr = p->hdr;
     mp.part_o = p->part_o;
     mp.part_lse = p->part_lse;
     mp.out = static_cast<uint16_t*>(out);
     mp.lse = lse;
     mp.B = p->B; mp.Hq = p->Hq; mp.Hkv = p->Hkv; mp.G = p->G; mp.D = p->D; mp.S_max = p->S_max;
-    pa::pa_merge_kernel<<<p->B * p->Hkv, 128, 0, st>>>(mp);
+    le = launch_merge(p->n_sm, st, mp);
+  }
+  if (le != cudaSuccess) {
+    set_err("pa_run: launch failed: %s", cudaGetErrorString(le));
+    return PA_ERR_CUDA;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -576,8 +627,11 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   const long blocks_per_req = ((long)capacity * page_size + tpb - 1) / tpb;
   const long max_items = (long)batch * heads_kv * blocks_per_req;
   const size_t o_req = align_up(sizeof(pa::WsHeader), 256);
-  const size_t o_items = align_up(o_req + sizeof(int4) * (size_t)batch, 256);
-  const size_t need = o_items + sizeof(pa::WorkItem) * (size_t)max_items;
+  const size_t o_aux = align_up(o_req + sizeof(int4) * (size_t)batch, 256);
+  const size_t o_uoff = align_up(o_aux + sizeof(int4) * (size_t)batch, 256);
+  const size_t o_split = align_up(o_uoff + sizeof(int) * (size_t)(batch + 1), 256);
+  const size_t o_items = align_up(o_split + sizeof(int) * (size_t)batch, 256);
+  const size_t need = o_items + sizeof(pa::PackedItem) * (size_t)max_items;
   if (max_items > (1L << 30) || need > (size_t)PA_NOALLOC_SCRATCH_BYTES) {
     set_err("pa_run_noalloc: this geometry needs %zu bytes of scratch (%ld work items); the "
             "static scratch holds %u bytes -- use pa_create_plan / pa_run instead",
@@ -639,8 +693,11 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   pa::SchedParams sp;
   sp.seq_lens = seq_lens;
   sp.cu_q_lens = cu_q_lens;
-  sp.items = reinterpret_cast<pa::WorkItem*>(base + o_items);
+  sp.items = reinterpret_cast<pa::PackedItem*>(base + o_items);
+  sp.split_list = reinterpret_cast<int*>(base + o_split);
   sp.req_info = reinterpret_cast<int4*>(base + o_req);
+  sp.req_aux = reinterpret_cast<int4*>(base + o_aux);
+  sp.unit_off = reinterpret_cast<int*>(base + o_uoff);
   sp.hdr = hdr;
   sp.max_items = (int)max_items;
   sp.B = batch; sp.Hkv = heads_kv; sp.G = G; sp.C = capacity; sp.ps = page_size; sp.BN = BN;
@@ -668,17 +725,10 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   ap.box_h = box_h;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)head_dim);
   ap.scale_log2 = sc * 1.4426950408889634f;
-  const dim3 grid(nd->n_sm), block(pa::kThreads);
-  switch (head_dim) {
-    case 64:
-      pa::pa_attention_kernel<64><<<grid, block, pa::TileCfg<64>::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, ap);
-      break;
-    case 128:
-      pa::pa_attention_kernel<128><<<grid, block, pa::TileCfg<128>::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, ap);
-      break;
-    default:
-      pa::pa_attention_kernel<256><<<grid, block, pa::TileCfg<256>::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, ap);
-      break;
+  e = launch_attention_d(head_dim, nd->n_sm, st, tm_q, tm_k, tm_v, ap);
+  if (e != cudaSuccess) {
+    set_err("pa_run_noalloc: launch failed: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -6,10 +6,13 @@
 //      split)), longest first, plus per-request split counts.
 //   2. pa_attention_kernel<D>: persistent, one CTA per SM, warp-specialised:
 //        warps 0-3  softmax / correction / epilogue (one thread per query row)
-//        warp  4    producer: page-table-driven TMA gathers of K and V pages,
-//                   Q tiles by TMA (or plain loads for partial blocks)
+//        warp  4    producer: page-table-driven TMA gathers of K and V pages
 //        warp  5    MMA issuer: tcgen05 S = Q K^T and O += P V, TMEM accumulators
+//        warp  6    Q loader: Q tiles by TMA (or plain loads for partial blocks)
 //   3. pa_merge_kernel: log-sum-exp merge of split-KV partial states.
+// Kernels 2 and 3 are launched as programmatic dependents of the kernel
+// before them: their prologues overlap it, and `griddepcontrol.wait` orders
+// their first read of its results.
 //
 // Sources: page-table contract and page-pool bound from "integrate PrimTS FMHA
 // kernels" (TensorRT-LLM PR #17399, "Unified page-table metadata"); GQA
@@ -34,9 +37,36 @@ struct WorkItem {
   int q_tok0, n_tok;     // query tokens of the block (local to the request)
   int kv_lo, kv_hi;      // keys [kv_lo, kv_hi) processed by this item
   int kv_len, q_len;     // request lengths after validation
-  int t_base, pad;       // cu_q_lens[b]
+  int t_base;            // cu_q_lens[b]
 };
-static_assert(sizeof(WorkItem) == 48, "work item layout");
+
+// In memory an item is 32 bytes (two int4, written and read as vectors):
+//   {b, kvh | split << 16 | n_splits << 24, q_tok0, t_base}
+//   {kv_lo, kv_hi, kv_len, q_len}
+// n_tok is min(128 / G, q_len - q_tok0).
+struct __align__(16) PackedItem {
+  int4 a, c;
+};
+static_assert(sizeof(PackedItem) == 32, "work item layout");
+
+__device__ __forceinline__ WorkItem unpack_item(const PackedItem* items, int it, int tpb) {
+  // plain loads: the list was written by the kernel just before this one
+  const int4 a = items[it].a;
+  const int4 c = items[it].c;
+  WorkItem w;
+  w.b = a.x;
+  w.kvh = a.y & 0xffff;
+  w.split = (a.y >> 16) & 0xff;
+  w.n_splits = (a.y >> 24) & 0xff;
+  w.q_tok0 = a.z;
+  w.t_base = a.w;
+  w.kv_lo = c.x;
+  w.kv_hi = c.y;
+  w.kv_len = c.z;
+  w.q_len = c.w;
+  w.n_tok = min(tpb, w.q_len - w.q_tok0);
+  return w;
+}
 
 // Device status bits (mirror of PA_STATUS_* in pa.h).
 constexpr unsigned kStatusBadPage = 1u << 0;
@@ -48,14 +78,17 @@ constexpr unsigned kStatusTimeout = 1u << 4;
 struct WsHeader {
   unsigned status;
   int n_items;
-  int pad[62];
+  int n_split_reqs;   // requests split over KV (entries of the split list)
+  int pad[61];
 };
 
 constexpr int kBM = 128;              // query rows per tile (tcgen05 M)
-constexpr int kThreads = 192;         // 6 warps
+constexpr int kThreads = 224;         // 7 warps
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
+constexpr int kQWarp = 6;
 constexpr int kCostBuckets = 1024;
+constexpr int kSchedSmemReqs = 4096;  // unit offsets of up to this many requests live in smem
 constexpr int kMaxSplits = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows > 2^8
 
@@ -88,7 +121,7 @@ struct AttnParams {
   const int* cu_q_lens;       // [B+1] or nullptr
   uint16_t* out;              // bf16 [T, Hq, D]
   float* lse;                 // [T, Hq] or nullptr
-  const WorkItem* items;
+  const PackedItem* items;
   const WsHeader* hdr;
   float* part_o;              // [B*Hkv*S_max*128, D]
   float* part_lse;            // [B*Hkv*S_max*128]
@@ -132,8 +165,11 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
 struct SchedParams {
   const int* seq_lens;
   const int* cu_q_lens;
-  WorkItem* items;
+  PackedItem* items;
+  int* split_list;     // [B] requests with more than one split
   int4* req_info;      // [B] {n_splits, q_len, t_base, kv_len}
+  int4* req_aux;       // [B] {units, tiles per split, KV tiles of the single block, 0}
+  int* unit_off;       // [B + 1] exclusive prefix sum of units
   WsHeader* hdr;
   int max_items;
   int B, Hkv, G, C, ps, BN, tpb, S_max, forced_splits, n_ctas;
@@ -173,193 +209,264 @@ __device__ __forceinline__ ReqInfo read_request(const SchedParams& p, int b) {
 
 // Keys visible to the last row of query block [q0, q0 + n): the causal limit
 // aligned to the end of the request's KV, clamped to [0, kv_len].
-__device__ __forceinline__ int block_kv_hi(const ReqInfo& r, int q0, int n) {
-  int hi = q0 + n + (r.kv_len - r.q_len);
-  return hi < 0 ? 0 : (hi > r.kv_len ? r.kv_len : hi);
+__device__ __forceinline__ int block_kv_hi(int q_len, int kv_len, int q0, int n) {
+  int hi = q0 + n + (kv_len - q_len);
+  return hi < 0 ? 0 : (hi > kv_len ? kv_len : hi);
 }
 
-__device__ __forceinline__ int n_qblocks(const ReqInfo& r, int tpb) {
-  return r.q_len > 0 ? (r.q_len + tpb - 1) / tpb : 0;
-}
-
-// Split count and tiles per split of a request whose rows fit one query block.
-__device__ __forceinline__ void split_plan(const SchedParams& p, const ReqInfo& r, int chunk,
-                                           int& n_splits, int& per) {
-  const int tiles = ceil_div(block_kv_hi(r, 0, r.q_len), p.BN);
-  n_splits = 1;
-  per = tiles > 0 ? tiles : 1;
-  if (n_qblocks(r, p.tpb) != 1 || p.S_max <= 1 || tiles <= 1) return;
-  int s = p.forced_splits > 0 ? p.forced_splits : ceil_div(tiles, chunk);
-  if (s > p.S_max) s = p.S_max;
-  if (s > tiles) s = tiles;
-  if (s < 1) s = 1;
-  per = ceil_div(tiles, s);
-  n_splits = ceil_div(tiles, per);
+__device__ __forceinline__ int n_qblocks(int q_len, int tpb) {
+  return q_len > 0 ? (q_len + tpb - 1) / tpb : 0;
 }
 
 __device__ __forceinline__ int cost_bucket(int tiles) {
   return tiles < kCostBuckets ? tiles : kCostBuckets - 1;
 }
 
+// Exclusive scan of one int per thread over a 1024-thread block; returns the
+// thread's exclusive prefix and writes the block total to *total.
+__device__ __forceinline__ int block_scan_1024(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const int r = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+  *total = warp_sums[31];
+  __syncthreads();
+  return r;
+}
+
+// Cost (KV tiles) and shape of unit k of request b.
+struct Unit {
+  int q0, n_tok, kv_lo, kv_hi, split, cost;
+};
+
+__device__ __forceinline__ Unit unit_of(const SchedParams& p, const int4& ri, const int4& ra,
+                                        int k) {
+  Unit u;
+  const int ns = ri.x, q_len = ri.y, kv_len = ri.w;
+  if (ns > 1) {
+    const int per = ra.y, tiles = ra.z;
+    u.q0 = 0;
+    u.n_tok = q_len;
+    u.split = k;
+    u.kv_lo = k * per * p.BN;
+    u.kv_hi = min(block_kv_hi(q_len, kv_len, 0, q_len), (k + 1) * per * p.BN);
+    u.cost = min(per, tiles - k * per);
+  } else {
+    u.q0 = k * p.tpb;
+    u.n_tok = min(p.tpb, q_len - u.q0);
+    u.split = 0;
+    u.kv_lo = 0;
+    u.kv_hi = block_kv_hi(q_len, kv_len, u.q0, u.n_tok);
+    u.cost = ceil_div(u.kv_hi, p.BN);
+  }
+  return u;
+}
+
+// One CTA of 1024 threads.
+//   1. validate every request, count the KV tiles of all work;
+//   2. choose splits (about two waves of CTAs over all work, or the forced
+//      count) for requests whose packed rows fit one 128-row tile; count the
+//      units (query blocks or splits) of each request and prefix-sum them;
+//   3. histogram of unit costs, scanned in descending cost order;
+//   4. every unit writes its Hkv items at its cost bucket's cursor, so the
+//      work list comes out longest first.
+// Atomics on the histogram and the cursors are aggregated per warp.
 __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ int hist[kCostBuckets];
   __shared__ int cursor[kCostBuckets];
   __shared__ unsigned long long total_tiles;
   __shared__ int s_chunk;
   __shared__ unsigned s_flags;
   __shared__ int warp_sums[32];
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   for (int i = tid; i < kCostBuckets; i += blockDim.x) hist[i] = 0;
   if (tid == 0) { total_tiles = 0; s_flags = 0; }
   __syncthreads();
 
-  // Pass A: validate requests, count the KV tiles of all work.
+  // 1.
   unsigned long long my_tiles = 0;
   unsigned my_flags = 0;
   for (int b = tid; b < p.B; b += blockDim.x) {
     const ReqInfo r = read_request(p, b);
     my_flags |= r.flags;
-    const int nb = n_qblocks(r, p.tpb);
+    const int nb = n_qblocks(r.q_len, p.tpb);
+    int t = 0;
     for (int m = 0; m < nb; ++m) {
       const int q0 = m * p.tpb;
-      const int n = min(p.tpb, r.q_len - q0);
-      my_tiles += (unsigned long long)p.Hkv * ceil_div(block_kv_hi(r, q0, n), p.BN);
+      t += ceil_div(block_kv_hi(r.q_len, r.kv_len, q0, min(p.tpb, r.q_len - q0)), p.BN);
     }
+    my_tiles += (unsigned long long)p.Hkv * t;
   }
-  atomicAdd(&total_tiles, my_tiles);
-  if (my_flags) atomicOr(&s_flags, my_flags);
+  for (int o = 16; o > 0; o >>= 1) {
+    my_tiles += __shfl_xor_sync(0xffffffffu, my_tiles, o);
+    my_flags |= __shfl_xor_sync(0xffffffffu, my_flags, o);
+  }
+  if (lane == 0) {
+    atomicAdd(&total_tiles, my_tiles);
+    if (my_flags) atomicOr(&s_flags, my_flags);
+  }
   __syncthreads();
   if (tid == 0) {
-    // tiles per split so that the whole launch is about two waves of CTAs
     const unsigned long long target = (unsigned long long)p.n_ctas * 2ull;
-    unsigned long long c = (total_tiles + target - 1) / target;
+    const unsigned long long c = (total_tiles + target - 1) / target;
     s_chunk = (int)(c < 4 ? 4 : (c > (1ull << 30) ? (1ull << 30) : c));
     if (s_flags) atomicOr(&p.hdr->status, s_flags);
   }
   __syncthreads();
   const int chunk = s_chunk;
 
-  // Pass B: histogram of item costs (KV tiles per item).
-  for (int b = tid; b < p.B; b += blockDim.x) {
-    const ReqInfo r = read_request(p, b);
-    int ns, per;
-    split_plan(p, r, chunk, ns, per);
-    const int nb = n_qblocks(r, p.tpb);
-    if (ns > 1) {
-      const int tiles = ceil_div(block_kv_hi(r, 0, r.q_len), p.BN);
-      for (int s = 0; s < ns; ++s) {
-        const int t = min(per, tiles - s * per);
-        atomicAdd(&hist[cost_bucket(t)], p.Hkv);
+  // 2.
+  __shared__ int s_nsplit;
+  __shared__ int s_uoff[kSchedSmemReqs + 1];
+  if (tid == 0) s_nsplit = 0;
+  __syncthreads();
+  int running = 0;
+  for (int b0 = 0; b0 < p.B; b0 += blockDim.x) {
+    const int b = b0 + tid;
+    int units = 0;
+    if (b < p.B) {
+      const ReqInfo r = read_request(p, b);
+      const int nb = n_qblocks(r.q_len, p.tpb);
+      const int tiles = ceil_div(block_kv_hi(r.q_len, r.kv_len, 0, r.q_len), p.BN);
+      int ns = 1, per = tiles > 0 ? tiles : 1;
+      if (nb == 1 && p.S_max > 1 && tiles > 1) {
+        int sp = p.forced_splits > 0 ? p.forced_splits : ceil_div(tiles, chunk);
+        sp = min(sp, min(p.S_max, tiles));
+        if (sp < 1) sp = 1;
+        per = ceil_div(tiles, sp);
+        ns = ceil_div(tiles, per);
       }
-    } else {
-      for (int m = 0; m < nb; ++m) {
-        const int q0 = m * p.tpb;
-        const int n = min(p.tpb, r.q_len - q0);
-        atomicAdd(&hist[cost_bucket(ceil_div(block_kv_hi(r, q0, n), p.BN))], p.Hkv);
-      }
+      units = ns > 1 ? ns : nb;
+      p.req_info[b] = make_int4(ns, r.q_len, r.t_base, r.kv_len);
+      p.req_aux[b] = make_int4(units, per, tiles, 0);
+      if (ns > 1) p.split_list[atomicAdd(&s_nsplit, 1)] = b;
     }
+    int total;
+    const int off = block_scan_1024(units, warp_sums, &total);
+    if (b < p.B) {
+      p.unit_off[b] = running + off;
+      if (b < kSchedSmemReqs) s_uoff[b] = running + off;
+    }
+    running += total;
+  }
+  if (tid == 0) {
+    p.unit_off[p.B] = running;
+    if (p.B <= kSchedSmemReqs) s_uoff[p.B] = running;
+    p.hdr->n_split_reqs = s_nsplit;
   }
   __syncthreads();
+  const int U = running;
+  const int* uoff = p.B <= kSchedSmemReqs ? s_uoff : p.unit_off;
 
-  // Exclusive scan over buckets in descending cost order (longest items first).
+  // 3.
+  for (int u0 = 0; u0 < U; u0 += blockDim.x) {
+    const int u = u0 + tid;
+    int key = -1 - lane;     // distinct per idle lane
+    if (u < U) {
+      int lo = 0, hi = p.B - 1;            // last b with unit_off[b] <= u
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (uoff[mid] <= u) lo = mid; else hi = mid - 1;
+      }
+      const Unit un = unit_of(p, p.req_info[lo], p.req_aux[lo], u - uoff[lo]);
+      key = cost_bucket(un.cost);
+    }
+    const unsigned grp = __match_any_sync(0xffffffffu, key);
+    if (key >= 0 && lane == __ffs(grp) - 1) atomicAdd(&hist[key], __popc(grp) * p.Hkv);
+  }
+  __syncthreads();
   {
-    const int lane = tid & 31, warp = tid >> 5;
-    int v = 0;
-    const int bucket = kCostBuckets - 1 - tid;        // blockDim.x == kCostBuckets
-    if (tid < kCostBuckets) v = hist[bucket];
-    int x = v;
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_sums[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
-      }
-      warp_sums[lane] = w;   // inclusive
-    }
-    __syncthreads();
-    const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
-    if (tid < kCostBuckets) cursor[bucket] = before;
-    if (tid == blockDim.x - 1) {
-      const int total = warp_sums[(blockDim.x >> 5) - 1];
-      p.hdr->n_items = total < p.max_items ? total : p.max_items;
-    }
+    const int bucket = kCostBuckets - 1 - tid;
+    const int v = hist[bucket];
+    int total;
+    const int before = block_scan_1024(v, warp_sums, &total);
+    cursor[bucket] = before;
+    if (tid == 0) p.hdr->n_items = total < p.max_items ? total : p.max_items;
   }
   __syncthreads();
 
-  // Pass C: emit the items.
-  for (int b = tid; b < p.B; b += blockDim.x) {
-    const ReqInfo r = read_request(p, b);
-    int ns, per;
-    split_plan(p, r, chunk, ns, per);
-    p.req_info[b] = make_int4(ns, r.q_len, r.t_base, r.kv_len);
-    const int nb = n_qblocks(r, p.tpb);
-    WorkItem w;
-    w.b = b;
-    w.n_splits = ns;
-    w.kv_len = r.kv_len;
-    w.q_len = r.q_len;
-    w.t_base = r.t_base;
-    w.pad = 0;
-    if (ns > 1) {
-      const int hi = block_kv_hi(r, 0, r.q_len);
-      const int tiles = ceil_div(hi, p.BN);
-      for (int s = 0; s < ns; ++s) {
-        const int t = min(per, tiles - s * per);
-        w.split = s;
-        w.q_tok0 = 0;
-        w.n_tok = r.q_len;
-        w.kv_lo = s * per * p.BN;
-        w.kv_hi = min(hi, (s + 1) * per * p.BN);
-        for (int g = 0; g < p.Hkv; ++g) {
-          w.kvh = g;
-          const int pos = atomicAdd(&cursor[cost_bucket(t)], 1);
-          if (pos < p.max_items) p.items[pos] = w;
-        }
+  // 4.  Each unit owns Hkv consecutive items; the warp writes the items of its
+  // 32 units cooperatively (item i of the warp -> unit i / Hkv, head i % Hkv),
+  // so consecutive lanes store consecutive 32-byte items.
+  for (int u0 = 0; u0 < U; u0 += blockDim.x) {
+    const int u = u0 + tid;
+    int key = -1 - lane;
+    int b = 0;
+    Unit un = {0, 0, 0, 0, 0, 0};
+    int4 ri = make_int4(0, 0, 0, 0);
+    if (u < U) {
+      int lo = 0, hi = p.B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (uoff[mid] <= u) lo = mid; else hi = mid - 1;
       }
-    } else {
-      for (int m = 0; m < nb; ++m) {
-        const int q0 = m * p.tpb;
-        const int n = min(p.tpb, r.q_len - q0);
-        w.split = 0;
-        w.q_tok0 = q0;
-        w.n_tok = n;
-        w.kv_lo = 0;
-        w.kv_hi = block_kv_hi(r, q0, n);
-        const int t = ceil_div(w.kv_hi, p.BN);
-        for (int g = 0; g < p.Hkv; ++g) {
-          w.kvh = g;
-          const int pos = atomicAdd(&cursor[cost_bucket(t)], 1);
-          if (pos < p.max_items) p.items[pos] = w;
-        }
+      b = lo;
+      ri = p.req_info[b];
+      un = unit_of(p, ri, p.req_aux[b], u - uoff[b]);
+      key = cost_bucket(un.cost);
+    }
+    const unsigned grp = __match_any_sync(0xffffffffu, key);
+    const int leader = __ffs(grp) - 1;
+    int base = 0;
+    if (key >= 0 && lane == leader) base = atomicAdd(&cursor[key], __popc(grp) * p.Hkv);
+    base = __shfl_sync(0xffffffffu, base, leader);
+    const int pos = key >= 0 ? base + __popc(grp & ((1u << lane) - 1)) * p.Hkv : -1;
+    const int packed = (un.split << 16) | (ri.x << 24);
+    for (int i0 = 0; i0 < 32 * p.Hkv; i0 += 32) {
+      const int i = i0 + lane;
+      const int src = i / p.Hkv, g = i - src * p.Hkv;
+      const int spos = __shfl_sync(0xffffffffu, pos, src);
+      const int sb = __shfl_sync(0xffffffffu, b, src);
+      const int spk = __shfl_sync(0xffffffffu, packed, src);
+      const int sq0 = __shfl_sync(0xffffffffu, un.q0, src);
+      const int stb = __shfl_sync(0xffffffffu, ri.z, src);
+      const int slo = __shfl_sync(0xffffffffu, un.kv_lo, src);
+      const int shi = __shfl_sync(0xffffffffu, un.kv_hi, src);
+      const int skv = __shfl_sync(0xffffffffu, ri.w, src);
+      const int sql = __shfl_sync(0xffffffffu, ri.y, src);
+      if (spos >= 0 && spos + g < p.max_items) {
+        PackedItem* dst = p.items + spos + g;
+        dst->a = make_int4(sb, g | spk, sq0, stb);
+        dst->c = make_int4(slo, shi, skv, sql);
       }
     }
   }
 }
 
 // =========================================================================== attention
+// Q loader warp: one Q tile per item, into the single Q buffer.  Full blocks
+// inside [0, T) use one TMA box per 64-column chunk; partial blocks (decode,
+// last block of a request) use plain 16-byte loads of the live rows only,
+// stored with the same 128-byte swizzle the TMA applies (16-byte unit u of
+// row r lands at unit u ^ (r % 8) of that row).
 template <int D>
-__device__ __forceinline__ void producer_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
-                                              const CUtensorMap* tm_v, const AttnParams& p,
-                                              uint32_t sQ, uint32_t sKV, uint32_t bar0,
-                                              int n_items, volatile int* abort) {
+__device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const AttnParams& p,
+                                              uint32_t sQ, uint32_t bar0, int n_items,
+                                              volatile int* abort) {
   using C = TileCfg<D>;
   const int lane = threadIdx.x & 31;
   const int G = p.G;
   const int T = p.cu_q_lens ? p.cu_q_lens[p.B] : p.B;
-  uint32_t ld_idx = 0, q_cnt = 0;
-  bool ok = true;
-  for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-    const WorkItem w = p.items[it];
-    const int n = item_tiles(w, C::BN);
-    if (n == 0) continue;
-    // ---- Q tile
-    if (!warp_wait(bar0 + 8 * C::B_QEMPTY, (q_cnt & 1) ^ 1, abort)) { ok = false; break; }
+  uint32_t q_cnt = 0;
+  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    const WorkItem w = unpack_item(p.items, it, p.tpb);
+    if (item_tiles(w, C::BN) == 0) continue;
+    if (!warp_wait(bar0 + 8 * C::B_QEMPTY, (q_cnt & 1) ^ 1, abort)) break;
     const int t0 = w.t_base + w.q_tok0;
     if (w.n_tok == p.tpb && t0 + p.tpb <= T) {
       if (lane == 0) {
@@ -368,9 +475,6 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_q, const CUt
           tma_load_3d(sQ + c * C::Q_CHUNK, tm_q, bar0 + 8 * C::B_QFULL, c * 64, w.kvh * G, t0);
       }
     } else {
-      // Partial block: plain 16-byte loads of the live rows only, stored with the
-      // same 128-byte swizzle the TMA uses (16-byte unit u of row r lands at
-      // unit u ^ (r % 8) of that row).
       const int rows = w.n_tok * G;
       const int units = rows * (D / 8);
       for (int u = lane; u < units; u += 32) {
@@ -387,7 +491,37 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_q, const CUt
       if (lane == 0) mbar_arrive(bar0 + 8 * C::B_QFULL);
     }
     ++q_cnt;
-    // ---- K / V tiles, gathered page by page
+  }
+  if (*abort && lane == 0 && q_cnt > 0) mbar_drain(bar0 + 8 * C::B_QFULL, (q_cnt - 1) & 1);
+}
+
+// Page id of this lane's box in tile j of item w (0 for lanes without a box).
+__device__ __forceinline__ int tile_page_id(const AttnParams& p, const WorkItem& w, int j, int BN,
+                                            int lane) {
+  const int n0 = w.kv_lo + j * BN;
+  const int live = min(w.kv_len - n0, BN);
+  if (lane * p.box_h >= live) return 0;
+  const int col = (n0 + lane * p.box_h) / p.ps;
+  return __ldg(p.page_table + (size_t)w.b * p.C + col);
+}
+
+// KV producer warp: K and V tiles in the MMA's consumption order into the slot
+// ring.  One TMA box is one page (or the part of a page inside the tile) of
+// one KV head; lane k issues box k.  The page ids of tile j+1 are fetched
+// right after tile j's K is issued, so the table read is off the critical path.
+template <int D>
+__device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                              const AttnParams& p, uint32_t sKV, uint32_t bar0,
+                                              int n_items, volatile int* abort) {
+  using C = TileCfg<D>;
+  const int lane = threadIdx.x & 31;
+  uint32_t ld_idx = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    const WorkItem w = unpack_item(p.items, it, p.tpb);
+    const int n = item_tiles(w, C::BN);
+    if (n == 0) continue;
+    int pid0 = tile_page_id(p, w, 0, C::BN, lane), pid1 = 0, pid2 = 0;   // tile j -> pid[j % 3]
     for (int s = 0; s < 2 * n; ++s) {
       int j;
       bool is_v;
@@ -405,10 +539,10 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_q, const CUt
       const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
       if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
       __syncwarp();
+      const int jm = j % 3;
+      int page = jm == 0 ? pid0 : (jm == 1 ? pid1 : pid2);
       if (lane < nbox) {
-        const int tok = n0 + lane * p.box_h;
-        const int col = tok / p.ps, row = tok - col * p.ps;
-        int page = p.page_table[(size_t)w.b * p.C + col];
+        const int row = (n0 + lane * p.box_h) % p.ps;
         if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
           atomicOr(p.status, kStatusBadPage);
           page = -1;   // out of the tensor map: the box reads as zeros
@@ -417,6 +551,11 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_q, const CUt
         const uint32_t dst = sKV + slot * C::SLOT_BYTES + lane * p.box_h * 128;
         for (int c = 0; c < C::DCH; ++c)
           tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, row, page);
+      }
+      if (!is_v && j + 1 < n) {
+        const int nx = tile_page_id(p, w, j + 1, C::BN, lane);
+        const int jn = (j + 1) % 3;
+        if (jn == 0) pid0 = nx; else if (jn == 1) pid1 = nx; else pid2 = nx;
       }
       ++ld_idx;
     }
@@ -427,7 +566,6 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_q, const CUt
       const uint32_t first = ld_idx > (uint32_t)C::NSLOT ? ld_idx - C::NSLOT : 0;
       for (uint32_t k = first; k < ld_idx; ++k)
         mbar_drain(bar0 + 8 * (C::B_KVFULL + k % C::NSLOT), (k / C::NSLOT) & 1);
-      if (q_cnt > 0) mbar_drain(bar0 + 8 * C::B_QFULL, (q_cnt - 1) & 1);
     }
   }
 }
@@ -442,7 +580,7 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
   uint32_t ld_idx = 0, g_base = 0, q_cnt = 0;
   bool ok = true;
   for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-    const WorkItem w = p.items[it];
+    const WorkItem w = unpack_item(p.items, it, p.tpb);
     const int n = item_tiles(w, C::BN);
     if (n == 0) continue;
     if (!mbar_wait(bar0 + 8 * C::B_QFULL, q_cnt & 1, abort)) { ok = false; break; }
@@ -511,7 +649,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
   uint32_t g_base = 0, ld_base = 0;
   bool ok = true;
   for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-    const WorkItem w = p.items[it];
+    const WorkItem w = unpack_item(p.items, it, p.tpb);
     const int n = item_tiles(w, BN);
     const int n_rows = w.n_tok * G;
     const bool real = r < n_rows;
@@ -546,13 +684,17 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
       const int n0 = w.kv_lo + j * BN;
       if (warp_active) {
         float s[BN];
+        {
+          uint32_t v[BN / 32][32];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(trow + sb * BN + c * 32, v);
-          tmem_ld_wait(v);
+          for (int c = 0; c < BN / 32; ++c) tmem_ld32(trow + sb * BN + c * 32, v[c]);
+          tmem_ld_wait(v[0]);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(v[e]);
+          for (int c = 1; c < BN / 32; ++c) reg_tie(v[c]);
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(v[c][e]);
         }
         const int nvis = lim - n0;
         if (nvis < BN) {
@@ -575,13 +717,19 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
           tc_fence_after();
           const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(trow + C::O_COL + c * 32, v);
-            tmem_ld_wait(v);
+          for (int c = 0; c < D / 32; c += 2) {
+            uint32_t v[2][32];
+            tmem_ld32(trow + C::O_COL + c * 32, v[0]);
+            tmem_ld32(trow + C::O_COL + c * 32 + 32, v[1]);
+            tmem_ld_wait(v[0]);
+            reg_tie(v[1]);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-            tmem_st32(trow + C::O_COL + c * 32, v);
+            for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                v[h2][e] = __float_as_uint(__uint_as_float(v[h2][e]) * alpha);
+              tmem_st32(trow + C::O_COL + (c + h2) * 32, v[h2]);
+            }
           }
           tmem_st_wait();
         }
@@ -648,28 +796,36 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       const float lse_v = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + C::O_COL + c * 32, v);
-        tmem_ld_wait(v);
+      for (int c = 0; c < D / 32; c += 2) {
+        uint32_t vv[2][32];
+        tmem_ld32(trow + C::O_COL + c * 32, vv[0]);
+        tmem_ld32(trow + C::O_COL + c * 32 + 32, vv[1]);
+        tmem_ld_wait(vv[0]);
+        reg_tie(vv[1]);
         if (real) {
-          if (split) {
-            float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + c * 32);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv_l, __uint_as_float(v[4 * e + 1]) * inv_l,
-                                   __uint_as_float(v[4 * e + 2]) * inv_l,
-                                   __uint_as_float(v[4 * e + 3]) * inv_l);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)t * p.Hq + h) * D + c * 32);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const uint32_t* v = vv[h2];
+            if (split) {
+              float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + (c + h2) * 32);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint4 q4;
-              q4.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * inv_l, __uint_as_float(v[8 * e + 1]) * inv_l);
-              q4.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * inv_l, __uint_as_float(v[8 * e + 3]) * inv_l);
-              q4.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * inv_l, __uint_as_float(v[8 * e + 5]) * inv_l);
-              q4.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * inv_l, __uint_as_float(v[8 * e + 7]) * inv_l);
-              dst[e] = q4;
+              for (int e = 0; e < 8; ++e)
+                dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv_l,
+                                     __uint_as_float(v[4 * e + 1]) * inv_l,
+                                     __uint_as_float(v[4 * e + 2]) * inv_l,
+                                     __uint_as_float(v[4 * e + 3]) * inv_l);
+            } else {
+              uint4* dst =
+                  reinterpret_cast<uint4*>(p.out + ((size_t)t * p.Hq + h) * D + (c + h2) * 32);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint4 q4;
+                q4.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * inv_l, __uint_as_float(v[8 * e + 1]) * inv_l);
+                q4.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * inv_l, __uint_as_float(v[8 * e + 3]) * inv_l);
+                q4.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * inv_l, __uint_as_float(v[8 * e + 5]) * inv_l);
+                q4.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * inv_l, __uint_as_float(v[8 * e + 7]) * inv_l);
+                dst[e] = q4;
+              }
             }
           }
         }
@@ -727,18 +883,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (warp == kProducerWarp && (threadIdx.x & 31) == 0) {
-    tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
+  if (warp == kQWarp && (threadIdx.x & 31) == 0) tma_prefetch_desc(&tm_q);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything above overlaps the scheduler kernel; its work list is read below
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int n_items = p.hdr->n_items;
 
   if (warp == kProducerWarp) {
-    producer_role<D>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bar0, n_items, abort);
+    producer_role<D>(&tm_k, &tm_v, p, sKV, bar0, n_items, abort);
+  } else if (warp == kQWarp) {
+    q_loader_role<D>(&tm_q, p, sQ, bar0, n_items, abort);
   } else if (warp == kMmaWarp) {
     if ((threadIdx.x & 31) == 0) mma_role<D>(p, sQ, sKV, bar0, tmem, n_items, abort);
     __syncwarp();
@@ -758,6 +919,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // =========================================================================== merge
 struct MergeParams {
   const int4* req_info;  // {n_splits, q_len, t_base, kv_len}
+  const int* split_list;
+  const WsHeader* hdr;
   const float* part_o;
   const float* part_lse;
   uint16_t* out;
@@ -767,47 +930,57 @@ struct MergeParams {
 
 // out = sum_s exp(lse_s - L) O_s with L = ln sum_s exp(lse_s): the exact merge
 // of attention states over disjoint key ranges; empty splits (lse_s = -inf)
-// get weight 0.
+// get weight 0.  One warp per (split request, KV head, row); the loads of
+// several splits are kept in flight together.
 __global__ void __launch_bounds__(128) pa_merge_kernel(MergeParams p) {
-  const int bh = blockIdx.x;
-  const int b = bh / p.Hkv, kvh = bh % p.Hkv;
-  const int4 ri = p.req_info[b];
-  const int ns = ri.x;
-  if (ns <= 1) return;
-  const int n_rows = ri.y * p.G;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int n_req = p.hdr->n_split_reqs;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < n_rows; r += 4) {
-    const size_t base = (size_t)bh * p.S_max * kBM + r;   // + s * kBM
-    float l0 = lane < ns ? p.part_lse[base + (size_t)lane * kBM] : -INFINITY;
-    float l1 = lane + 32 < ns ? p.part_lse[base + (size_t)(lane + 32) * kBM] : -INFINITY;
+  const int n_units = n_req * p.Hkv * kBM;
+  for (int u = blockIdx.x * 4 + warp; u < n_units; u += gridDim.x * 4) {
+    const int r = u % kBM;
+    const int kh = u / kBM;
+    const int kvh = kh % p.Hkv;
+    const int b = p.split_list[kh / p.Hkv];
+    const int4 ri = p.req_info[b];
+    const int ns = ri.x;
+    if (r >= ri.y * p.G) continue;
+    const size_t base = ((size_t)b * p.Hkv + kvh) * p.S_max * kBM + r;   // + s * kBM
+    const float l0 = lane < ns ? p.part_lse[base + (size_t)lane * kBM] : -INFINITY;
+    const float l1 = lane + 32 < ns ? p.part_lse[base + (size_t)(lane + 32) * kBM] : -INFINITY;
     float m = fmaxf(l0, l1);
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float e = 0.f;
-    if (m != -INFINITY) {
+    if (m != -INFINITY)
       e = (l0 == -INFINITY ? 0.f : expf(l0 - m)) + (l1 == -INFINITY ? 0.f : expf(l1 - m));
-    }
     for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
     const float L = (m == -INFINITY) ? -INFINITY : m + logf(e);
+    const float w0 = (L == -INFINITY || l0 == -INFINITY) ? 0.f : expf(l0 - L);
+    const float w1 = (L == -INFINITY || l1 == -INFINITY) ? 0.f : expf(l1 - L);
     const int t = ri.z + r / p.G;
     const int h = kvh * p.G + r % p.G;
-    for (int d = lane * 4; d < p.D; d += 128) {
+    for (int d0 = 0; d0 < p.D; d0 += 128) {          // warp-uniform loop
+      const int d = d0 + lane * 4;
+      const bool act = d < p.D;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-      if (L != -INFINITY) {
-        for (int s = 0; s < ns; ++s) {
-          const float ls = p.part_lse[base + (size_t)s * kBM];
-          if (ls == -INFINITY) continue;
-          const float wgt = expf(ls - L);
-          const float4 o = *reinterpret_cast<const float4*>(p.part_o + (base + (size_t)s * kBM) * p.D + d);
+#pragma unroll 4
+      for (int s = 0; s < ns; ++s) {
+        const float wgt = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
+        if (act) {
+          const float4 o =
+              *reinterpret_cast<const float4*>(p.part_o + (base + (size_t)s * kBM) * p.D + d);
           a0 = fmaf(wgt, o.x, a0);
           a1 = fmaf(wgt, o.y, a1);
           a2 = fmaf(wgt, o.z, a2);
           a3 = fmaf(wgt, o.w, a3);
         }
       }
-      uint2 pk;
-      pk.x = pack_bf16x2(a0, a1);
-      pk.y = pack_bf16x2(a2, a3);
-      *reinterpret_cast<uint2*>(p.out + ((size_t)t * p.Hq + h) * p.D + d) = pk;
+      if (act) {
+        uint2 pk;
+        pk.x = pack_bf16x2(a0, a1);
+        pk.y = pack_bf16x2(a2, a3);
+        *reinterpret_cast<uint2*>(p.out + ((size_t)t * p.Hq + h) * p.D + d) = pk;
+      }
     }
     if (lane == 0 && p.lse) p.lse[(size_t)t * p.Hq + h] = L;
   }
