@@ -49,10 +49,7 @@ struct __align__(16) PackedItem {
 };
 static_assert(sizeof(PackedItem) == 32, "work item layout");
 
-__device__ __forceinline__ WorkItem unpack_item(const PackedItem* items, int it, int tpb) {
-  // plain loads: the list was written by the kernel just before this one
-  const int4 a = items[it].a;
-  const int4 c = items[it].c;
+__device__ __forceinline__ WorkItem unpack_raw(const int4& a, const int4& c, int tpb) {
   WorkItem w;
   w.b = a.x;
   w.kvh = a.y & 0xffff;
@@ -67,6 +64,31 @@ __device__ __forceinline__ WorkItem unpack_item(const PackedItem* items, int it,
   w.n_tok = min(tpb, w.q_len - w.q_tok0);
   return w;
 }
+
+// The items of this CTA (blockIdx.x, + gridDim.x, ...), each read one item
+// ahead so that its load latency hides behind the current item.
+struct ItemStream {
+  const PackedItem* items;
+  int n_items, tpb, it;
+  int4 na, nc;
+  __device__ __forceinline__ ItemStream(const PackedItem* items_, int n, int tpb_)
+      : items(items_), n_items(n), tpb(tpb_), it(blockIdx.x) {
+    // plain loads: the list was written by the kernel just before this one
+    if (it < n_items) { na = items[it].a; nc = items[it].c; }
+  }
+  __device__ __forceinline__ bool next(WorkItem& w) {
+    if (it >= n_items) return false;
+    w = unpack_raw(na, nc, tpb);
+    it += gridDim.x;
+    if (it < n_items) { na = items[it].a; nc = items[it].c; }
+    return true;
+  }
+  __device__ __forceinline__ bool peek(WorkItem& w) const {
+    if (it >= n_items) return false;
+    w = unpack_raw(na, nc, tpb);
+    return true;
+  }
+};
 
 // Device status bits (mirror of PA_STATUS_* in pa.h).
 constexpr unsigned kStatusBadPage = 1u << 0;
@@ -100,16 +122,18 @@ struct TileCfg {
   static constexpr int Q_BYTES = kBM * D * 2;
   static constexpr int SLOT_CHUNK = BN * 128;         // bytes of one K/V column chunk
   static constexpr int SLOT_BYTES = BN * D * 2;
-  static constexpr int NSLOT = (D == 64) ? 12 : (D == 128 ? 6 : 5);
+  static constexpr int QBUF = (D == 256) ? 1 : 2;      // Q tiles in flight
+  static constexpr int NSLOT = (D == 64) ? 12 : 5;
   static constexpr int O_COL = 2 * BN;                // TMEM: S0 [0,BN), S1 [BN,2BN), O
   static constexpr int TMEM_COLS = 512;
-  // barriers: q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full[2], p_full[2],
-  //           pv_done[2], o_empty, drain
-  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = 2 + NSLOT,
-                       B_SFULL = 2 + 2 * NSLOT, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
-                       B_OEMPTY = B_PVDONE + 2, B_DRAIN = B_OEMPTY + 1, NBAR = B_DRAIN + 1;
+  // barriers: q_full[QBUF], q_empty[QBUF], kv_full[NSLOT], kv_empty[NSLOT], s_full[2],
+  //           p_full[2], pv_done[2], o_empty, drain
+  static constexpr int B_QFULL = 0, B_QEMPTY = QBUF, B_KVFULL = 2 * QBUF,
+                       B_KVEMPTY = 2 * QBUF + NSLOT, B_SFULL = 2 * QBUF + 2 * NSLOT,
+                       B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2, B_OEMPTY = B_PVDONE + 2,
+                       B_DRAIN = B_OEMPTY + 1, NBAR = B_DRAIN + 1;
   static constexpr int BAR_BYTES = 512;
-  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + NSLOT * SLOT_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + QBUF * Q_BYTES + NSLOT * SLOT_BYTES + BAR_BYTES;
   static_assert(NBAR * 8 + 16 <= BAR_BYTES, "barrier area");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(O_COL + D <= TMEM_COLS, "TMEM columns");
@@ -373,7 +397,15 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
   const int U = running;
   const int* uoff = p.B <= kSchedSmemReqs ? s_uoff : p.unit_off;
 
-  // 3.
+  // 3.  Ordering.  A request with several query blocks (prefill) keeps its
+  // units together, last block (most keys) first, and the block of units is
+  // placed by its largest cost: the CTAs then work on few requests at a time
+  // and the K/V tiles those blocks share are re-read from L2, not DRAM.  Other
+  // units (decode-like, KV splits) are placed one by one, longest first.
+  for (int b = tid; b < p.B; b += blockDim.x) {
+    const int4 ri = p.req_info[b], ra = p.req_aux[b];
+    if (ri.x == 1 && ra.x > 1) atomicAdd(&hist[cost_bucket(ra.z)], ra.x * p.Hkv);
+  }
   for (int u0 = 0; u0 < U; u0 += blockDim.x) {
     const int u = u0 + tid;
     int key = -1 - lane;     // distinct per idle lane
@@ -383,8 +415,8 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
         const int mid = (lo + hi + 1) >> 1;
         if (uoff[mid] <= u) lo = mid; else hi = mid - 1;
       }
-      const Unit un = unit_of(p, p.req_info[lo], p.req_aux[lo], u - uoff[lo]);
-      key = cost_bucket(un.cost);
+      const int4 ri = p.req_info[lo], ra = p.req_aux[lo];
+      if (!(ri.x == 1 && ra.x > 1)) key = cost_bucket(unit_of(p, ri, ra, u - uoff[lo]).cost);
     }
     const unsigned grp = __match_any_sync(0xffffffffu, key);
     if (key >= 0 && lane == __ffs(grp) - 1) atomicAdd(&hist[key], __popc(grp) * p.Hkv);
@@ -399,6 +431,15 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
     if (tid == 0) p.hdr->n_items = total < p.max_items ? total : p.max_items;
   }
   __syncthreads();
+  for (int b = tid; b < p.B; b += blockDim.x) {
+    const int4 ri = p.req_info[b];
+    int4 ra = p.req_aux[b];
+    if (ri.x == 1 && ra.x > 1) {
+      ra.w = atomicAdd(&cursor[cost_bucket(ra.z)], ra.x * p.Hkv);
+      p.req_aux[b] = ra;
+    }
+  }
+  __syncthreads();
 
   // 4.  Each unit owns Hkv consecutive items; the warp writes the items of its
   // 32 units cooperatively (item i of the warp -> unit i / Hkv, head i % Hkv),
@@ -409,6 +450,7 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
     int b = 0;
     Unit un = {0, 0, 0, 0, 0, 0};
     int4 ri = make_int4(0, 0, 0, 0);
+    int pos = -1;
     if (u < U) {
       int lo = 0, hi = p.B - 1;
       while (lo < hi) {
@@ -417,15 +459,18 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
       }
       b = lo;
       ri = p.req_info[b];
-      un = unit_of(p, ri, p.req_aux[b], u - uoff[b]);
-      key = cost_bucket(un.cost);
+      const int4 ra = p.req_aux[b];
+      const int k = u - uoff[b];
+      un = unit_of(p, ri, ra, k);
+      if (ri.x == 1 && ra.x > 1) pos = ra.w + (ra.x - 1 - k) * p.Hkv;   // grouped request
+      else key = cost_bucket(un.cost);
     }
     const unsigned grp = __match_any_sync(0xffffffffu, key);
     const int leader = __ffs(grp) - 1;
     int base = 0;
     if (key >= 0 && lane == leader) base = atomicAdd(&cursor[key], __popc(grp) * p.Hkv);
     base = __shfl_sync(0xffffffffu, base, leader);
-    const int pos = key >= 0 ? base + __popc(grp & ((1u << lane) - 1)) * p.Hkv : -1;
+    if (key >= 0) pos = base + __popc(grp & ((1u << lane) - 1)) * p.Hkv;
     const int packed = (un.split << 16) | (ri.x << 24);
     for (int i0 = 0; i0 < 32 * p.Hkv; i0 += 32) {
       const int i = i0 + lane;
@@ -463,36 +508,58 @@ __device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const Att
   const int G = p.G;
   const int T = p.cu_q_lens ? p.cu_q_lens[p.B] : p.B;
   uint32_t q_cnt = 0;
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-    const WorkItem w = unpack_item(p.items, it, p.tpb);
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+  while (items.next(w)) {
     if (item_tiles(w, C::BN) == 0) continue;
-    if (!warp_wait(bar0 + 8 * C::B_QEMPTY, (q_cnt & 1) ^ 1, abort)) break;
+    const uint32_t qb = q_cnt % C::QBUF;
+    const uint32_t sQb = sQ + qb * C::Q_BYTES;
+    const uint32_t qfull = bar0 + 8 * (C::B_QFULL + qb);
+    if (!warp_wait(bar0 + 8 * (C::B_QEMPTY + qb), ((q_cnt / C::QBUF) & 1) ^ 1, abort)) break;
     const int t0 = w.t_base + w.q_tok0;
     if (w.n_tok == p.tpb && t0 + p.tpb <= T) {
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar0 + 8 * C::B_QFULL, C::DCH * p.tpb * G * 128);
+        mbar_arrive_expect_tx(qfull, C::DCH * p.tpb * G * 128);
         for (int c = 0; c < C::DCH; ++c)
-          tma_load_3d(sQ + c * C::Q_CHUNK, tm_q, bar0 + 8 * C::B_QFULL, c * 64, w.kvh * G, t0);
+          tma_load_3d(sQb + c * C::Q_CHUNK, tm_q, qfull, c * 64, w.kvh * G, t0);
       }
     } else {
       const int rows = w.n_tok * G;
       const int units = rows * (D / 8);
-      for (int u = lane; u < units; u += 32) {
-        const int r = u / (D / 8), c16 = u % (D / 8);
-        const int t = t0 + r / G, h = w.kvh * G + r % G;
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)t * p.Hq + h) * D) + c16);
-        const uint32_t dst = sQ + (c16 >> 3) * C::Q_CHUNK + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y),
-                     "r"(v.z), "r"(v.w)
-                     : "memory");
+      for (int u0 = 0; u0 < units; u0 += 8 * 32) {
+        uint4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {          // all loads first, then the stores
+          const int u = u0 + k * 32 + lane;
+          if (u < units) {
+            const int r = u / (D / 8), c16 = u % (D / 8);
+            const int t = t0 + r / G, h = w.kvh * G + r % G;
+            v[k] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)t * p.Hq + h) * D) + c16);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int u = u0 + k * 32 + lane;
+          if (u < units) {
+            const int r = u / (D / 8), c16 = u % (D / 8);
+            const uint32_t dst =
+                sQb + (c16 >> 3) * C::Q_CHUNK + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[k].x),
+                         "r"(v[k].y), "r"(v[k].z), "r"(v[k].w)
+                         : "memory");
+          }
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar0 + 8 * C::B_QFULL);
+      if (lane == 0) mbar_arrive(qfull);
     }
     ++q_cnt;
   }
-  if (*abort && lane == 0 && q_cnt > 0) mbar_drain(bar0 + 8 * C::B_QFULL, (q_cnt - 1) & 1);
+  if (*abort && lane == 0) {
+    for (uint32_t k = q_cnt > (uint32_t)C::QBUF ? q_cnt - C::QBUF : 0; k < q_cnt; ++k)
+      mbar_drain(bar0 + 8 * (C::B_QFULL + k % C::QBUF), (k / C::QBUF) & 1);
+  }
 }
 
 // Page id of this lane's box in tile j of item w (0 for lanes without a box).
@@ -517,11 +584,24 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
-  for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-    const WorkItem w = unpack_item(p.items, it, p.tpb);
+  int pid_next = 0;
+  bool have_next = false;
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+  while (ok && items.next(w)) {
     const int n = item_tiles(w, C::BN);
-    if (n == 0) continue;
-    int pid0 = tile_page_id(p, w, 0, C::BN, lane), pid1 = 0, pid2 = 0;   // tile j -> pid[j % 3]
+    if (n == 0) {
+      have_next = false;
+      continue;
+    }
+    // Page ids are loop-carried so that no load result is used in the
+    // iteration that issues it: pid_k holds tile j's ids when K_j is issued
+    // (loaded one K-step earlier), pid_v holds tile j-1's for V_{j-1}, and
+    // pid_v_next keeps tile j's for V_j.  Tile 0 was fetched during the
+    // previous item when possible.
+    int pid_k = have_next ? pid_next : tile_page_id(p, w, 0, C::BN, lane);
+    int pid_v = 0, pid_v_next = 0;
+    have_next = false;
     for (int s = 0; s < 2 * n; ++s) {
       int j;
       bool is_v;
@@ -539,8 +619,14 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
       const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
       if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
       __syncwarp();
-      const int jm = j % 3;
-      int page = jm == 0 ? pid0 : (jm == 1 ? pid1 : pid2);
+      int page;
+      if (!is_v) {
+        pid_v = pid_v_next;
+        pid_v_next = pid_k;
+        page = pid_k;
+      } else {
+        page = (j == n - 1) ? pid_v_next : pid_v;
+      }
       if (lane < nbox) {
         const int row = (n0 + lane * p.box_h) % p.ps;
         if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
@@ -552,10 +638,16 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
         for (int c = 0; c < C::DCH; ++c)
           tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, row, page);
       }
-      if (!is_v && j + 1 < n) {
-        const int nx = tile_page_id(p, w, j + 1, C::BN, lane);
-        const int jn = (j + 1) % 3;
-        if (jn == 0) pid0 = nx; else if (jn == 1) pid1 = nx; else pid2 = nx;
+      if (!is_v) {
+        if (j + 1 < n) {
+          pid_k = tile_page_id(p, w, j + 1, C::BN, lane);
+        } else {
+          WorkItem nw;
+          if (items.peek(nw) && item_tiles(nw, C::BN) > 0) {
+            pid_next = tile_page_id(p, nw, 0, C::BN, lane);
+            have_next = true;
+          }
+        }
       }
       ++ld_idx;
     }
@@ -579,11 +671,14 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, false, true);
   uint32_t ld_idx = 0, g_base = 0, q_cnt = 0;
   bool ok = true;
-  for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-    const WorkItem w = unpack_item(p.items, it, p.tpb);
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+  while (ok && items.next(w)) {
     const int n = item_tiles(w, C::BN);
     if (n == 0) continue;
-    if (!mbar_wait(bar0 + 8 * C::B_QFULL, q_cnt & 1, abort)) { ok = false; break; }
+    const uint32_t qb = q_cnt % C::QBUF;
+    const uint32_t sQb = sQ + qb * C::Q_BYTES;
+    if (!mbar_wait(bar0 + 8 * (C::B_QFULL + qb), (q_cnt / C::QBUF) & 1, abort)) { ok = false; break; }
     tc_fence_after();
     for (int s = 0; s < 2 * n; ++s) {
       int j;
@@ -601,14 +696,14 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
         // S[sb] = Q K^T: K-major A (Q) and B (K), 16 columns of D per MMA
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(sQ + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024);
+          const uint64_t ad = smem_desc_sw128(sQb + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024);
           const uint64_t bd =
               smem_desc_sw128(slot_addr + (kk >> 2) * C::SLOT_CHUNK + (kk & 3) * 32, 16, 1024);
           mma_ss(tmem + sb * C::BN, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar0 + 8 * (C::B_SFULL + sb));
         tc_commit(bar0 + 8 * (C::B_KVEMPTY + slot));
-        if (j == n - 1) tc_commit(bar0 + 8 * C::B_QEMPTY);
+        if (j == n - 1) tc_commit(bar0 + 8 * (C::B_QEMPTY + qb));
       } else {
         if (!mbar_wait(bar0 + 8 * (C::B_PFULL + sb), (g >> 1) & 1, abort)) { ok = false; break; }
         if (j == 0 && !mbar_wait(bar0 + 8 * C::B_OEMPTY, (q_cnt & 1) ^ 1, abort)) {
@@ -648,8 +743,9 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
   const int G = p.G;
   uint32_t g_base = 0, ld_base = 0;
   bool ok = true;
-  for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-    const WorkItem w = unpack_item(p.items, it, p.tpb);
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+  while (ok && items.next(w)) {
     const int n = item_tiles(w, BN);
     const int n_rows = w.n_tok * G;
     const bool real = r < n_rows;
@@ -854,16 +950,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;             // 1024-B aligned for SW128
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t sQ = base;
-  const uint32_t sKV = base + C::Q_BYTES;
+  const uint32_t sKV = base + C::QBUF * C::Q_BYTES;
   const uint32_t bar0 = sKV + C::NSLOT * C::SLOT_BYTES;
-  uint8_t* bar_ptr = smem + C::Q_BYTES + C::NSLOT * C::SLOT_BYTES;
+  uint8_t* bar_ptr = smem + C::QBUF * C::Q_BYTES + C::NSLOT * C::SLOT_BYTES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NBAR);
   volatile int* abort = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 4);
 
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    mbar_init(bar0 + 8 * C::B_QFULL, 1);
-    mbar_init(bar0 + 8 * C::B_QEMPTY, 1);
+    for (int i = 0; i < C::QBUF; ++i) {
+      mbar_init(bar0 + 8 * (C::B_QFULL + i), 1);
+      mbar_init(bar0 + 8 * (C::B_QEMPTY + i), 1);
+    }
     for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(bar0 + 8 * (C::B_KVFULL + i), 1);
       mbar_init(bar0 + 8 * (C::B_KVEMPTY + i), 1);
