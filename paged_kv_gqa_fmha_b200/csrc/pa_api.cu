@@ -82,7 +82,16 @@ struct pa_plan {
 
 namespace {
 
-int kv_tile(int D) { return D == 256 ? 64 : 128; }
+int kv_tile(int D) {
+  return D == 64 ? pa::TileCfg<64>::BN : (D == 128 ? pa::TileCfg<128>::BN : pa::TileCfg<256>::BN);
+}
+
+// CTAs of the persistent attention grid: one or two per SM depending on D.
+int attn_grid(int D, int n_sm) {
+  const int c = D == 64 ? pa::TileCfg<64>::CTAS
+                        : (D == 128 ? pa::TileCfg<128>::CTAS : pa::TileCfg<256>::CTAS);
+  return c * n_sm;
+}
 
 int auto_smax(int B, int Hkv, int n_sm) {
   const long units = (long)B * Hkv;
@@ -157,7 +166,7 @@ cudaError_t launch_attention(int n_sm, cudaStream_t st, const CUtensorMap& tq,
                              const CUtensorMap& tk, const CUtensorMap& tv,
                              const pa::AttnParams& ap) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_sm);
+  cfg.gridDim = dim3(pa::TileCfg<D>::CTAS * n_sm);
   cfg.blockDim = dim3(pa::kThreads);
   cfg.dynamicSmemBytes = pa::TileCfg<D>::SMEM_BYTES;
   cfg.stream = st;
@@ -434,7 +443,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.tpb = p->tpb;
   sp.S_max = p->num_splits == 1 ? 1 : p->S_max;
   sp.forced_splits = p->num_splits > 1 ? p->num_splits : 0;
-  sp.n_ctas = p->n_sm;
+  sp.n_ctas = attn_grid(p->D, p->n_sm);
   pa::pa_schedule_kernel<<<1, pa::kCostBuckets, 0, st>>>(sp);
 
   pa::AttnParams ap;
@@ -704,7 +713,7 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   sp.tpb = tpb;
   sp.S_max = 1;             // no KV splits on this path
   sp.forced_splits = 0;
-  sp.n_ctas = nd->n_sm;
+  sp.n_ctas = attn_grid(head_dim, nd->n_sm);
   pa::pa_schedule_kernel<<<1, pa::kCostBuckets, 0, st>>>(sp);
 
   pa::AttnParams ap;

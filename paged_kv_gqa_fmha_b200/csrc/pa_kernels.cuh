@@ -114,18 +114,26 @@ constexpr int kSchedSmemReqs = 4096;  // unit offsets of up to this many request
 constexpr int kMaxSplits = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows > 2^8
 
+// Tile configuration per head dimension.  D = 64 and 128 run two CTAs per SM
+// (64-key tiles, 256 TMEM columns, ~100 KB of shared memory each): two
+// independent load -> S -> softmax -> P V chains per SM hide each other's
+// latencies, which one CTA per SM cannot.  D = 256 needs the whole SM.
 template <int D>
 struct TileCfg {
-  static constexpr int BN = (D == 256) ? 64 : 128;   // keys per KV tile
+  static constexpr int CTAS = (D == 256) ? 1 : 2;      // CTAs per SM
+  // 14 warps on 4 sub-partitions: at most 4 warps x 32 lanes x 128 = 16 K registers each
+  static constexpr int MAXREG = (CTAS == 2) ? 128 : 255;
+  static constexpr int BN = 64;                       // keys per KV tile
   static constexpr int DCH = D / 64;                  // 128-byte column chunks per row
   static constexpr int Q_CHUNK = kBM * 128;           // bytes of one Q column chunk
   static constexpr int Q_BYTES = kBM * D * 2;
   static constexpr int SLOT_CHUNK = BN * 128;         // bytes of one K/V column chunk
   static constexpr int SLOT_BYTES = BN * D * 2;
-  static constexpr int QBUF = (D == 256) ? 1 : 2;      // Q tiles in flight
-  static constexpr int NSLOT = (D == 64) ? 12 : 5;
+  static constexpr int QBUF = (D == 64) ? 2 : 1;      // Q tiles in flight
+  static constexpr int NSLOT = (D == 64) ? 8 : (D == 128 ? 4 : 5);
   static constexpr int O_COL = 2 * BN;                // TMEM: S0 [0,BN), S1 [BN,2BN), O
-  static constexpr int TMEM_COLS = 512;
+  static constexpr int TMEM_COLS = (O_COL + D <= 256) ? 256 : 512;
+  static constexpr int OCH = (CTAS == 2) ? 1 : 2;     // 32-column O chunks per TMEM wait
   // barriers: q_full[QBUF], q_empty[QBUF], kv_full[NSLOT], kv_empty[NSLOT], s_full[2],
   //           p_full[2], pv_done[2], o_empty, drain
   static constexpr int B_QFULL = 0, B_QEMPTY = QBUF, B_KVFULL = 2 * QBUF,
@@ -136,6 +144,7 @@ struct TileCfg {
   static constexpr int SMEM_BYTES = 1024 + QBUF * Q_BYTES + NSLOT * SLOT_BYTES + BAR_BYTES;
   static_assert(NBAR * 8 + 16 <= BAR_BYTES, "barrier area");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(CTAS == 1 || 2 * SMEM_BYTES <= 228 * 1024, "two CTAs per SM");
   static_assert(O_COL + D <= TMEM_COLS, "TMEM columns");
 };
 
@@ -813,14 +822,15 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
           tc_fence_after();
           const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
 #pragma unroll 1
-          for (int c = 0; c < D / 32; c += 2) {
-            uint32_t v[2][32];
-            tmem_ld32(trow + C::O_COL + c * 32, v[0]);
-            tmem_ld32(trow + C::O_COL + c * 32 + 32, v[1]);
-            tmem_ld_wait(v[0]);
-            reg_tie(v[1]);
+          for (int c = 0; c < D / 32; c += C::OCH) {
+            uint32_t v[C::OCH][32];
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
+            for (int h2 = 0; h2 < C::OCH; ++h2) tmem_ld32(trow + C::O_COL + (c + h2) * 32, v[h2]);
+            tmem_ld_wait(v[0]);
+#pragma unroll
+            for (int h2 = 1; h2 < C::OCH; ++h2) reg_tie(v[h2]);
+#pragma unroll
+            for (int h2 = 0; h2 < C::OCH; ++h2) {
 #pragma unroll
               for (int e = 0; e < 32; ++e)
                 v[h2][e] = __float_as_uint(__uint_as_float(v[h2][e]) * alpha);
@@ -892,15 +902,16 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       const float lse_v = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; c += 2) {
-        uint32_t vv[2][32];
-        tmem_ld32(trow + C::O_COL + c * 32, vv[0]);
-        tmem_ld32(trow + C::O_COL + c * 32 + 32, vv[1]);
+      for (int c = 0; c < D / 32; c += C::OCH) {
+        uint32_t vv[C::OCH][32];
+#pragma unroll
+        for (int h2 = 0; h2 < C::OCH; ++h2) tmem_ld32(trow + C::O_COL + (c + h2) * 32, vv[h2]);
         tmem_ld_wait(vv[0]);
-        reg_tie(vv[1]);
+#pragma unroll
+        for (int h2 = 1; h2 < C::OCH; ++h2) reg_tie(vv[h2]);
         if (real) {
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
+          for (int h2 = 0; h2 < C::OCH; ++h2) {
             const uint32_t* v = vv[h2];
             if (split) {
               float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + (c + h2) * 32);
@@ -940,7 +951,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(TileCfg<D>::MAXREG)
     pa_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
