@@ -168,6 +168,15 @@ PA_API size_t pa_workspace_bytes(const pa_plan *plan);
 /* Largest number of KV splits this plan can use for one request. */
 PA_API int pa_max_splits(const pa_plan *plan);
 
+/* Prefill kernel choice for head_dim 64/128.  0 (default): every query block
+ * runs on the one-stage kernel (two CTAs per SM).  1: requests with two or more
+ * 128-row query blocks run on the two-stage kernel, which pairs consecutive
+ * blocks of one KV head so that each K/V tile feeds 256 query rows (half the
+ * K/V reads); it is correct on every geometry it accepts but currently slower
+ * than the one-stage kernel.  May reallocate the workspace; call it outside
+ * graph capture.  PA_ERR_UNSUPPORTED for head_dim 256. */
+PA_API int pa_set_two_stage_prefill(pa_plan *plan, int on);
+
 /* Kernel timing for benchmarks.  pa_profile_start makes the next `max_runs`
  * (1..4096) calls of pa_run record a CUDA event pair on their stream around
  * the attention kernel.  pa_profile_read synchronises on those events, writes
@@ -196,7 +205,7 @@ PA_API int pa_profile_read(pa_plan *plan, float *attn_ms, int *n_runs, int *laun
  * array of PA_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU which loads the
  * library holds until the process exits.  A geometry whose worst-case work
  * list does not fit (batch * heads_kv * ceil(capacity * page_size * G / 128)
- * items of 32 bytes, plus 40 bytes per request and a small header) is
+ * items of 32 bytes, plus 44 bytes per request and a small header) is
  * rejected with PA_ERR_UNSUPPORTED and a message saying so.  KV splitting is
  * not used on this path (each (request, KV head, query block) is one item),
  * so there is no split merge and no partial-state storage.

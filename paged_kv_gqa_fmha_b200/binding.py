@@ -26,7 +26,8 @@ STATUS_TIMEOUT = 1 << 4
 
 EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_scale",
            "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
-           "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc")
+           "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc",
+           "pa_set_two_stage_prefill")
 
 # Size of the library's static scratch array used by pa_run_noalloc.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -74,6 +75,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_profile_start.restype = I
     lib.pa_profile_read.argtypes = [P, ctypes.POINTER(F), ctypes.POINTER(I), ctypes.POINTER(I)]
     lib.pa_profile_read.restype = I
+    lib.pa_set_two_stage_prefill.argtypes = [P, I]
+    lib.pa_set_two_stage_prefill.restype = I
     lib.pa_run_noalloc.argtypes = [I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P]
     lib.pa_run_noalloc.restype = I
     if path == LIB_PATH:
@@ -119,6 +122,9 @@ class Plan:
 
     def set_num_splits(self, n: int):
         _check(self._lib.pa_set_num_splits(self._h, int(n)))
+
+    def set_two_stage_prefill(self, on: bool):
+        _check(self._lib.pa_set_two_stage_prefill(self._h, 1 if on else 0))
 
     def set_scale(self, s: float):
         _check(self._lib.pa_set_scale(self._h, float(s)))

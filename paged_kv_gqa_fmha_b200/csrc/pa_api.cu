@@ -17,6 +17,7 @@
 
 #include "../../include/pa.h"
 #include "pa_kernels.cuh"
+#include "pa_prefill.cuh"
 
 namespace {
 
@@ -68,7 +69,13 @@ struct pa_plan {
   int4* req_aux;
   int* unit_off;
   int* split_list;
+  int* unit_off2;
   pa::PackedItem* items;
+  pa::PackedItem* items2;     // query-block pairs (two-stage prefill kernel)
+  int max_items2;
+  bool use_pairs;             // head_dim <= 128: prefill runs on the two-stage kernel
+  int last_launches;          // kernels the last pa_run enqueued
+  int box_h2;                 // page box height of the two-stage kernel (BN = 128)
   float* part_lse;
   float* part_o;
   // attention-kernel timing (pa_profile_*)
@@ -78,6 +85,7 @@ struct pa_plan {
   const void* tm_ptr[3];
   int tm_num_pages;
   CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_k2, tm_v2;   // page boxes of box_h2 rows
 };
 
 namespace {
@@ -113,6 +121,7 @@ int alloc_workspace(pa_plan* p) {
     return PA_ERR_UNSUPPORTED;
   }
   (void)G;
+  const long max_items2 = p->use_pairs ? (long)p->B * p->Hkv * ((blocks_per_req + 1) / 2) : 0;
   const size_t n_part_rows = p->S_max > 1 ? (size_t)p->B * p->Hkv * p->S_max * pa::kBM : 0;
   size_t off = 0;
   const size_t o_hdr = off; off = align_up(off + sizeof(pa::WsHeader), 256);
@@ -121,6 +130,8 @@ int alloc_workspace(pa_plan* p) {
   const size_t o_uoff = off; off = align_up(off + sizeof(int) * (size_t)(p->B + 1), 256);
   const size_t o_split = off; off = align_up(off + sizeof(int) * (size_t)p->B, 256);
   const size_t o_items = off; off = align_up(off + sizeof(pa::PackedItem) * (size_t)max_items, 256);
+  const size_t o_uoff2 = off; off = align_up(off + sizeof(int) * (size_t)(p->B + 1), 256);
+  const size_t o_items2 = off; off = align_up(off + sizeof(pa::PackedItem) * (size_t)max_items2, 256);
   const size_t o_plse = off; off = align_up(off + sizeof(float) * n_part_rows, 256);
   const size_t o_po = off; off = align_up(off + sizeof(float) * n_part_rows * p->D, 256);
   void* ws = nullptr;
@@ -145,6 +156,9 @@ int alloc_workspace(pa_plan* p) {
   p->unit_off = reinterpret_cast<int*>(c + o_uoff);
   p->split_list = reinterpret_cast<int*>(c + o_split);
   p->items = reinterpret_cast<pa::PackedItem*>(c + o_items);
+  p->unit_off2 = reinterpret_cast<int*>(c + o_uoff2);
+  p->items2 = reinterpret_cast<pa::PackedItem*>(c + o_items2);
+  p->max_items2 = (int)max_items2;
   p->part_lse = reinterpret_cast<float*>(c + o_plse);
   p->part_o = reinterpret_cast<float*>(c + o_po);
   p->max_items = (int)max_items;
@@ -153,9 +167,31 @@ int alloc_workspace(pa_plan* p) {
 
 template <int D>
 cudaError_t set_smem_attr() {
-  return cudaFuncSetAttribute(pa::pa_attention_kernel<D>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              pa::TileCfg<D>::SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(pa::pa_attention_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       pa::TileCfg<D>::SMEM_BYTES);
+  if constexpr (D <= 128) {
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(pa::pa_pair_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               pa::PairCfg<D>::SMEM_BYTES);
+  }
+  return e;
+}
+
+template <int D>
+cudaError_t launch_pairs(int n_sm, cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& tk,
+                         const CUtensorMap& tv, const pa::AttnParams& ap) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_sm);
+  cfg.blockDim = dim3(pa::PairCfg<D>::THREADS);
+  cfg.dynamicSmemBytes = pa::PairCfg<D>::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pa::pa_pair_kernel<D>, tq, tk, tv, ap);
 }
 
 // The attention kernel and the merge are programmatic dependents of the
@@ -247,6 +283,13 @@ int build_maps(pa_plan* p, const void* q, const void* k, const void* v) {
     if (rc) return rc;
     rc = encode(&p->tm_v, v, 4, dims, str, box, "v_pool");
     if (rc) return rc;
+    if (p->use_pairs) {
+      cuuint32_t box2[4] = {64, 1, (cuuint32_t)p->box_h2, 1};
+      rc = encode(&p->tm_k2, k, 4, dims, str, box2, "k_pool");
+      if (rc) return rc;
+      rc = encode(&p->tm_v2, v, 4, dims, str, box2, "v_pool");
+      if (rc) return rc;
+    }
   }
   p->tm_ptr[0] = q;
   p->tm_ptr[1] = k;
@@ -324,6 +367,9 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->BN = kv_tile(head_dim);
   p->tpb = pa::kBM / G;
   p->box_h = page_size < p->BN ? page_size : p->BN;
+  p->use_pairs = false;       // pa_set_two_stage_prefill turns it on (head_dim <= 128)
+  p->last_launches = 2;
+  p->box_h2 = page_size < 128 ? page_size : 128;
   p->S_max = auto_smax(batch, heads_kv, n_sm);
   p->ws = nullptr;
   p->prof_ev = nullptr;
@@ -437,6 +483,11 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.req_aux = p->req_aux;
   sp.unit_off = p->unit_off;
   sp.split_list = p->split_list;
+  // without cu_q_lens every request is one decode token: no query-block pairs
+  const bool pairs = p->use_pairs && cu_q_lens != nullptr;
+  sp.items2 = pairs ? p->items2 : nullptr;
+  sp.unit_off2 = p->unit_off2;
+  sp.max_items2 = p->max_items2;
   sp.hdr = p->hdr;
   sp.max_items = p->max_items;
   sp.B = p->B; sp.Hkv = p->Hkv; sp.G = p->G; sp.C = p->C; sp.ps = p->ps; sp.BN = p->BN;
@@ -465,7 +516,17 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.scale_log2 = p->scale * 1.4426950408889634f;
   const bool prof = p->prof_on && p->prof_n < p->prof_cap;
   if (prof) cudaEventRecord(p->prof_ev[2 * p->prof_n], st);
-  cudaError_t le = launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, ap);
+  cudaError_t le = cudaSuccess;
+  if (pairs) {
+    // query-block pairs (prefill) first, on the two-stage kernel
+    pa::AttnParams ap2 = ap;
+    ap2.items = p->items2;
+    ap2.box_h = p->box_h2;
+    le = p->D == 64 ? launch_pairs<64>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, ap2)
+                    : launch_pairs<128>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, ap2);
+  }
+  if (le == cudaSuccess)
+    le = launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, ap);
   if (prof) {
     cudaEventRecord(p->prof_ev[2 * p->prof_n + 1], st);
     ++p->prof_n;
@@ -486,10 +547,32 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     set_err("pa_run: launch failed: %s", cudaGetErrorString(le));
     return PA_ERR_CUDA;
   }
+  p->last_launches = 2 + (pairs ? 1 : 0) + (sp.S_max > 1 ? 1 : 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_err("pa_run: launch failed: %s", cudaGetErrorString(e));
     return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+int pa_set_two_stage_prefill(pa_plan* p, int on) {
+  if (!p) { set_err("pa_set_two_stage_prefill: NULL plan"); return PA_ERR_INVALID; }
+  if (on && p->D > 128) {
+    set_err("pa_set_two_stage_prefill: head_dim %d has no two-stage kernel (64 and 128 only)",
+            p->D);
+    return PA_ERR_UNSUPPORTED;
+  }
+  const bool want = on != 0;
+  if (want != p->use_pairs) {
+    const bool old = p->use_pairs;
+    p->use_pairs = want;
+    int rc = alloc_workspace(p);
+    if (rc != PA_OK) {
+      p->use_pairs = old;
+      return rc;
+    }
+    p->tm_num_pages = -1;   // rebuild tensor maps (two-stage boxes)
   }
   return PA_OK;
 }
@@ -535,7 +618,8 @@ int pa_profile_read(pa_plan* p, float* attn_ms, int* n_runs, int* launches_per_r
   }
   *attn_ms = total;
   *n_runs = p->prof_n;
-  if (launches_per_run) *launches_per_run = (p->num_splits != 1 && p->S_max > 1) ? 3 : 2;
+  if (launches_per_run)
+    *launches_per_run = p->last_launches;
   p->prof_on = 0;
   p->prof_n = 0;
   return PA_OK;
@@ -639,7 +723,8 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   const size_t o_aux = align_up(o_req + sizeof(int4) * (size_t)batch, 256);
   const size_t o_uoff = align_up(o_aux + sizeof(int4) * (size_t)batch, 256);
   const size_t o_split = align_up(o_uoff + sizeof(int) * (size_t)(batch + 1), 256);
-  const size_t o_items = align_up(o_split + sizeof(int) * (size_t)batch, 256);
+  const size_t o_uoff2 = align_up(o_split + sizeof(int) * (size_t)batch, 256);
+  const size_t o_items = align_up(o_uoff2 + sizeof(int) * (size_t)(batch + 1), 256);
   const size_t need = o_items + sizeof(pa::PackedItem) * (size_t)max_items;
   if (max_items > (1L << 30) || need > (size_t)PA_NOALLOC_SCRATCH_BYTES) {
     set_err("pa_run_noalloc: this geometry needs %zu bytes of scratch (%ld work items); the "
@@ -704,6 +789,9 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   sp.cu_q_lens = cu_q_lens;
   sp.items = reinterpret_cast<pa::PackedItem*>(base + o_items);
   sp.split_list = reinterpret_cast<int*>(base + o_split);
+  sp.items2 = nullptr;      // every request on the one-stage kernel
+  sp.unit_off2 = reinterpret_cast<int*>(base + o_uoff2);
+  sp.max_items2 = 0;
   sp.req_info = reinterpret_cast<int4*>(base + o_req);
   sp.req_aux = reinterpret_cast<int4*>(base + o_aux);
   sp.unit_off = reinterpret_cast<int*>(base + o_uoff);

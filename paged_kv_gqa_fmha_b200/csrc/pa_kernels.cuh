@@ -101,7 +101,8 @@ struct WsHeader {
   unsigned status;
   int n_items;
   int n_split_reqs;   // requests split over KV (entries of the split list)
-  int pad[61];
+  int n_items2;       // items of the query-block-pair list (two-stage prefill kernel)
+  int pad[60];
 };
 
 constexpr int kBM = 128;              // query rows per tile (tcgen05 M)
@@ -199,6 +200,9 @@ struct SchedParams {
   const int* seq_lens;
   const int* cu_q_lens;
   PackedItem* items;
+  PackedItem* items2;  // pairs of query blocks, or nullptr when pairs are not used
+  int* unit_off2;      // [B + 1] exclusive prefix sum of pair units
+  int max_items2;
   int* split_list;     // [B] requests with more than one split
   int4* req_info;      // [B] {n_splits, q_len, t_base, kv_len}
   int4* req_aux;       // [B] {units, tiles per split, KV tiles of the single block, 0}
@@ -363,15 +367,18 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
   __syncthreads();
   const int chunk = s_chunk;
 
-  // 2.
+  // 2.  A request with two or more query blocks goes to the pair list when the
+  // two-stage prefill kernel is in use (items2 != nullptr): one unit per pair of
+  // consecutive blocks.  Every other request goes to the main list.
   __shared__ int s_nsplit;
   __shared__ int s_uoff[kSchedSmemReqs + 1];
+  __shared__ int s_uoff2[kSchedSmemReqs + 1];
   if (tid == 0) s_nsplit = 0;
   __syncthreads();
-  int running = 0;
+  int running = 0, running2 = 0;
   for (int b0 = 0; b0 < p.B; b0 += blockDim.x) {
     const int b = b0 + tid;
-    int units = 0;
+    int units = 0, units2 = 0;
     if (b < p.B) {
       const ReqInfo r = read_request(p, b);
       const int nb = n_qblocks(r.q_len, p.tpb);
@@ -384,27 +391,71 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
         per = ceil_div(tiles, sp);
         ns = ceil_div(tiles, per);
       }
-      units = ns > 1 ? ns : nb;
+      if (p.items2 != nullptr && ns == 1 && nb >= 2) units2 = (nb + 1) / 2;
+      else units = ns > 1 ? ns : nb;
       p.req_info[b] = make_int4(ns, r.q_len, r.t_base, r.kv_len);
       p.req_aux[b] = make_int4(units, per, tiles, 0);
       if (ns > 1) p.split_list[atomicAdd(&s_nsplit, 1)] = b;
     }
-    int total;
+    int total, total2;
     const int off = block_scan_1024(units, warp_sums, &total);
+    const int off2 = block_scan_1024(units2, warp_sums, &total2);
     if (b < p.B) {
       p.unit_off[b] = running + off;
-      if (b < kSchedSmemReqs) s_uoff[b] = running + off;
+      p.unit_off2[b] = running2 + off2;
+      if (b < kSchedSmemReqs) {
+        s_uoff[b] = running + off;
+        s_uoff2[b] = running2 + off2;
+      }
     }
     running += total;
+    running2 += total2;
   }
   if (tid == 0) {
     p.unit_off[p.B] = running;
-    if (p.B <= kSchedSmemReqs) s_uoff[p.B] = running;
+    p.unit_off2[p.B] = running2;
+    if (p.B <= kSchedSmemReqs) {
+      s_uoff[p.B] = running;
+      s_uoff2[p.B] = running2;
+    }
     p.hdr->n_split_reqs = s_nsplit;
+    const int n2 = running2 * p.Hkv;
+    p.hdr->n_items2 = n2 < p.max_items2 ? n2 : p.max_items2;
   }
   __syncthreads();
   const int U = running;
   const int* uoff = p.B <= kSchedSmemReqs ? s_uoff : p.unit_off;
+  const int U2 = running2;
+  const int* uoff2 = p.B <= kSchedSmemReqs ? s_uoff2 : p.unit_off2;
+
+  // 2b.  Pair list: each request's pairs stay together, last pair (most keys)
+  // first; a unit writes its Hkv items (one per KV head) at consecutive places.
+  for (int u0 = 0; u0 < U2; u0 += blockDim.x) {
+    const int u = u0 + tid;
+    if (u < U2) {
+      int lo = 0, hi = p.B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (uoff2[mid] <= u) lo = mid; else hi = mid - 1;
+      }
+      const int b = lo;
+      const int4 ri = p.req_info[b];
+      const int k = u - uoff2[b];
+      const int units2 = uoff2[b + 1] - uoff2[b];
+      const int pair = units2 - 1 - k;
+      const int q0 = 2 * pair * p.tpb;
+      const int ntok = min(2 * p.tpb, ri.y - q0);
+      const int hi_kv = block_kv_hi(ri.y, ri.w, q0, ntok);
+      const int pos = u * p.Hkv;
+      for (int g = 0; g < p.Hkv; ++g) {
+        if (pos + g < p.max_items2) {
+          PackedItem* dst = p.items2 + pos + g;
+          dst->a = make_int4(b, g | (1 << 24), q0, ri.z);
+          dst->c = make_int4(0, hi_kv, ri.w, ri.y);
+        }
+      }
+    }
+  }
 
   // 3.  Ordering.  A request with several query blocks (prefill) keeps its
   // units together, last block (most keys) first, and the block of units is
@@ -564,6 +615,14 @@ __device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const Att
       if (lane == 0) mbar_arrive(qfull);
     }
     ++q_cnt;
+    // Q is read once, so it always comes from DRAM: pull the next item's Q
+    // tile into L2 now so that its load is short when its turn comes.
+    WorkItem nw;
+    if (lane == 0 && items.peek(nw) && item_tiles(nw, C::BN) > 0 && nw.n_tok == p.tpb) {
+      const int tn = nw.t_base + nw.q_tok0;
+      if (tn + p.tpb <= T)
+        for (int c = 0; c < C::DCH; ++c) tma_prefetch_l2_3d(tm_q, c * 64, nw.kvh * G, tn);
+    }
   }
   if (*abort && lane == 0) {
     for (uint32_t k = q_cnt > (uint32_t)C::QBUF ? q_cnt - C::QBUF : 0; k < q_cnt; ++k)

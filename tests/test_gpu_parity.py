@@ -68,6 +68,20 @@ def test_decode_without_cu_q_lens():
     compare(out, lse, *oracle_all(w))
 
 
+@pytest.mark.parametrize("D,ps,G", [(128, 16, 4), (128, 64, 1), (64, 32, 8), (128, 128, 3)])
+def test_two_stage_prefill_kernel(D, ps, G):
+    """The optional two-stage kernel (query-block pairs) against the oracle,
+    with odd block counts, partial pairs, chunked prefill and decode rows in
+    the same batch (those stay on the one-stage kernel)."""
+    spec = W.custom_spec("pairs", 2 * G, 2, D, ps, [300, 1, 129, 77, 5], [300, 700, 400, 77, 900])
+    w = gen(spec, 30 + D + ps + G)
+    plan = make_plan(w)
+    plan.set_two_stage_prefill(True)
+    out, lse, _ = gpu_run(w, plan)
+    assert plan.status() == 0
+    compare(out, lse, *oracle_all(w))
+
+
 # ------------------------------------------------------------------ split-KV (a8)
 @pytest.mark.parametrize("splits", [1, 2, 7, 0])
 def test_split_invariance(splits):
