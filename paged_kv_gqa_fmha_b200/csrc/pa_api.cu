@@ -369,7 +369,7 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->box_h = page_size < p->BN ? page_size : p->BN;
   p->use_pairs = false;       // pa_set_two_stage_prefill turns it on (head_dim <= 128)
   p->last_launches = 2;
-  p->box_h2 = page_size < 128 ? page_size : 128;
+  p->box_h2 = page_size < pa::PairCfg<128>::BN ? page_size : pa::PairCfg<128>::BN;
   p->S_max = auto_smax(batch, heads_kv, n_sm);
   p->ws = nullptr;
   p->prof_ev = nullptr;

@@ -11,51 +11,56 @@
 // "[Perf][FA4] Warm up dense (paged) FA4 attention kernels" (vLLM PR #48156,
 // review thread) describes, written here from that description.
 //
+// Q lives in tensor memory.  Q is read once per item, so it always comes from
+// DRAM; with one CTA per SM a Q tile held in shared memory for the whole item
+// would leave either no room to load the next item's Q early or too little
+// room for the K/V ring.  Here the Q loader fills a shared-memory staging
+// buffer, the softmax warps copy their stage's rows into TMEM at the start of
+// the item and release the staging buffer at once, so the next item's Q loads
+// while the current item runs.  S = Q K^T then takes A from TMEM.
+//
 // Roles (11 warps, one CTA per SM):
-//   warps 0-3   softmax / correction / epilogue of stage A (one thread per row)
+//   warps 0-3   stage A: Q copy to TMEM, softmax, correction, epilogue
 //   warps 4-7   the same for stage B
 //   warp  8     K/V producer (page-table-driven TMA, order K0 V0 K1 V1 ...)
 //   warp  9     MMA issuer (one thread)
-//   warp  10    Q loader (both stages' Q tiles)
-// TMEM (512 columns): S_A [0, BN), S_B [BN, 2BN), O_A [2BN, 2BN + D), O_B after.
+//   warp  10    Q loader
+// TMEM (512 columns): S_A, S_B (BN each), O_A, O_B (D each), Q_A, Q_B (D/2 each).
 // Each stage has a single S buffer: S_X(j+1) is issued after P_X(j) V(j), so
 // the completion of S_X(j+1) also guarantees that P_X(j) V(j) has completed.
 #pragma once
 
 #include "pa_kernels.cuh"
 
-#ifndef PA_PAIR_QBUF
-#define PA_PAIR_QBUF 1
-#endif
-
 namespace pa {
 
 template <int D>
 struct PairCfg {
   static_assert(D == 64 || D == 128, "two-stage kernel: head_dim 64 or 128");
-  static constexpr int BN = 128;
+  static constexpr int BN = 64;
   static constexpr int DCH = D / 64;
   static constexpr int Q_CHUNK = kBM * 128;
   static constexpr int Q_BYTES = kBM * D * 2;          // one stage
   static constexpr int SLOT_CHUNK = BN * 128;
   static constexpr int SLOT_BYTES = BN * D * 2;
-  static constexpr int QBUF = PA_PAIR_QBUF;             // pairs of Q tiles in flight
-  static constexpr int NSLOT = (D == 64) ? (QBUF == 2 ? 8 : 12) : (QBUF == 2 ? 3 : 5);
+  static constexpr int NSLOT = (D == 64) ? 16 : 10;
   static constexpr int S_COL = 0;                      // + stage * BN
   static constexpr int O_COL = 2 * BN;                 // + stage * D
+  static constexpr int Q_COL = 2 * BN + 2 * D;         // + stage * D / 2
   static constexpr int TMEM_COLS = 512;
   static constexpr int THREADS = 352;
   static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, Q_WARP = 10;
-  // barriers: q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full[2], p_full[2],
-  //           pv_done[2], o_empty[2], drain
-  static constexpr int B_QFULL = 0, B_QEMPTY = QBUF, B_KVFULL = 2 * QBUF,
-                       B_KVEMPTY = 2 * QBUF + NSLOT, B_SFULL = 2 * QBUF + 2 * NSLOT, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
-                       B_OEMPTY = B_PVDONE + 2, B_DRAIN = B_OEMPTY + 2, NBAR = B_DRAIN + 1;
+  // barriers: q_full, q_smem_empty, q_tmem[2], kv_full[NSLOT], kv_empty[NSLOT],
+  //           s_full[2], p_full[2], pv_done[2], o_empty[2], drain
+  static constexpr int B_QFULL = 0, B_QSMEM = 1, B_QTMEM = 2, B_KVFULL = 4,
+                       B_KVEMPTY = 4 + NSLOT, B_SFULL = 4 + 2 * NSLOT, B_PFULL = B_SFULL + 2,
+                       B_PVDONE = B_PFULL + 2, B_OEMPTY = B_PVDONE + 2, B_DRAIN = B_OEMPTY + 2,
+                       NBAR = B_DRAIN + 1;
   static constexpr int BAR_BYTES = 512;
-  static constexpr int SMEM_BYTES = 1024 + 2 * QBUF * Q_BYTES + NSLOT * SLOT_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + 2 * Q_BYTES + NSLOT * SLOT_BYTES + BAR_BYTES;
   static_assert(NBAR * 8 + 16 <= BAR_BYTES, "barrier area");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static_assert(O_COL + 2 * D <= TMEM_COLS, "TMEM columns");
+  static_assert(Q_COL + D <= TMEM_COLS, "TMEM columns");
 };
 
 // Tokens of the two stages and KV tiles each needs.
@@ -95,10 +100,10 @@ __device__ __forceinline__ void pair_q_loader(const CUtensorMap* tm_q, const Att
   while (items.next(w)) {
     const PairShape ps = pair_shape(w, p.tpb, C::BN);
     if (ps.n == 0) continue;
-    const uint32_t qb = q_cnt % C::QBUF;
-    if (!warp_wait(bar0 + 8 * (C::B_QEMPTY + qb), ((q_cnt / C::QBUF) & 1) ^ 1, abort)) break;
-    const uint32_t qfull = bar0 + 8 * (C::B_QFULL + qb);
-    const uint32_t sQb = sQ + qb * 2 * C::Q_BYTES;
+    // the staging buffer is free once all eight softmax warps copied the last Q
+    if (!warp_wait(bar0 + 8 * C::B_QSMEM, (q_cnt & 1) ^ 1, abort)) break;
+    const uint32_t qfull = bar0 + 8 * C::B_QFULL;
+    const uint32_t sQb = sQ;
     bool tma[2];
     uint32_t tma_bytes = 0;
     for (int x = 0; x < 2; ++x) {
@@ -160,10 +165,7 @@ __device__ __forceinline__ void pair_q_loader(const CUtensorMap* tm_q, const Att
       }
     }
   }
-  if (*abort && lane == 0) {
-    for (uint32_t k = q_cnt > (uint32_t)C::QBUF ? q_cnt - C::QBUF : 0; k < q_cnt; ++k)
-      mbar_drain(bar0 + 8 * (C::B_QFULL + k % C::QBUF), (k / C::QBUF) & 1);
-  }
+  if (*abort && lane == 0 && q_cnt > 0) mbar_drain(bar0 + 8 * C::B_QFULL, (q_cnt - 1) & 1);
 }
 
 // K/V producer: tile j of an item is loaded as K_j then V_j (load index 2j and
@@ -251,16 +253,16 @@ __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUt
 //   S_A(0), S_B(0)
 //   for j: P_A(j) V(j); S_A(j+1); P_B(j) V(j); S_B(j+1)
 // so the tensor core works on one stage while the other stage's softmax runs.
+// S_X = Q_X K^T with Q_X read from TMEM; P_X V with P_X read from TMEM.
 template <int D>
-__device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint32_t sKV,
-                                         uint32_t bar0, uint32_t tmem, int n_items,
-                                         volatile int* abort) {
+__device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sKV, uint32_t bar0,
+                                         uint32_t tmem, int n_items, volatile int* abort) {
   using C = PairCfg<D>;
   constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, C::BN, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, false, true);
-  uint32_t ld_base = 0, q_cnt = 0;
+  uint32_t ld_base = 0;
   uint32_t g[2] = {0, 0};     // tiles processed per stage (phase counters)
-  uint32_t itc[2] = {0, 0};   // items per stage that had tiles (o_empty phases)
+  uint32_t itc[2] = {0, 0};   // items per stage that had tiles (q_tmem / o_empty phases)
   bool ok = true;
   ItemStream items(p.items, n_items, p.tpb);
   WorkItem w;
@@ -271,14 +273,14 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
     tc_fence_after();
     return true;
   };
-  auto issue_s = [&](int x, uint32_t k_idx, uint32_t qX) {
+  auto issue_s = [&](int x, uint32_t k_idx) {
     const uint32_t slot_addr = sKV + (k_idx % C::NSLOT) * C::SLOT_BYTES;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t ad = smem_desc_sw128(qX + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024);
       const uint64_t bd =
           smem_desc_sw128(slot_addr + (kk >> 2) * C::SLOT_CHUNK + (kk & 3) * 32, 16, 1024);
-      mma_ss(tmem + C::S_COL + x * C::BN, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+      mma_ts(tmem + C::S_COL + x * C::BN, tmem + C::Q_COL + x * (D / 2) + kk * 8, bd, kIdescS,
+             kk > 0 ? 1u : 0u);
     }
     tc_commit(bar0 + 8 * (C::B_SFULL + x));
   };
@@ -297,17 +299,16 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
     const PairShape ps = pair_shape(w, p.tpb, C::BN);
     const int n = ps.n;
     if (n == 0) continue;
-    const uint32_t qb = q_cnt % C::QBUF;
-    const uint32_t sQb = sQ + qb * 2 * C::Q_BYTES;
-    const uint32_t qempty = bar0 + 8 * (C::B_QEMPTY + qb);
-    if (!mbar_wait(bar0 + 8 * (C::B_QFULL + qb), (q_cnt / C::QBUF) & 1, abort)) { ok = false; break; }
+    // Q of each working stage copied into TMEM by its softmax warps
+    for (int x = 0; x < 2 && ok; ++x)
+      if (ps.nt[x] > 0 && !mbar_wait(bar0 + 8 * (C::B_QTMEM + x), itc[x] & 1, abort)) ok = false;
+    if (!ok) break;
     tc_fence_after();
     // tile 0: S of both stages
     if (!kv_wait(ld_base)) { ok = false; break; }
     for (int x = 0; x < 2; ++x)
-      if (ps.nt[x] > 0) issue_s(x, ld_base, sQb + x * C::Q_BYTES);
+      if (ps.nt[x] > 0) issue_s(x, ld_base);
     tc_commit(bar0 + 8 * (C::B_KVEMPTY + ld_base % C::NSLOT));
-    if (n == 1) tc_commit(qempty);
     for (int j = 0; j < n && ok; ++j) {
       const uint32_t v_idx = ld_base + 2 * j + 1, k_next = ld_base + 2 * j + 2;
       if (!kv_wait(v_idx)) { ok = false; break; }
@@ -328,11 +329,8 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
             if (!kv_wait(k_next)) { ok = false; break; }
             k_ready = true;
           }
-          if (j + 1 < ps.nt[x]) issue_s(x, k_next, sQb + x * C::Q_BYTES);
-          if (x == 1) {
-            tc_commit(bar0 + 8 * (C::B_KVEMPTY + k_next % C::NSLOT));
-            if (j + 2 == n) tc_commit(qempty);
-          }
+          if (j + 1 < ps.nt[x]) issue_s(x, k_next);
+          if (x == 1) tc_commit(bar0 + 8 * (C::B_KVEMPTY + k_next % C::NSLOT));
         }
       }
     }
@@ -341,7 +339,6 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
       if (ps.nt[x] > 0) ++itc[x];
     }
     ld_base += 2 * n;
-    ++q_cnt;
   }
   tc_commit(bar0 + 8 * C::B_DRAIN);
   mbar_drain(bar0 + 8 * C::B_DRAIN, 0);
@@ -352,8 +349,9 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
 // P is stored (fewer live registers); P_X(j-1) V(j-1) has completed by then
 // because S_X(j), whose completion was awaited, was issued after it.
 template <int D>
-__device__ __forceinline__ void pair_softmax(const AttnParams& p, uint32_t sKV, uint32_t bar0,
-                                             uint32_t tmem, int n_items, volatile int* abort) {
+__device__ __forceinline__ void pair_softmax(const AttnParams& p, uint32_t sQ, uint32_t sKV,
+                                             uint32_t bar0, uint32_t tmem, int n_items,
+                                             volatile int* abort) {
   using C = PairCfg<D>;
   constexpr int BN = C::BN;
   const int x = threadIdx.x >> 7;
@@ -363,7 +361,7 @@ __device__ __forceinline__ void pair_softmax(const AttnParams& p, uint32_t sKV, 
   const uint32_t s_col = C::S_COL + x * BN, o_col = C::O_COL + x * D;
   const uint32_t sfull = bar0 + 8 * (C::B_SFULL + x), pfull = bar0 + 8 * (C::B_PFULL + x);
   const int G = p.G;
-  uint32_t g = 0, ld_base = 0;
+  uint32_t g = 0, ld_base = 0, q_cnt = 0;
   bool ok = true;
   ItemStream items(p.items, n_items, p.tpb);
   WorkItem w;
@@ -377,6 +375,38 @@ __device__ __forceinline__ void pair_softmax(const AttnParams& p, uint32_t sKV, 
     const int q_first = w.q_tok0 + x * p.tpb;
     const int t = w.t_base + q_first + r / G;
     const int h = w.kvh * G + r % G;
+    if (n > 0) {
+      // Q: copy this stage's rows from the staging buffer into TMEM (bf16
+      // pairs, element 2c in the low half of column c, as the MMA reads A),
+      // then release the staging buffer.  Every softmax warp arrives, so the
+      // release completes only after both stages copied.
+      if (!warp_wait(bar0 + 8 * C::B_QFULL, q_cnt & 1, abort)) { ok = false; break; }
+      if (nt > 0 && warp_active) {
+        const uint32_t src = sQ + x * C::Q_BYTES + r * 128;
+#pragma unroll
+        for (int h32 = 0; h32 < D / 64; ++h32) {
+          uint32_t qv[32];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t a = src + h32 * C::Q_CHUNK + ((u ^ (r & 7)) << 4);
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(qv[4 * u]), "=r"(qv[4 * u + 1]), "=r"(qv[4 * u + 2]),
+                           "=r"(qv[4 * u + 3])
+                         : "r"(a));
+          }
+          tmem_st32(trow + C::Q_COL + x * (D / 2) + h32 * 32, qv);
+        }
+        tmem_st_wait();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar0 + 8 * C::B_QSMEM);
+        if (nt > 0) mbar_arrive(bar0 + 8 * (C::B_QTMEM + x));
+      }
+      ++q_cnt;
+    }
     if (tok > 0 && nt == 0) {
       // no key is visible to any row of this stage: O = 0, LSE = -inf
       if (real) {
@@ -529,18 +559,18 @@ __global__ void __maxnreg__(168)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t sQ = base;
-  const uint32_t sKV = base + 2 * C::QBUF * C::Q_BYTES;
+  const uint32_t sKV = base + 2 * C::Q_BYTES;
   const uint32_t bar0 = sKV + C::NSLOT * C::SLOT_BYTES;
-  uint8_t* bar_ptr = smem + 2 * C::QBUF * C::Q_BYTES + C::NSLOT * C::SLOT_BYTES;
+  uint8_t* bar_ptr = smem + 2 * C::Q_BYTES + C::NSLOT * C::SLOT_BYTES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NBAR);
   volatile int* abort = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 4);
 
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::QBUF; ++i) {
-      mbar_init(bar0 + 8 * (C::B_QFULL + i), 1);
-      mbar_init(bar0 + 8 * (C::B_QEMPTY + i), 1);
-    }
+    mbar_init(bar0 + 8 * C::B_QFULL, 1);
+    mbar_init(bar0 + 8 * C::B_QSMEM, 8);
+    mbar_init(bar0 + 8 * (C::B_QTMEM + 0), 4);
+    mbar_init(bar0 + 8 * (C::B_QTMEM + 1), 4);
     for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(bar0 + 8 * (C::B_KVFULL + i), 1);
       mbar_init(bar0 + 8 * (C::B_KVEMPTY + i), 1);
@@ -577,10 +607,10 @@ __global__ void __maxnreg__(168)
   } else if (warp == C::Q_WARP) {
     pair_q_loader<D>(&tm_q, p, sQ, bar0, n_items, abort);
   } else if (warp == C::MMA_WARP) {
-    if ((threadIdx.x & 31) == 0) pair_mma<D>(p, sQ, sKV, bar0, tmem, n_items, abort);
+    if ((threadIdx.x & 31) == 0) pair_mma<D>(p, sKV, bar0, tmem, n_items, abort);
     __syncwarp();
   } else {
-    pair_softmax<D>(p, sKV, bar0, tmem, n_items, abort);
+    pair_softmax<D>(p, sQ, sKV, bar0, tmem, n_items, abort);
   }
 
   tc_fence_before();
