@@ -82,9 +82,11 @@ struct pa_plan {
   cudaEvent_t* prof_ev;
   int prof_cap, prof_n, prof_on;
   // tensor-map cache
-  const void* tm_ptr[3];
+  const void* tm_ptr[4];       // q, k_pool, v_pool, out the maps were encoded for
   int tm_num_pages;
   CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_o;            // out, box (32, G, 32 / G), 64-byte swizzle
+  int o_tma;                   // tm_o is used (G divides 32)
   CUtensorMap tm_k2, tm_v2;   // page boxes of box_h2 rows
 };
 
@@ -200,7 +202,7 @@ cudaError_t launch_pairs(int n_sm, cudaStream_t st, const CUtensorMap& tq, const
 template <int D>
 cudaError_t launch_attention(int n_sm, cudaStream_t st, const CUtensorMap& tq,
                              const CUtensorMap& tk, const CUtensorMap& tv,
-                             const pa::AttnParams& ap) {
+                             const CUtensorMap& to, const pa::AttnParams& ap) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pa::TileCfg<D>::CTAS * n_sm);
   cfg.blockDim = dim3(pa::kThreads);
@@ -211,16 +213,16 @@ cudaError_t launch_attention(int n_sm, cudaStream_t st, const CUtensorMap& tq,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, pa::pa_attention_kernel<D>, tq, tk, tv, ap);
+  return cudaLaunchKernelEx(&cfg, pa::pa_attention_kernel<D>, tq, tk, tv, to, ap);
 }
 
 cudaError_t launch_attention_d(int D, int n_sm, cudaStream_t st, const CUtensorMap& tq,
                                const CUtensorMap& tk, const CUtensorMap& tv,
-                               const pa::AttnParams& ap) {
+                               const CUtensorMap& to, const pa::AttnParams& ap) {
   switch (D) {
-    case 64: return launch_attention<64>(n_sm, st, tq, tk, tv, ap);
-    case 128: return launch_attention<128>(n_sm, st, tq, tk, tv, ap);
-    default: return launch_attention<256>(n_sm, st, tq, tk, tv, ap);
+    case 64: return launch_attention<64>(n_sm, st, tq, tk, tv, to, ap);
+    case 128: return launch_attention<128>(n_sm, st, tq, tk, tv, to, ap);
+    default: return launch_attention<256>(n_sm, st, tq, tk, tv, to, ap);
   }
 }
 
@@ -239,7 +241,8 @@ cudaError_t launch_merge(int n_sm, cudaStream_t st, const pa::MergeParams& mp) {
 }
 
 int encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
-           const cuuint64_t* strides, const cuuint32_t* box, const char* what) {
+           const cuuint64_t* strides, const cuuint32_t* box, const char* what,
+           CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     set_err("pa: cuTensorMapEncodeTiled is not available from the driver");
@@ -247,7 +250,7 @@ int encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
   }
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_err("pa: cuTensorMapEncodeTiled(%s) failed with %d", what, (int)r);
@@ -256,8 +259,8 @@ int encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
   return PA_OK;
 }
 
-int build_maps(pa_plan* p, const void* q, const void* k, const void* v) {
-  if (p->tm_ptr[0] == q && p->tm_ptr[1] == k && p->tm_ptr[2] == v &&
+int build_maps(pa_plan* p, const void* q, const void* k, const void* v, void* out) {
+  if (p->tm_ptr[0] == q && p->tm_ptr[1] == k && p->tm_ptr[2] == v && p->tm_ptr[3] == out &&
       p->tm_num_pages == p->num_pages)
     return PA_OK;
   const cuuint64_t e = 2;  // bytes per bf16
@@ -271,6 +274,13 @@ int build_maps(pa_plan* p, const void* q, const void* k, const void* v) {
     cuuint32_t box[3] = {64, (cuuint32_t)p->G, (cuuint32_t)p->tpb};
     int rc = encode(&p->tm_q, q, 3, dims, str, box, "q");
     if (rc) return rc;
+    // out has q's layout; a softmax warp stores its 32 rows = 32 / G whole tokens
+    p->o_tma = (32 % p->G == 0) ? 1 : 0;
+    if (p->o_tma) {
+      cuuint32_t obox[3] = {32, (cuuint32_t)p->G, (cuuint32_t)(32 / p->G)};
+      rc = encode(&p->tm_o, out, 3, dims, str, obox, "out", CU_TENSOR_MAP_SWIZZLE_64B);
+      if (rc) return rc;
+    }
   }
   // pools [P, ps, Hkv, D]: dims (D, Hkv, ps, P); box (64, 1, box_h, 1).
   {
@@ -294,6 +304,7 @@ int build_maps(pa_plan* p, const void* q, const void* k, const void* v) {
   p->tm_ptr[0] = q;
   p->tm_ptr[1] = k;
   p->tm_ptr[2] = v;
+  p->tm_ptr[3] = out;
   p->tm_num_pages = p->num_pages;
   return PA_OK;
 }
@@ -374,7 +385,8 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->ws = nullptr;
   p->prof_ev = nullptr;
   p->prof_cap = p->prof_n = p->prof_on = 0;
-  p->tm_ptr[0] = p->tm_ptr[1] = p->tm_ptr[2] = nullptr;
+  p->tm_ptr[0] = p->tm_ptr[1] = p->tm_ptr[2] = p->tm_ptr[3] = nullptr;
+  p->o_tma = 0;
   p->tm_num_pages = -1;
   if (alloc_workspace(p) != PA_OK) {
     delete p;
@@ -471,7 +483,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     set_err("pa_run: current device %d is not the plan's device %d", dev, p->device);
     return PA_ERR_INVALID;
   }
-  int rc = build_maps(p, q, k_pool, v_pool);
+  int rc = build_maps(p, q, k_pool, v_pool, out);
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
@@ -513,6 +525,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.S_max = p->S_max;
   ap.tpb = p->tpb;
   ap.box_h = p->box_h;
+  ap.o_tma = p->o_tma;
   ap.scale_log2 = p->scale * 1.4426950408889634f;
   const bool prof = p->prof_on && p->prof_n < p->prof_cap;
   if (prof) cudaEventRecord(p->prof_ev[2 * p->prof_n], st);
@@ -526,7 +539,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
                     : launch_pairs<128>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, ap2);
   }
   if (le == cudaSuccess)
-    le = launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, ap);
+    le = launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, p->tm_o, ap);
   if (prof) {
     cudaEventRecord(p->prof_ev[2 * p->prof_n + 1], st);
     ++p->prof_n;
@@ -820,9 +833,12 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   ap.S_max = 1;
   ap.tpb = tpb;
   ap.box_h = box_h;
+  ap.o_tma = 0;   // no map of out here: every block stores O directly
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)head_dim);
   ap.scale_log2 = sc * 1.4426950408889634f;
-  e = launch_attention_d(head_dim, nd->n_sm, st, tm_q, tm_k, tm_v, ap);
+  CUtensorMap tm_none;
+  memset(&tm_none, 0, sizeof(tm_none));
+  e = launch_attention_d(head_dim, nd->n_sm, st, tm_q, tm_k, tm_v, tm_none, ap);
   if (e != cudaSuccess) {
     set_err("pa_run_noalloc: launch failed: %s", cudaGetErrorString(e));
     return PA_ERR_CUDA;

@@ -4,7 +4,7 @@
 //   1. pa_schedule_kernel: reads seq_lens / cu_q_lens on the device and writes
 //      a work list (one item per (request, KV head, 128-row query block, KV
 //      split)), longest first, plus per-request split counts.
-//   2. pa_attention_kernel<D>: persistent, one CTA per SM, warp-specialised:
+//   2. pa_attention_kernel<D>: persistent (two CTAs per SM for D <= 128), warp-specialised:
 //        warps 0-3  softmax / correction / epilogue (one thread per query row)
 //        warp  4    producer: page-table-driven TMA gathers of K and V pages
 //        warp  5    MMA issuer: tcgen05 S = Q K^T and O += P V, TMEM accumulators
@@ -142,10 +142,15 @@ struct TileCfg {
                        B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2, B_OEMPTY = B_PVDONE + 2,
                        B_DRAIN = B_OEMPTY + 1, NBAR = B_DRAIN + 1;
   static constexpr int BAR_BYTES = 512;
-  static constexpr int SMEM_BYTES = 1024 + QBUF * Q_BYTES + NSLOT * SLOT_BYTES + BAR_BYTES;
+  // epilogue staging: per softmax warp 32 rows x 32 columns of bf16 (64-byte
+  // swizzle); D = 256 has no room for it next to its five K/V slots
+  static constexpr int EPI_WARP_BYTES = 32 * 64;
+  static constexpr int EPI_BYTES = (D == 256) ? 0 : 4 * EPI_WARP_BYTES;
+  static constexpr int SMEM_BYTES =
+      1024 + QBUF * Q_BYTES + NSLOT * SLOT_BYTES + EPI_BYTES + BAR_BYTES;
   static_assert(NBAR * 8 + 16 <= BAR_BYTES, "barrier area");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static_assert(CTAS == 1 || 2 * SMEM_BYTES <= 228 * 1024, "two CTAs per SM");
+  static_assert(CTAS == 1 || 2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
   static_assert(O_COL + D <= TMEM_COLS, "TMEM columns");
 };
 
@@ -161,6 +166,7 @@ struct AttnParams {
   float* part_lse;            // [B*Hkv*S_max*128]
   unsigned* status;
   int B, Hq, Hkv, G, C, ps, num_pages, S_max, tpb, box_h;
+  int o_tma;                  // 1: full blocks store O through the tensor map of out
   float scale_log2;
 };
 
@@ -801,7 +807,8 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
 }
 
 template <int D>
-__device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, uint32_t bar0,
+__device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const AttnParams& p,
+                                             uint32_t sKV, uint32_t sEpi, uint32_t bar0,
                                              uint32_t tmem, int n_items, volatile int* abort) {
   using C = TileCfg<D>;
   constexpr int BN = C::BN;
@@ -809,6 +816,8 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
   const int warp = r >> 5, lane = r & 31;
   const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);   // this warp's lanes
   const int G = p.G;
+  const int T = p.cu_q_lens ? __ldg(p.cu_q_lens + p.B) : p.B;
+  const uint32_t sEpiW = sEpi + warp * C::EPI_WARP_BYTES;
   uint32_t g_base = 0, ld_base = 0;
   bool ok = true;
   ItemStream items(p.items, n_items, p.tpb);
@@ -960,6 +969,10 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
     if (warp_active) {
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       const float lse_v = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      // whole blocks of 32 / G tokens per warp go out through TMA stores
+      const bool o_tma = C::EPI_BYTES > 0 && !split && p.o_tma && w.n_tok == p.tpb &&
+                         w.t_base + w.q_tok0 + p.tpb <= T;
+      const int t_w0 = w.t_base + w.q_tok0 + warp * (32 / G);
 #pragma unroll 1
       for (int c = 0; c < D / 32; c += C::OCH) {
         uint32_t vv[C::OCH][32];
@@ -980,6 +993,29 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
                                      __uint_as_float(v[4 * e + 1]) * inv_l,
                                      __uint_as_float(v[4 * e + 2]) * inv_l,
                                      __uint_as_float(v[4 * e + 3]) * inv_l);
+            } else if (o_tma) {
+              // 32 rows x 32 columns staged in the 64-byte swizzle of the out
+              // tensor map, then written by one TMA store per warp (full
+              // 64-byte row pieces instead of one 16-byte piece per row)
+              if (lane == 0) bulk_wait_read_all();   // previous store has read the buffer
+              __syncwarp();
+              const uint32_t row_addr = sEpiW + lane * 64;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint32_t a = row_addr + ((e ^ ((lane >> 1) & 3)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                             "r"(pack_bf16x2(__uint_as_float(v[8 * e + 0]) * inv_l, __uint_as_float(v[8 * e + 1]) * inv_l)),
+                             "r"(pack_bf16x2(__uint_as_float(v[8 * e + 2]) * inv_l, __uint_as_float(v[8 * e + 3]) * inv_l)),
+                             "r"(pack_bf16x2(__uint_as_float(v[8 * e + 4]) * inv_l, __uint_as_float(v[8 * e + 5]) * inv_l)),
+                             "r"(pack_bf16x2(__uint_as_float(v[8 * e + 6]) * inv_l, __uint_as_float(v[8 * e + 7]) * inv_l))
+                             : "memory");
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(tm_o, sEpiW, (c + h2) * 32, w.kvh * G, t_w0);
+                bulk_commit_group();
+              }
             } else {
               uint4* dst =
                   reinterpret_cast<uint4*>(p.out + ((size_t)t * p.Hq + h) * D + (c + h2) * 32);
@@ -1007,13 +1043,15 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sKV, 
     g_base += n;
     ld_base += 2 * n;
   }
+  if (lane == 0) bulk_wait_all();   // O stores complete before the CTA exits
 }
 
 template <int D>
 __global__ void __maxnreg__(TileCfg<D>::MAXREG)
     pa_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_o, const AttnParams p) {
   using C = TileCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -1021,8 +1059,9 @@ __global__ void __maxnreg__(TileCfg<D>::MAXREG)
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t sQ = base;
   const uint32_t sKV = base + C::QBUF * C::Q_BYTES;
-  const uint32_t bar0 = sKV + C::NSLOT * C::SLOT_BYTES;
-  uint8_t* bar_ptr = smem + C::QBUF * C::Q_BYTES + C::NSLOT * C::SLOT_BYTES;
+  const uint32_t sEpi = sKV + C::NSLOT * C::SLOT_BYTES;
+  const uint32_t bar0 = sEpi + C::EPI_BYTES;
+  uint8_t* bar_ptr = smem + C::QBUF * C::Q_BYTES + C::NSLOT * C::SLOT_BYTES + C::EPI_BYTES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NBAR);
   volatile int* abort = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 4);
 
@@ -1072,7 +1111,7 @@ __global__ void __maxnreg__(TileCfg<D>::MAXREG)
     if ((threadIdx.x & 31) == 0) mma_role<D>(p, sQ, sKV, bar0, tmem, n_items, abort);
     __syncwarp();
   } else {
-    softmax_role<D>(p, sKV, bar0, tmem, n_items, abort);
+    softmax_role<D>(&tm_o, p, sKV, sEpi, bar0, tmem, n_items, abort);
   }
 
   tc_fence_before();
