@@ -75,7 +75,7 @@ struct pa_plan {
   int max_items2;
   bool use_pairs;             // head_dim <= 128: prefill runs on the two-stage kernel
   int last_launches;          // kernels the last pa_run enqueued
-  int box_h2;                 // page box height of the two-stage kernel (BN = 128)
+  int box_h2;                 // page box height of the two-stage kernel
   float* part_lse;
   float* part_o;
   // attention-kernel timing (pa_profile_*)
@@ -182,7 +182,7 @@ cudaError_t set_smem_attr() {
 
 template <int D>
 cudaError_t launch_pairs(int n_sm, cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& tk,
-                         const CUtensorMap& tv, const pa::AttnParams& ap) {
+                         const CUtensorMap& tv, const CUtensorMap& to, const pa::AttnParams& ap) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_sm);
   cfg.blockDim = dim3(pa::PairCfg<D>::THREADS);
@@ -193,7 +193,7 @@ cudaError_t launch_pairs(int n_sm, cudaStream_t st, const CUtensorMap& tq, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, pa::pa_pair_kernel<D>, tq, tk, tv, ap);
+  return cudaLaunchKernelEx(&cfg, pa::pa_pair_kernel<D>, tq, tk, tv, to, ap);
 }
 
 // The attention kernel and the merge are programmatic dependents of the
@@ -535,8 +535,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     pa::AttnParams ap2 = ap;
     ap2.items = p->items2;
     ap2.box_h = p->box_h2;
-    le = p->D == 64 ? launch_pairs<64>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, ap2)
-                    : launch_pairs<128>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, ap2);
+    le = p->D == 64 ? launch_pairs<64>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, p->tm_o, ap2)
+                    : launch_pairs<128>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, p->tm_o, ap2);
   }
   if (le == cudaSuccess)
     le = launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, p->tm_o, ap);
