@@ -172,10 +172,22 @@ PA_API int pa_max_splits(const pa_plan *plan);
  * runs on the one-stage kernel (two CTAs per SM).  1: requests with two or more
  * 128-row query blocks run on the two-stage kernel, which pairs consecutive
  * blocks of one KV head so that each K/V tile feeds 256 query rows (half the
- * K/V reads); it is correct on every geometry it accepts but currently slower
- * than the one-stage kernel.  May reallocate the workspace; call it outside
- * graph capture.  PA_ERR_UNSUPPORTED for head_dim 256. */
+ * K/V reads) and keeps two score buffers per block.  May reallocate the
+ * workspace; call it outside graph capture.  PA_ERR_UNSUPPORTED for head_dim
+ * 256. */
 PA_API int pa_set_two_stage_prefill(pa_plan *plan, int on);
+
+/* Decode kernel choice for runs with cu_q_lens == NULL (one query token per
+ * request) and at most 32 query heads per KV head.  The decode kernel computes
+ * S^T = K Q^T and O^T = V^T P^T with the 128 keys of a tile as the MMA's M
+ * dimension and the G query rows (padded to 16 or 32) as N -- the same online
+ * softmax ("FlashAttention", Dao et al., Algorithm 1) with 1/8 to 1/4 of the
+ * tensor work of 128-row query tiles.  Default: head_dim 128 runs on it,
+ * head_dim 256 on the one-stage kernel.  on = 1: head_dim 128 and 256 run on
+ * it.  on = 0: every such run uses the one-stage kernel.  The two paths agree
+ * within the stated tolerances, not bit for bit.  Takes effect at the next
+ * pa_run; no reallocation.  PA_ERR_INVALID for a NULL plan. */
+PA_API int pa_set_decode_kernel(pa_plan *plan, int on);
 
 /* Kernel timing for benchmarks.  pa_profile_start makes the next `max_runs`
  * (1..4096) calls of pa_run record a CUDA event pair on their stream around

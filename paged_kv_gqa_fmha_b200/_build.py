@@ -7,6 +7,7 @@ runtime is linked statically, so the library only needs the NVIDIA driver.
 """
 from __future__ import annotations
 
+import glob
 import os
 import shutil
 import subprocess
@@ -17,8 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpa_b200.so")
 SOURCES = [os.path.join(CSRC, "pa_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_kernels.cuh", "sm100.cuh")] + [
-    os.path.join(ROOT, "include", "pa.h")]
+DEPS = sorted(glob.glob(os.path.join(CSRC, "*"))) + [os.path.join(ROOT, "include", "pa.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

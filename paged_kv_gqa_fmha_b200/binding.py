@@ -27,7 +27,7 @@ STATUS_TIMEOUT = 1 << 4
 EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_scale",
            "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
            "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc",
-           "pa_set_two_stage_prefill")
+           "pa_set_two_stage_prefill", "pa_set_decode_kernel")
 
 # Size of the library's static scratch array used by pa_run_noalloc.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -77,6 +77,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_profile_read.restype = I
     lib.pa_set_two_stage_prefill.argtypes = [P, I]
     lib.pa_set_two_stage_prefill.restype = I
+    lib.pa_set_decode_kernel.argtypes = [P, I]
+    lib.pa_set_decode_kernel.restype = I
     lib.pa_run_noalloc.argtypes = [I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P]
     lib.pa_run_noalloc.restype = I
     if path == LIB_PATH:
@@ -125,6 +127,12 @@ class Plan:
 
     def set_two_stage_prefill(self, on: bool):
         _check(self._lib.pa_set_two_stage_prefill(self._h, 1 if on else 0))
+
+    def set_decode_kernel(self, on: bool):
+        """Decode-only runs (cu_q_lens None): True puts head_dim 128 and 256 on
+        the keys-as-M decode kernel, False puts both on the one-stage kernel
+        (default: head_dim 128 on the decode kernel, 256 on the one-stage)."""
+        _check(self._lib.pa_set_decode_kernel(self._h, 1 if on else 0))
 
     def set_scale(self, s: float):
         _check(self._lib.pa_set_scale(self._h, float(s)))

@@ -18,6 +18,7 @@
 #include "../../include/pa.h"
 #include "pa_kernels.cuh"
 #include "pa_prefill.cuh"
+#include "pa_decode.cuh"
 
 namespace {
 
@@ -86,6 +87,7 @@ struct pa_plan {
   int tm_num_pages;
   CUtensorMap tm_q, tm_k, tm_v;
   CUtensorMap tm_o;            // out, box (32, G, 32 / G), 64-byte swizzle
+  int use_dec;                 // decode kernel: -1 head_dim 128 only (default), 1 128 and 256, 0 never
   int o_tma;                   // tm_o is used (G divides 32)
   CUtensorMap tm_k2, tm_v2;   // page boxes of box_h2 rows
 };
@@ -167,6 +169,13 @@ int alloc_workspace(pa_plan* p) {
   return PA_OK;
 }
 
+template <int D, int RR>
+cudaError_t set_decode_smem_attr() {
+  return cudaFuncSetAttribute(pa::pa_decode_kernel<D, RR>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              pa::DecCfg<D, pa::DecRows<RR>::NR>::SMEM_BYTES);
+}
+
 template <int D>
 cudaError_t set_smem_attr() {
   cudaError_t e = cudaFuncSetAttribute(pa::pa_attention_kernel<D>,
@@ -177,7 +186,46 @@ cudaError_t set_smem_attr() {
       e = cudaFuncSetAttribute(pa::pa_pair_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                pa::PairCfg<D>::SMEM_BYTES);
   }
+  if constexpr (D >= 128) {
+    if (e == cudaSuccess) e = set_decode_smem_attr<D, 4>();
+    if (e == cudaSuccess) e = set_decode_smem_attr<D, 8>();
+    if (e == cudaSuccess) e = set_decode_smem_attr<D, 16>();
+    if (e == cudaSuccess) e = set_decode_smem_attr<D, 32>();
+  }
   return e;
+}
+
+// Decode-only runs: G query rows per (request, KV head), RR = G rounded up.
+template <int D, int RR>
+cudaError_t launch_decode_rr(int n_sm, cudaStream_t st, const CUtensorMap& tk,
+                             const CUtensorMap& tv, const pa::AttnParams& ap) {
+  using C = pa::DecCfg<D, pa::DecRows<RR>::NR>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_sm);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pa::pa_decode_kernel<D, RR>, tk, tv, ap);
+}
+
+template <int D>
+cudaError_t launch_decode_d(int G, int n_sm, cudaStream_t st, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const pa::AttnParams& ap) {
+  if (G <= 4) return launch_decode_rr<D, 4>(n_sm, st, tk, tv, ap);
+  if (G <= 8) return launch_decode_rr<D, 8>(n_sm, st, tk, tv, ap);
+  if (G <= 16) return launch_decode_rr<D, 16>(n_sm, st, tk, tv, ap);
+  return launch_decode_rr<D, 32>(n_sm, st, tk, tv, ap);
+}
+
+cudaError_t launch_decode(int D, int G, int n_sm, cudaStream_t st, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const pa::AttnParams& ap) {
+  return D == 128 ? launch_decode_d<128>(G, n_sm, st, tk, tv, ap)
+                  : launch_decode_d<256>(G, n_sm, st, tk, tv, ap);
 }
 
 template <int D>
@@ -387,6 +435,7 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->prof_cap = p->prof_n = p->prof_on = 0;
   p->tm_ptr[0] = p->tm_ptr[1] = p->tm_ptr[2] = p->tm_ptr[3] = nullptr;
   p->o_tma = 0;
+  p->use_dec = -1;
   p->tm_num_pages = -1;
   if (alloc_workspace(p) != PA_OK) {
     delete p;
@@ -506,7 +555,11 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.tpb = p->tpb;
   sp.S_max = p->num_splits == 1 ? 1 : p->S_max;
   sp.forced_splits = p->num_splits > 1 ? p->num_splits : 0;
-  sp.n_ctas = attn_grid(p->D, p->n_sm);
+  // decode-only runs (one query token per request) with up to 32 query heads
+  // per KV head go to the keys-as-M decode kernel (one CTA per SM)
+  const bool dec = cu_q_lens == nullptr && p->G <= 32 &&
+                   ((p->use_dec == -1 && p->D == 128) || (p->use_dec == 1 && p->D >= 128));
+  sp.n_ctas = dec ? p->n_sm : attn_grid(p->D, p->n_sm);
   pa::pa_schedule_kernel<<<1, pa::kCostBuckets, 0, st>>>(sp);
 
   pa::AttnParams ap;
@@ -539,7 +592,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
                     : launch_pairs<128>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, p->tm_o, ap2);
   }
   if (le == cudaSuccess)
-    le = launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, p->tm_o, ap);
+    le = dec ? launch_decode(p->D, p->G, p->n_sm, st, p->tm_k, p->tm_v, ap)
+             : launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, p->tm_o, ap);
   if (prof) {
     cudaEventRecord(p->prof_ev[2 * p->prof_n + 1], st);
     ++p->prof_n;
@@ -566,6 +620,12 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     set_err("pa_run: launch failed: %s", cudaGetErrorString(e));
     return PA_ERR_CUDA;
   }
+  return PA_OK;
+}
+
+int pa_set_decode_kernel(pa_plan* p, int on) {
+  if (!p) { set_err("pa_set_decode_kernel: NULL plan"); return PA_ERR_INVALID; }
+  p->use_dec = on ? 1 : 0;
   return PA_OK;
 }
 

@@ -1,0 +1,619 @@
+// pa_decode.cuh -- decode attention with keys on the MMA's M side (sm_100a,
+// head_dim 128/256, G <= 32 query heads per KV head, one query token per request).
+//
+// In decode a (request, KV head) pair has only G query rows (G = Hq / Hkv),
+// so a 128-row query tile would spend 128/G times the useful tensor work and
+// the power that goes with it.  Here the products are transposed so that the
+// 128 keys of a tile fill the MMA's M dimension and the G rows (padded to NR =
+// 16 or 32) are its N dimension:
+//   S^T = K Q^T          M = 128 keys, N = NR rows, K = D   (A = K tile, B = Q)
+//   O^T += V^T P^T       M = 128 of D, N = NR rows, K = 128 keys
+//                        (A = V tile read MN-major, B = P^T written by softmax)
+// The online softmax of "FlashAttention" (Dao et al., Algorithm 1) then runs
+// across threads: thread t owns key t of the tile (TMEM lane t of S^T) and
+// d = t of every 128-wide half of O^T.  Row maxima are block reductions per
+// tile; row sums stay per thread and are reduced once in the epilogue, which
+// is exact because every thread rescales its partial sum by the same factor.
+//
+// Roles (8 warps, one CTA per SM):
+//   warps 0-3  softmax / correction / epilogue
+//   warps 4, 7 K/V producers (page-table-driven TMA, order K0 K1 V0 K2 V1 ...);
+//              warp 4 issues the even loads of that order, warp 7 the odd ones:
+//              one issuing warp per SM does not keep HBM busy with page-sized boxes
+//   warp  5    MMA issuer (warp-collective issue)
+//   warp  6    Q loader (Q tiles of NR rows, double-buffered where room allows)
+#pragma once
+
+#include "pa_kernels.cuh"
+
+namespace pa {
+
+template <int D, int NR>
+struct DecCfg {
+  static_assert(D == 128 || D == 256, "decode kernel: head_dim 128 or 256");
+  static_assert(NR == 16 || NR == 32, "decode kernel: 16 or 32 padded rows");
+  static constexpr int BN = 128;                      // keys per tile (M of S^T)
+  static constexpr int DCH = D / 64;                  // 128-byte column chunks of a K/V row
+  static constexpr int DH = D / 128;                  // M = 128 halves of O^T
+  static constexpr int SLOT_CHUNK = BN * 128;         // one 64-column chunk of a K/V tile
+  static constexpr int SLOT_BYTES = BN * D * 2;
+  static constexpr int NSLOT = (D == 128) ? 6 : 3;
+  static constexpr int Q_CHUNK = NR * 128;            // Q tile: NR rows x 64 columns per chunk
+  static constexpr int Q_BYTES = NR * D * 2;
+  static constexpr int QBUF = (D == 256 && NR == 32) ? 1 : 2;   // Q tiles in flight
+  static constexpr int P_CHUNK = NR * 128;            // P^T: NR rows x 64 keys per chunk
+  static constexpr int P_BYTES = NR * BN * 2;
+  static constexpr int RED_BYTES = 3 * 4 * NR * 4;    // row maxima of 4 warps (two tiles), row sums
+  static constexpr int S_COL = 0;                     // + buffer * NR
+  static constexpr int O_COL = 2 * NR;                // + half * NR
+  static constexpr int TMEM_USED = O_COL + DH * NR;
+  static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : (TMEM_USED <= 64 ? 64 : 128);
+  static constexpr int THREADS = 256;
+  static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5, Q_WARP = 6, PRODUCER2_WARP = 7;
+  // barriers: q_full[2], q_empty[2], kv_full[NSLOT], kv_empty[NSLOT], s_full[2],
+  //           p_full[2], pv_done[2], o_empty, drain, red[2] (row maxima), red_sum
+  static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NSLOT,
+                       B_SFULL = 4 + 2 * NSLOT, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
+                       B_OEMPTY = B_PVDONE + 2, B_DRAIN = B_OEMPTY + 1, B_RED = B_DRAIN + 1,
+                       B_REDSUM = B_RED + 2, NBAR = B_REDSUM + 1;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + NSLOT * SLOT_BYTES + QBUF * Q_BYTES + 2 * P_BYTES +
+                                    RED_BYTES + BAR_BYTES;
+  static_assert(NBAR * 8 + 16 <= BAR_BYTES, "barrier area");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(TMEM_USED <= TMEM_COLS, "TMEM columns");
+};
+
+// Q loader: the NR-row Q tile of each item (rows past G * n_tok are left as
+// they are; they only feed columns of S^T and O^T that are never read).
+template <int D, int NR>
+__device__ __forceinline__ void dec_q_loader(const AttnParams& p, uint32_t sQ, uint32_t bar0,
+                                             int n_items, volatile int* abort) {
+  using C = DecCfg<D, NR>;
+  const int lane = threadIdx.x & 31;
+  const int G = p.G;
+  uint32_t q_cnt = 0;
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+  while (items.next(w)) {
+    if (w.kv_hi <= w.kv_lo) continue;
+    const uint32_t qb = q_cnt % C::QBUF;
+    if (!warp_wait(bar0 + 8 * (C::B_QEMPTY + qb), ((q_cnt / C::QBUF) & 1) ^ 1, abort)) break;
+    const uint32_t base = sQ + qb * C::Q_BYTES;
+    const int rows = w.n_tok * G;
+    const int units = rows * (D / 8);                 // 16-byte pieces
+    const int t0 = w.t_base + w.q_tok0;
+    for (int u0 = 0; u0 < units; u0 += 4 * 32) {
+      uint4 v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int u = u0 + k * 32 + lane;
+        if (u < units) {
+          const int r = u / (D / 8), c16 = u % (D / 8);
+          const int t = t0 + r / G, h = w.kvh * G + r % G;
+          v[k] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)t * p.Hq + h) * D) + c16);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int u = u0 + k * 32 + lane;
+        if (u < units) {
+          const int r = u / (D / 8), c16 = u % (D / 8);
+          const uint32_t dst =
+              base + (c16 >> 3) * C::Q_CHUNK + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[k].x),
+                       "r"(v[k].y), "r"(v[k].z), "r"(v[k].w)
+                       : "memory");
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar0 + 8 * (C::B_QFULL + qb));
+    ++q_cnt;
+  }
+}
+
+// K/V producer: tiles of 128 keys in kv_sequence order; one TMA box per page
+// (or part of a page) per 64-column chunk, lane k issuing box k.  Producer
+// `which` (0 or 1) issues the loads whose index has that parity; both walk the
+// whole order so that they agree on slots and page ids.  The page ids a lane
+// needs are loaded three tiles ahead (pf0..pf2 hold tiles j..j+2 when K_j is
+// reached), and the first three tiles of the next item are loaded during the
+// current item's last K, so no table read is waited on in the loop.
+template <int D, int NR>
+__device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                             const AttnParams& p, uint32_t sKV, uint32_t bar0,
+                                             int n_items, uint32_t which, volatile int* abort) {
+  using C = DecCfg<D, NR>;
+  const int lane = threadIdx.x & 31;
+  uint32_t ld_idx = 0;
+  bool ok = true;
+  int nx0 = 0, nx1 = 0, nx2 = 0;
+  bool have_next = false;
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+  while (ok && items.next(w)) {
+    const int n = item_tiles(w, C::BN);
+    if (n == 0) {
+      have_next = false;
+      continue;
+    }
+    int pf0, pf1, pf2;
+    if (have_next) {
+      pf0 = nx0; pf1 = nx1; pf2 = nx2;
+    } else {
+      // tile_page_id reads nothing for tiles past the item (it returns 0)
+      pf0 = tile_page_id(p, w, 0, C::BN, lane);
+      pf1 = tile_page_id(p, w, 1, C::BN, lane);
+      pf2 = tile_page_id(p, w, 2, C::BN, lane);
+    }
+    have_next = false;
+    int pid_v = 0, pid_v_next = 0;
+    for (int s = 0; s < 2 * n; ++s) {
+      int j;
+      bool is_v;
+      kv_sequence(s, n, j, is_v);
+      int page;
+      if (!is_v) {
+        pid_v = pid_v_next;
+        pid_v_next = pf0;
+        page = pf0;
+        pf0 = pf1;
+        pf1 = pf2;
+        pf2 = tile_page_id(p, w, j + 3, C::BN, lane);
+      } else {
+        page = (j == n - 1) ? pid_v_next : pid_v;
+      }
+      const bool mine = (ld_idx & 1u) == which;
+      const uint32_t slot = ld_idx % C::NSLOT;
+      if (mine &&
+          !warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
+        ok = false;
+        break;
+      }
+      const int n0 = w.kv_lo + j * C::BN;
+      // every live row of the tile is loaded (rows past the item's range
+      // included) so that no stale shared memory meets the products
+      const int live = min(w.kv_len - n0, C::BN);
+      const int nbox = ceil_div(live, p.box_h);
+      const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
+      if (mine && lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
+      __syncwarp();
+      if (mine && lane < nbox) {
+        const int row = (n0 + lane * p.box_h) % p.ps;
+        if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
+          atomicOr(p.status, kStatusBadPage);
+          page = -1;   // out of the tensor map: the box reads as zeros
+        }
+        const CUtensorMap* tm = is_v ? tm_v : tm_k;
+        const uint32_t dst = sKV + slot * C::SLOT_BYTES + lane * p.box_h * 128;
+        for (int c = 0; c < C::DCH; ++c)
+          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, row, page);
+      }
+      if (!is_v && j == n - 1) {
+        WorkItem nw;
+        if (items.peek(nw) && item_tiles(nw, C::BN) > 0) {
+          nx0 = tile_page_id(p, nw, 0, C::BN, lane);
+          nx1 = tile_page_id(p, nw, 1, C::BN, lane);
+          nx2 = tile_page_id(p, nw, 2, C::BN, lane);
+          have_next = true;
+        }
+      }
+      ++ld_idx;
+    }
+  }
+  if (!ok || *abort) {
+    // wait (bounded) for this producer's copies still in flight
+    if (lane == 0) {
+      const uint32_t first = ld_idx > (uint32_t)C::NSLOT ? ld_idx - C::NSLOT : 0;
+      for (uint32_t k = first; k < ld_idx; ++k)
+        if ((k & 1u) == which) mbar_drain(bar0 + 8 * (C::B_KVFULL + k % C::NSLOT), (k / C::NSLOT) & 1);
+    }
+  }
+}
+
+// MMA issuer (all 32 lanes; one elected lane issues).  Per item of n tiles:
+//   S^T(0) | S^T(1) O^T+=V(0)^T P^T(0) | S^T(2) O^T+=V(1)^T P^T(1) | ...
+// g counts tiles over all items: S^T(g) and P^T(g) use buffer g & 1.
+template <int D, int NR>
+__device__ __forceinline__ void dec_mma(const AttnParams& p, uint32_t sQ, uint32_t sKV,
+                                        uint32_t sP, uint32_t bar0, uint32_t tmem, int n_items,
+                                        volatile int* abort) {
+  using C = DecCfg<D, NR>;
+  constexpr uint32_t kIdescS = idesc_bf16_f32(128, NR, false, false);
+  constexpr uint32_t kIdescO = idesc_bf16_f32(128, NR, true, false);
+  uint32_t ld_idx = 0, g = 0, q_cnt = 0;
+  bool ok = true;
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+
+  auto kv_wait = [&](uint32_t idx) -> bool {
+    const uint32_t slot = idx % C::NSLOT;
+    if (!warp_wait(bar0 + 8 * (C::B_KVFULL + slot), (idx / C::NSLOT) & 1, abort)) return false;
+    tc_fence_after();
+    return true;
+  };
+  // S^T(gs) = K Q^T: A = K tile (K-major, 128 keys), B = Q tile (K-major, NR rows)
+  auto issue_s = [&](uint32_t gs, uint32_t k_idx, uint32_t sQb) {
+    const uint32_t slot_addr = sKV + (k_idx % C::NSLOT) * C::SLOT_BYTES;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t ad =
+          smem_desc_sw128(slot_addr + (kk >> 2) * C::SLOT_CHUNK + (kk & 3) * 32, 16, 1024);
+      const uint64_t bd = smem_desc_sw128(sQb + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024);
+      mma_ss_w(tmem + C::S_COL + (gs & 1) * NR, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+    }
+    tc_commit_w(bar0 + 8 * (C::B_SFULL + (gs & 1)));
+  };
+  // O^T += V^T P^T(gp): A = V tile read MN-major (M = 128 columns of D),
+  // B = P^T (K-major, NR rows x 128 keys)
+  auto issue_o = [&](uint32_t gp, uint32_t v_idx, bool first) {
+    const uint32_t slot_addr = sKV + (v_idx % C::NSLOT) * C::SLOT_BYTES;
+    const uint32_t pb = sP + (gp & 1) * C::P_BYTES;
+#pragma unroll
+    for (int kk = 0; kk < C::BN / 16; ++kk) {
+      const uint64_t bd = smem_desc_sw128(pb + (kk >> 2) * C::P_CHUNK + (kk & 3) * 32, 16, 1024);
+#pragma unroll
+      for (int hh = 0; hh < C::DH; ++hh) {
+        const uint64_t ad = smem_desc_sw128(slot_addr + 2 * hh * C::SLOT_CHUNK + kk * 16 * 128,
+                                            C::SLOT_CHUNK, 1024);
+        mma_ss_w(tmem + C::O_COL + hh * NR, ad, bd, kIdescO, (!first || kk > 0) ? 1u : 0u);
+      }
+    }
+    tc_commit_w(bar0 + 8 * (C::B_PVDONE + (gp & 1)));
+  };
+
+  while (ok && items.next(w)) {
+    const int n = item_tiles(w, C::BN);
+    if (n == 0) continue;
+    const uint32_t qb = q_cnt % C::QBUF;
+    const uint32_t sQb = sQ + qb * C::Q_BYTES;
+    if (!warp_wait(bar0 + 8 * (C::B_QFULL + qb), (q_cnt / C::QBUF) & 1, abort)) { ok = false; break; }
+    tc_fence_after();
+    if (!kv_wait(ld_idx)) { ok = false; break; }
+    issue_s(g, ld_idx, sQb);
+    tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + ld_idx % C::NSLOT));
+    if (n == 1) tc_commit_w(bar0 + 8 * (C::B_QEMPTY + qb));
+    for (int j = 0; j < n && ok; ++j) {
+      if (j + 1 < n) {
+        const uint32_t k_idx = ld_idx + (2 * (j + 1) - 1);
+        if (!kv_wait(k_idx)) { ok = false; break; }
+        issue_s(g + j + 1, k_idx, sQb);
+        tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + k_idx % C::NSLOT));
+        if (j + 2 == n) tc_commit_w(bar0 + 8 * (C::B_QEMPTY + qb));
+      }
+      const uint32_t v_idx = ld_idx + (j == n - 1 ? 2 * n - 1 : 2 * j + 2);
+      if (!kv_wait(v_idx)) { ok = false; break; }
+      const uint32_t gp = g + j;
+      if (!warp_wait(bar0 + 8 * (C::B_PFULL + (gp & 1)), (gp >> 1) & 1, abort)) { ok = false; break; }
+      if (j == 0 && !warp_wait(bar0 + 8 * C::B_OEMPTY, (q_cnt & 1) ^ 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      issue_o(gp, v_idx, j == 0);
+      tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + v_idx % C::NSLOT));
+    }
+    g += n;
+    ld_idx += 2 * n;
+    ++q_cnt;
+  }
+  tc_commit_w(bar0 + 8 * C::B_DRAIN);
+  if ((threadIdx.x & 31) == 0) mbar_drain(bar0 + 8 * C::B_DRAIN, 0);
+  __syncwarp();
+}
+
+template <int NR>
+__device__ __forceinline__ void ld_cols(uint32_t taddr, uint32_t (&r)[NR]);
+template <>
+__device__ __forceinline__ void ld_cols<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  tmem_ld16(taddr, r);
+  tmem_ld_wait(r);
+}
+template <>
+__device__ __forceinline__ void ld_cols<32>(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_ld32(taddr, r);
+  tmem_ld_wait(r);
+}
+template <int NR>
+__device__ __forceinline__ void st_cols(uint32_t taddr, const uint32_t (&r)[NR]) {
+#pragma unroll
+  for (int c = 0; c < NR; c += 16) tmem_st16(taddr + c, r + c);
+}
+
+// Sum (or max) of one value per thread over the 128 softmax threads for each
+// of RR rows: butterfly within the warp, then the four warp results through
+// shared memory behind an mbarrier (bounded wait; count 4, one arrival per warp).
+template <int RR, bool MAX>
+__device__ __forceinline__ bool block_reduce_rows(float (&v)[RR], float* red, uint32_t bar,
+                                                  uint32_t phase, volatile int* abort) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int r = 0; r < RR; ++r) {
+    float x = v[r];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float y = __shfl_xor_sync(0xffffffffu, x, o);
+      x = MAX ? fmaxf(x, y) : x + y;
+    }
+    v[r] = x;
+  }
+  if (lane < RR) {
+    // lane r stores row r (a select chain instead of a dynamic register index)
+    float x = v[0];
+#pragma unroll
+    for (int r = 1; r < RR; ++r) x = lane == r ? v[r] : x;
+    red[warp * RR + lane] = x;
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  if (!warp_wait(bar, phase, abort)) return false;
+#pragma unroll
+  for (int r = 0; r < RR; ++r) {
+    const float a = red[r], b = red[RR + r], c = red[2 * RR + r], d = red[3 * RR + r];
+    v[r] = MAX ? fmaxf(fmaxf(a, b), fmaxf(c, d)) : (a + b) + (c + d);
+  }
+  return true;
+}
+
+// Softmax, correction and epilogue (warps 0-3).  Thread t owns key t of each
+// tile and column d = 128 h + t of O.  Every thread holds the running maximum
+// of every row (identical in all threads) and its own share of the row sums.
+// A decode item is one query token: its G rows see the same keys [kv_lo, kv_hi).
+// Rows G .. RR-1 (padding) are held at -inf, so their P is 0.
+template <int D, int NR, int RR>
+__device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, uint32_t sP,
+                                            float* red, uint32_t bar0, uint32_t tmem,
+                                            int n_items, volatile int* abort) {
+  using C = DecCfg<D, NR>;
+  constexpr int BN = C::BN;
+  const int t = threadIdx.x;
+  const int warp = t >> 5, lane = t & 31;
+  const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);   // this warp's lanes
+  const int G = p.G;
+  // this thread's P^T column: 16-byte unit u of row r sits at u ^ (r & 7)
+  const uint32_t p_col = (t >> 6) * C::P_CHUNK + (t & 7) * 2;
+  const int p_unit = (t & 63) >> 3;
+  uint32_t g = 0, ld_base = 0, q_cnt = 0;
+  bool ok = true;
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+  while (ok && items.next(w)) {
+    const int n = item_tiles(w, BN);
+    const bool split = w.n_splits > 1;
+    const size_t prow0 = (((size_t)w.b * p.Hkv + w.kvh) * p.S_max + w.split) * kBM;
+    const size_t orow0 = (size_t)(w.t_base + w.q_tok0) * p.Hq + (size_t)w.kvh * G;
+    if (n == 0) {
+      // no key: O = 0, LSE = -inf
+      for (int r = 0; r < G; ++r) {
+#pragma unroll
+        for (int hh = 0; hh < C::DH; ++hh) {
+          const int d = hh * 128 + t;
+          if (split) p.part_o[(prow0 + r) * D + d] = 0.f;
+          else p.out[(orow0 + r) * D + d] = 0;
+        }
+        if (t == 0) {
+          if (split) p.part_lse[prow0 + r] = -INFINITY;
+          else if (p.lse) p.lse[orow0 + r] = -INFINITY;
+        }
+      }
+      continue;
+    }
+    float m_run[RR], l_part[RR];
+#pragma unroll
+    for (int r = 0; r < RR; ++r) {
+      m_run[r] = -INFINITY;
+      l_part[r] = 0.f;
+    }
+    for (int j = 0; j < n && ok; ++j) {
+      const uint32_t gj = g + j, sb = gj & 1;
+      if (!warp_wait(bar0 + 8 * (C::B_SFULL + sb), (gj >> 1) & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      const int n0 = w.kv_lo + j * BN;
+      const bool valid = n0 + t < w.kv_hi;
+      float s[RR];
+      {
+        uint32_t v[NR];
+        ld_cols<NR>(tl + C::S_COL + sb * NR, v);
+#pragma unroll
+        for (int r = 0; r < RR; ++r)
+          s[r] = (valid && r < G) ? __uint_as_float(v[r]) : -INFINITY;   // mask by select
+      }
+      float mx[RR];
+#pragma unroll
+      for (int r = 0; r < RR; ++r) mx[r] = s[r];
+      if (!block_reduce_rows<RR, true>(mx, red + sb * 4 * RR, bar0 + 8 * (C::B_RED + sb),
+                                       (gj >> 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      float alpha[RR];
+      bool any = false;
+#pragma unroll
+      for (int r = 0; r < RR; ++r) {
+        const float m_new = fmaxf(m_run[r], mx[r] * p.scale_log2);
+        const bool need = m_new > m_run[r] + kRescaleThreshold;
+        alpha[r] = need ? ex2_approx(m_run[r] - m_new) : 1.f;   // 0 while m_run is -inf
+        any = any || (need && m_run[r] != -INFINITY);
+        m_run[r] = need ? m_new : m_run[r];
+      }
+      if (any && j > 0) {
+        // O^T holds the sum up to tile gj-1: wait for that product, then rescale
+        const uint32_t gp = gj - 1;
+        if (!warp_wait(bar0 + 8 * (C::B_PVDONE + (gp & 1)), (gp >> 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int hh = 0; hh < C::DH; ++hh) {
+          uint32_t o[NR];
+          ld_cols<NR>(tl + C::O_COL + hh * NR, o);
+#pragma unroll
+          for (int r = 0; r < RR; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
+          st_cols<NR>(tl + C::O_COL + hh * NR, o);
+        }
+        tmem_st_wait();
+      }
+      // P^T[r][t] (bf16) into buffer sb: row r of the B operand of O^T
+      const uint32_t pb = sP + sb * C::P_BYTES + p_col;
+#pragma unroll
+      for (int r = 0; r < RR; ++r) {
+        const float m_use = m_run[r] == -INFINITY ? 0.f : m_run[r];
+        const float pr = ex2_approx(fmaf(s[r], p.scale_log2, -m_use));
+        l_part[r] = fmaf(l_part[r], alpha[r], pr);
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(pb + r * 128 + ((p_unit ^ (r & 7)) << 4)),
+                     "h"(bf16_bits(pr))
+                     : "memory");
+      }
+      if (j == n - 1 && n0 + BN > w.kv_len) {
+        // rows at and past kv_len of the last V tile: tail slots or rows never
+        // loaded; P is 0 there but 0 * NaN would still poison O
+        const uint32_t ldv = ld_base + 2 * n - 1;
+        const uint32_t slot = ldv % C::NSLOT;
+        if (!warp_wait(bar0 + 8 * (C::B_KVFULL + slot), (ldv / C::NSLOT) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        const int z0 = w.kv_len - n0;
+        const int units = (BN - z0) * C::DCH * 8;
+        const uint32_t base = sKV + slot * C::SLOT_BYTES;
+        for (int uu = t; uu < units; uu += 128) {
+          const int row = z0 + uu / (C::DCH * 8);
+          const int rem = uu % (C::DCH * 8);
+          const uint32_t a = base + (rem >> 3) * C::SLOT_CHUNK + row * 128 + (rem & 7) * 16;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0) : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar0 + 8 * (C::B_PFULL + sb));
+    }
+    if (!ok) break;
+    g += n;
+    ld_base += 2 * n;
+    // ---- epilogue: O / l -> out (or the split partial), LSE
+    if (!block_reduce_rows<RR, false>(l_part, red + 2 * 4 * RR, bar0 + 8 * C::B_REDSUM,
+                                      q_cnt & 1, abort)) {
+      ok = false;
+      break;
+    }
+    const uint32_t gl = g - 1;
+    if (!warp_wait(bar0 + 8 * (C::B_PVDONE + (gl & 1)), (gl >> 1) & 1, abort)) { ok = false; break; }
+    tc_fence_after();
+#pragma unroll
+    for (int hh = 0; hh < C::DH; ++hh) {
+      uint32_t o[NR];
+      ld_cols<NR>(tl + C::O_COL + hh * NR, o);
+      const int d = hh * 128 + t;
+#pragma unroll
+      for (int r = 0; r < RR; ++r) {
+        if (r < G) {
+          const float inv_l = l_part[r] > 0.f ? 1.0f / l_part[r] : 0.f;
+          const float val = __uint_as_float(o[r]) * inv_l;
+          if (split) p.part_o[(prow0 + r) * D + d] = val;
+          else p.out[(orow0 + r) * D + d] = bf16_bits(val);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < RR; ++r) {
+      if (r < G && t == r) {
+        const float lse_v =
+            l_part[r] > 0.f ? (m_run[r] + log2f(l_part[r])) * 0.69314718055994531f : -INFINITY;
+        if (split) p.part_lse[prow0 + r] = lse_v;
+        else if (p.lse) p.lse[orow0 + r] = lse_v;
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar0 + 8 * C::B_OEMPTY);
+    ++q_cnt;
+  }
+}
+
+// RR: registers rows per thread (G rounded up to a power of two, >= 4);
+// NR: MMA rows (N), at least 16.
+template <int RR>
+struct DecRows {
+  static_assert(RR == 4 || RR == 8 || RR == 16 || RR == 32, "decode rows");
+  static constexpr int NR = RR < 16 ? 16 : RR;
+};
+
+template <int D, int RR>
+__global__ void __launch_bounds__(256, 1)
+    pa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  constexpr int NR = DecRows<RR>::NR;
+  using C = DecCfg<D, NR>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t sKV = base;
+  const uint32_t sQ = sKV + C::NSLOT * C::SLOT_BYTES;
+  const uint32_t sP = sQ + C::QBUF * C::Q_BYTES;
+  const uint32_t off_red = C::NSLOT * C::SLOT_BYTES + C::QBUF * C::Q_BYTES + 2 * C::P_BYTES;
+  float* red = reinterpret_cast<float*>(smem + off_red);
+  const uint32_t bar0 = base + off_red + C::RED_BYTES;
+  uint8_t* bar_ptr = smem + off_red + C::RED_BYTES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NBAR);
+  volatile int* abort = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 4);
+
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar0 + 8 * (C::B_QFULL + i), 1);
+      mbar_init(bar0 + 8 * (C::B_QEMPTY + i), 1);
+      mbar_init(bar0 + 8 * (C::B_SFULL + i), 1);
+      mbar_init(bar0 + 8 * (C::B_PFULL + i), 4);
+      mbar_init(bar0 + 8 * (C::B_PVDONE + i), 1);
+      mbar_init(bar0 + 8 * (C::B_RED + i), 4);
+    }
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(bar0 + 8 * (C::B_KVFULL + i), 1);
+      mbar_init(bar0 + 8 * (C::B_KVEMPTY + i), 1);
+    }
+    mbar_init(bar0 + 8 * C::B_OEMPTY, 4);
+    mbar_init(bar0 + 8 * C::B_DRAIN, 1);
+    mbar_init(bar0 + 8 * C::B_REDSUM, 4);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if ((warp == C::PRODUCER_WARP || warp == C::PRODUCER2_WARP) && (threadIdx.x & 31) == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // everything above overlaps the scheduler kernel; its work list is read below
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int n_items = p.hdr->n_items;
+
+  if (warp == C::PRODUCER_WARP || warp == C::PRODUCER2_WARP) {
+    dec_producer<D, NR>(&tm_k, &tm_v, p, sKV, bar0, n_items,
+                        warp == C::PRODUCER_WARP ? 0u : 1u, abort);
+  } else if (warp == C::Q_WARP) {
+    dec_q_loader<D, NR>(p, sQ, bar0, n_items, abort);
+  } else if (warp == C::MMA_WARP) {
+    dec_mma<D, NR>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
+  } else {
+    dec_softmax<D, NR, RR>(p, sKV, sP, red, bar0, tmem, n_items, abort);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort) atomicOr(p.status, kStatusTimeout);
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace pa

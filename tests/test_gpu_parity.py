@@ -68,6 +68,29 @@ def test_decode_without_cu_q_lens():
     compare(out, lse, *oracle_all(w))
 
 
+@pytest.mark.parametrize("D,ps,G,splits", [(128, 16, 4, 0), (128, 64, 1, 1), (128, 128, 8, 3),
+                                            (128, 32, 16, 0), (128, 16, 32, 2), (256, 128, 32, 0),
+                                            (256, 16, 2, 5), (256, 64, 12, 1)])
+def test_decode_kernel(D, ps, G, splits):
+    """Decode-only runs (no cu_q_lens) on the keys-as-M decode kernel: against
+    the oracle, and against the one-stage kernel on the same inputs.  Lengths
+    cover a single key, tails on both sides of the 128-key tile and of a page,
+    and requests long enough to be split."""
+    kv = [1, 15, 127, 128, 129, 300, 2048, 4097]
+    spec = W.custom_spec("deck", G * 2, 2, D, ps, [1] * len(kv), kv, decode_only=True)
+    w = gen(spec, 60 + D + ps + G + splits)
+    plan = make_plan(w, num_splits=splits)
+    plan.set_decode_kernel(True)
+    out, lse, _ = gpu_run(w, plan, use_cu=False)
+    assert plan.status() == 0
+    compare(out, lse, *oracle_all(w))
+    ref = make_plan(w, num_splits=splits)
+    ref.set_decode_kernel(False)
+    out1, lse1, _ = gpu_run(w, ref, use_cu=False)
+    assert torch.max(torch.abs(out.float() - out1.float())).item() <= 1e-2
+    assert torch.max(torch.abs(lse - lse1)).item() <= 1e-3
+
+
 @pytest.mark.parametrize("D,ps,G", [(128, 16, 4), (128, 64, 1), (64, 32, 8), (128, 128, 3)])
 def test_two_stage_prefill_kernel(D, ps, G):
     """The optional two-stage kernel (query-block pairs) against the oracle,
