@@ -6,7 +6,8 @@
 //      split)), longest first, plus per-request split counts.
 //   2. pa_attention_kernel<D>: persistent (two CTAs per SM for D <= 128), warp-specialised:
 //        warps 0-3  softmax / correction / epilogue (one thread per query row)
-//        warp  4    producer: page-table-driven TMA gathers of K and V pages
+//        warps 4, 7 producers: page-table-driven TMA gathers of K and V pages
+//                   (alternate loads: one issuing warp cannot keep HBM busy)
 //        warp  5    MMA issuer: tcgen05 S = Q K^T and O += P V, TMEM accumulators
 //        warp  6    Q loader: Q tiles by TMA (or plain loads for partial blocks)
 //   3. pa_merge_kernel: log-sum-exp merge of split-KV partial states.
@@ -106,10 +107,12 @@ struct WsHeader {
 };
 
 constexpr int kBM = 128;              // query rows per tile (tcgen05 M)
-constexpr int kThreads = 224;         // 7 warps
+constexpr int kThreads = 256;         // 8 warps
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kQWarp = 6;
+constexpr int kProducer2Warp = 7;     // second K/V producer: one issuing warp per CTA
+                                      // cannot keep HBM busy with page-sized boxes
 constexpr int kCostBuckets = 1024;
 constexpr int kSchedSmemReqs = 4096;  // unit offsets of up to this many requests live in smem
 constexpr int kMaxSplits = 64;
@@ -122,7 +125,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when th
 template <int D>
 struct TileCfg {
   static constexpr int CTAS = (D == 256) ? 1 : 2;      // CTAs per SM
-  // 14 warps on 4 sub-partitions: at most 4 warps x 32 lanes x 128 = 16 K registers each
+  // 16 warps on 4 sub-partitions: 4 warps x 32 lanes x 128 = 16 K registers each
   static constexpr int MAXREG = (CTAS == 2) ? 128 : 255;
   static constexpr int BN = 64;                       // keys per KV tile
   static constexpr int DCH = D / 64;                  // 128-byte column chunks per row
@@ -653,7 +656,7 @@ __device__ __forceinline__ int tile_page_id(const AttnParams& p, const WorkItem&
 template <int D>
 __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const AttnParams& p, uint32_t sKV, uint32_t bar0,
-                                              int n_items, volatile int* abort) {
+                                              int n_items, uint32_t which, volatile int* abort) {
   using C = TileCfg<D>;
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
@@ -680,8 +683,12 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
       int j;
       bool is_v;
       kv_sequence(s, n, j, is_v);
+      // both producers walk the whole order; this one issues the loads whose
+      // index has parity `which`
+      const bool mine = (ld_idx & 1u) == which;
       const uint32_t slot = ld_idx % C::NSLOT;
-      if (!warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
+      if (mine &&
+          !warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
         ok = false;
         break;
       }
@@ -691,7 +698,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
       const int live = min(w.kv_len - n0, C::BN);
       const int nbox = ceil_div(live, p.box_h);
       const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
-      if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
+      if (mine && lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
       __syncwarp();
       int page;
       if (!is_v) {
@@ -701,7 +708,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
       } else {
         page = (j == n - 1) ? pid_v_next : pid_v;
       }
-      if (lane < nbox) {
+      if (mine && lane < nbox) {
         const int row = (n0 + lane * p.box_h) % p.ps;
         if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
           atomicOr(p.status, kStatusBadPage);
@@ -731,7 +738,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
     if (lane == 0) {
       const uint32_t first = ld_idx > (uint32_t)C::NSLOT ? ld_idx - C::NSLOT : 0;
       for (uint32_t k = first; k < ld_idx; ++k)
-        mbar_drain(bar0 + 8 * (C::B_KVFULL + k % C::NSLOT), (k / C::NSLOT) & 1);
+        if ((k & 1u) == which) mbar_drain(bar0 + 8 * (C::B_KVFULL + k % C::NSLOT), (k / C::NSLOT) & 1);
     }
   }
 }
@@ -1089,7 +1096,7 @@ __global__ void __maxnreg__(TileCfg<D>::MAXREG)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == kProducerWarp && (threadIdx.x & 31) == 0) {
+  if ((warp == kProducerWarp || warp == kProducer2Warp) && (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
@@ -1103,8 +1110,8 @@ __global__ void __maxnreg__(TileCfg<D>::MAXREG)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int n_items = p.hdr->n_items;
 
-  if (warp == kProducerWarp) {
-    producer_role<D>(&tm_k, &tm_v, p, sKV, bar0, n_items, abort);
+  if (warp == kProducerWarp || warp == kProducer2Warp) {
+    producer_role<D>(&tm_k, &tm_v, p, sKV, bar0, n_items, warp == kProducerWarp ? 0u : 1u, abort);
   } else if (warp == kQWarp) {
     q_loader_role<D>(&tm_q, p, sQ, bar0, n_items, abort);
   } else if (warp == kMmaWarp) {
