@@ -326,6 +326,19 @@ def config_desc(w) -> str:
                min(q), max(q), min(kv), max(kv), w["seed"]))
 
 
+def attention_kernel_name(w, decode_only: bool) -> str:
+    """The kernel a default plan runs for this workload: decode-only head_dim
+    128 runs (no cu_q_lens) go to the keys-as-M decode kernel, whose rows
+    template is G rounded up to a power of two (at least 4)."""
+    G = w["Hq"] // w["Hkv"]
+    if decode_only and w["D"] == 128 and G <= 32:
+        rr = 4
+        while rr < G:
+            rr *= 2
+        return "pa_decode_kernel<128, %d>" % rr
+    return "pa_attention_kernel<%d>" % w["D"]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -414,7 +427,7 @@ def main():
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "pa_attention_kernel<%d>" % w["D"],
+                     "kernel": attention_kernel_name(w, spec.decode_only),
                      "algorithmic_bytes_per_launch": counts["bytes"],
                      "kernel_ms": attn_ms, "peak_source": "%s hbm_gbs" % peak_kind},
         "gpu_launches": per_run * args.steps,
