@@ -326,6 +326,21 @@ def config_desc(w) -> str:
                min(q), max(q), min(kv), max(kv), w["seed"]))
 
 
+def max_over_ranks(ms: float, device) -> float:
+    """Device time of the slowest rank (the whole job ends when it does); the
+    local time when no process group is running."""
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_value(kv_bytes_per_step: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job K+V GB/s: every rank runs `steps` steps of its own replica of
+    the workload, and the job takes the slowest rank's time."""
+    return kv_bytes_per_step * world * steps / (ms_max * 1e-3) / 1e9
+
+
 def attention_kernel_name(w, decode_only: bool) -> str:
     """The kernel a default plan runs for this workload: decode-only head_dim
     128 runs (no cu_q_lens) go to the keys-as-M decode kernel, whose rows
@@ -407,12 +422,9 @@ def main():
     ms, attn_ms, per_run, status = time_headline(w, plan, args.steps, args.warmup, dist_on)
     clk = clocks.stop()
     plan.close()
-    t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-    if dist_on:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, "cuda")
     ms_step = ms_max / args.steps
-    value = counts["kv_bytes"] * world * args.steps / (ms_max * 1e-3) / 1e9
+    value = replica_value(counts["kv_bytes"], world, args.steps, ms_max)
 
     achieved = counts["bytes"] / (attn_ms * 1e-3) / 1e9
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
