@@ -274,3 +274,63 @@ void oracle_merge_states(int n, int D, const double *o_s, const double *lse_s, d
     }
     *lse = L;
 }
+
+/*
+ * Paged KV append: the step before attention in serving, which writes this
+ * step's new K and V rows into the page pool.  "integrate PrimTS FMHA
+ * kernels" (TensorRT-LLM PR #17399), section "Planning, preprocessing, and
+ * workspace ownership", reuses the engine's fused preprocessing for the
+ * KV-cache append; the slot a token lands in follows section "Unified
+ * page-table metadata": logical page p of request b is page_table[b][p], and
+ * seq_lens[b] counts this step's tokens.  So with q_b = cu[b+1] - cu[b] new
+ * tokens (q_b = 1 when cu_q_lens is NULL) and kv_b = seq_lens[b], new token i
+ * of request b (packed row t = cu[b] + i of k_new / v_new, [T, Hkv, D]) is KV
+ * position j = kv_b - q_b + i and is copied, all Hkv heads at once, to
+ * page page_table[b][j / ps], slot j % ps of k_pool / v_pool ([P, ps, Hkv, D]).
+ * Nothing else in the pools changes.
+ *
+ * Requests that cannot be placed are skipped whole and reported in the
+ * returned bit mask (the same bits as the CUDA path's status word):
+ *   1  a page id outside [0, num_pages) (checked when num_pages > 0, or < 0)
+ *   2  q_b > kv_b
+ *   4  kv_b > C * ps
+ *   8  malformed cu_q_lens (cu[0] != 0 or decreasing)
+ */
+int oracle_append_kv(int B, int Hkv, int D, int ps, int C, int num_pages,
+                     const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_pool,
+                     uint16_t *v_pool, const int32_t *page_table, const int32_t *seq_lens,
+                     const int32_t *cu_q_lens) {
+    int flags = 0;
+    const long row = (long)Hkv * D;   /* elements of one token's K (or V) row */
+    if (cu_q_lens) {
+        if (cu_q_lens[0] != 0) return 8;
+        for (int b = 0; b < B; ++b)
+            if (cu_q_lens[b + 1] < cu_q_lens[b]) return 8;
+    }
+    for (int b = 0; b < B; ++b) {
+        const long t0 = cu_q_lens ? cu_q_lens[b] : b;
+        const int qb = cu_q_lens ? cu_q_lens[b + 1] - cu_q_lens[b] : 1;
+        const int kv = seq_lens[b];
+        if (qb == 0) continue;
+        if (qb > kv) { flags |= 2; continue; }
+        if ((long)kv > (long)C * ps) { flags |= 4; continue; }
+        int ok = 1;
+        for (int i = 0; i < qb && ok; ++i) {
+            const int j = kv - qb + i;
+            const int page = page_table[(long)b * C + j / ps];
+            if (page < 0 || (num_pages > 0 && page >= num_pages)) ok = 0;
+        }
+        if (!ok) { flags |= 1; continue; }
+        for (int i = 0; i < qb; ++i) {
+            const int j = kv - qb + i;
+            const long page = page_table[(long)b * C + j / ps];
+            const long dst = (page * ps + j % ps) * row;
+            const long src = (t0 + i) * row;
+            for (long e = 0; e < row; ++e) {
+                k_pool[dst + e] = k_new[src + e];
+                v_pool[dst + e] = v_new[src + e];
+            }
+        }
+    }
+    return flags;
+}

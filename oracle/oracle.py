@@ -47,6 +47,8 @@ def _declare(lib):
     lib.oracle_paged_attention_rows.restype = i
     lib.oracle_merge_states.argtypes = [i, i, P, P, P, P]
     lib.oracle_merge_states.restype = None
+    lib.oracle_append_kv.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P]
+    lib.oracle_append_kv.restype = i
     return lib
 
 
@@ -140,3 +142,22 @@ def merge_states(o_s, lse_s):
     lse = np.zeros((1,), dtype=np.float64)
     _load().oracle_merge_states(n, D, _ptr(o_s), _ptr(lse_s), _ptr(o), _ptr(lse))
     return o, float(lse[0])
+
+
+def append_kv(k_new, v_new, k_pool, v_pool, page_table, seq_lens, cu_q_lens, num_pages=0):
+    """Paged KV append (see ``oracle_append_kv``).  k_new / v_new: bf16 bits
+    [T, Hkv, D]; the pools ([P, ps, Hkv, D] bf16 bits) are copied and the
+    copies returned with the new rows written, plus the flag mask."""
+    k_new = _u16(k_new)
+    v_new = _u16(v_new)
+    k_out = _u16(k_pool).copy()
+    v_out = _u16(v_pool).copy()
+    page_table = _i32(page_table)
+    seq_lens = _i32(seq_lens)
+    cu = None if cu_q_lens is None else _i32(cu_q_lens)
+    P_, ps, Hkv, D = k_out.shape
+    B, C = page_table.shape
+    flags = _load().oracle_append_kv(B, Hkv, D, ps, C, int(num_pages), _ptr(k_new), _ptr(v_new),
+                                     _ptr(k_out), _ptr(v_out), _ptr(page_table), _ptr(seq_lens),
+                                     _ptr(cu))
+    return k_out, v_out, int(flags)
