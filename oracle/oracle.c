@@ -289,12 +289,14 @@ void oracle_merge_states(int n, int D, const double *o_s, const double *lse_s, d
  * page page_table[b][j / ps], slot j % ps of k_pool / v_pool ([P, ps, Hkv, D]).
  * Nothing else in the pools changes.
  *
- * Requests that cannot be placed are skipped whole and reported in the
- * returned bit mask (the same bits as the CUDA path's status word):
- *   1  a page id outside [0, num_pages) (checked when num_pages > 0, or < 0)
- *   2  q_b > kv_b
- *   4  kv_b > C * ps
- *   8  malformed cu_q_lens (cu[0] != 0 or decreasing)
+ * What cannot be placed is skipped and reported in the returned bit mask
+ * (the same bits as the CUDA path's status word); the pages fix no policy,
+ * this reading skips the least:
+ *   1  a token whose page id is outside [0, num_pages) (checked when
+ *      num_pages > 0; negative ids always): that token only
+ *   2  q_b > kv_b: the whole request
+ *   4  kv_b > C * ps: the whole request
+ *   8  malformed cu_q_lens (cu[0] != 0 or decreasing): nothing is written
  */
 int oracle_append_kv(int B, int Hkv, int D, int ps, int C, int num_pages,
                      const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_pool,
@@ -314,16 +316,10 @@ int oracle_append_kv(int B, int Hkv, int D, int ps, int C, int num_pages,
         if (qb == 0) continue;
         if (qb > kv) { flags |= 2; continue; }
         if ((long)kv > (long)C * ps) { flags |= 4; continue; }
-        int ok = 1;
-        for (int i = 0; i < qb && ok; ++i) {
-            const int j = kv - qb + i;
-            const int page = page_table[(long)b * C + j / ps];
-            if (page < 0 || (num_pages > 0 && page >= num_pages)) ok = 0;
-        }
-        if (!ok) { flags |= 1; continue; }
         for (int i = 0; i < qb; ++i) {
             const int j = kv - qb + i;
             const long page = page_table[(long)b * C + j / ps];
+            if (page < 0 || (num_pages > 0 && page >= num_pages)) { flags |= 1; continue; }
             const long dst = (page * ps + j % ps) * row;
             const long src = (t0 + i) * row;
             for (long e = 0; e < row; ++e) {

