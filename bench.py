@@ -489,7 +489,45 @@ def per_config(peaks):
         res[name] = r
         del w
         torch.cuda.empty_cache()
+    res["kv_append"] = kv_append_rates(bw)
     return res
+
+
+def kv_append_rates(bw):
+    """pa_append_kv on the K/V shapes of the prefill and decode workloads: new
+    rows drawn on the device, written into a shuffled pool.  Bytes per launch =
+    read + write of K and V rows (4 * T * Hkv * D * 2); CUDA events around 20
+    launches after 5 warm-up launches (rows and pools larger than L2 for the
+    prefill shape; the decode shape is latency-bound)."""
+    out = {}
+    for name in ("llama8b_causal_prefill", "llama8b_decode"):
+        w = W.generate(W.CONFIGS[name], W.default_seed(name), device="cuda")
+        T = w["q"].shape[0]
+        g = torch.Generator(device="cuda")
+        g.manual_seed(7)
+        k_new = torch.randn((T, w["Hkv"], w["D"]), generator=g, device="cuda").to(torch.bfloat16)
+        v_new = torch.randn((T, w["Hkv"], w["D"]), generator=g, device="cuda").to(torch.bfloat16)
+        plan = make_plan(w)
+        cu = None if W.CONFIGS[name].decode_only else w["cu_q_lens"]
+        args = (k_new, v_new, w["k_pool"], w["v_pool"], w["page_table"], w["seq_lens"], cu)
+        for _ in range(5):
+            plan.append_kv(*args)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(20):
+            plan.append_kv(*args)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 20
+        nbytes = 4 * T * w["Hkv"] * w["D"] * 2
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"tokens": T, "kernel_ms": ms, "bytes": nbytes, "kernel_GBps": gbs,
+                     "hbm_frac": gbs / bw, "status_word": plan.status()}
+        plan.close()
+        del w, k_new, v_new
+        torch.cuda.empty_cache()
+    return out
 
 
 if __name__ == "__main__":

@@ -189,6 +189,30 @@ PA_API int pa_set_two_stage_prefill(pa_plan *plan, int on);
  * pa_run; no reallocation.  PA_ERR_INVALID for a NULL plan. */
 PA_API int pa_set_decode_kernel(pa_plan *plan, int on);
 
+/* Paged KV append: write this step's new K and V rows into the pools before
+ * attention ("integrate PrimTS FMHA kernels", section "Planning,
+ * preprocessing, and workspace ownership": the KV-cache append of the
+ * preprocessing; slots per section "Unified page-table metadata").
+ *   k_new, v_new   bf16 [T, Hkv, D], packed like q (row cu_q_lens[b] + i is
+ *                  new token i of request b); T = cu_q_lens[B], or B when
+ *                  cu_q_lens is NULL (one new token per request)
+ *   k_pool, v_pool bf16 [P, ps, Hkv, D], written in place
+ *   page_table, seq_lens, cu_q_lens  as for pa_run; seq_lens counts the new
+ *                  tokens, so token i lands at KV position kv_b - q_b + i:
+ *                  page page_table[b][j / ps], slot j % ps
+ * All device pointers, 16-byte aligned, caller-owned; stream-ordered, no
+ * allocation, no host synchronisation, graph-capturable.  Returns PA_OK,
+ * PA_ERR_INVALID (NULL / misaligned pointer, wrong device) or PA_ERR_CUDA.
+ * What cannot be placed is skipped and flagged in the plan's status word
+ * (pa_get_status): a token on a page id outside [0, num_pages)
+ * (PA_STATUS_BAD_PAGE; checked when pa_set_num_pages was given, negative ids
+ * always), q_b > kv_b (PA_STATUS_Q_GT_KV, the request), kv_b > C * ps
+ * (PA_STATUS_KV_GT_CAPACITY, the request), malformed cu_q_lens
+ * (PA_STATUS_BAD_CU_Q, nothing written). */
+PA_API int pa_append_kv(pa_plan *plan, const void *k_new, const void *v_new, void *k_pool,
+                        void *v_pool, const int32_t *page_table, const int32_t *seq_lens,
+                        const int32_t *cu_q_lens, pa_stream_t stream);
+
 /* Kernel timing for benchmarks.  pa_profile_start makes the next `max_runs`
  * (1..4096) calls of pa_run record a CUDA event pair on their stream around
  * the attention kernel.  pa_profile_read synchronises on those events, writes

@@ -27,7 +27,7 @@ STATUS_TIMEOUT = 1 << 4
 EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_scale",
            "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
            "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc",
-           "pa_set_two_stage_prefill", "pa_set_decode_kernel")
+           "pa_set_two_stage_prefill", "pa_set_decode_kernel", "pa_append_kv")
 
 # Size of the library's static scratch array used by pa_run_noalloc.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -79,6 +79,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_set_two_stage_prefill.restype = I
     lib.pa_set_decode_kernel.argtypes = [P, I]
     lib.pa_set_decode_kernel.restype = I
+    lib.pa_append_kv.argtypes = [P, P, P, P, P, P, P, P, P]
+    lib.pa_append_kv.restype = I
     lib.pa_run_noalloc.argtypes = [I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P]
     lib.pa_run_noalloc.restype = I
     if path == LIB_PATH:
@@ -191,6 +193,41 @@ class Plan:
                                 _ptr(seq_lens), _ptr(cu_q_lens), _ptr(out), _ptr(lse),
                                 ctypes.c_void_p(stream)))
         return out, lse
+
+    def append_kv(self, k_new, v_new, k_pool, v_pool, page_table, seq_lens, cu_q_lens=None,
+                  stream=None):
+        """Write this step's new K/V rows ([T, Hkv, D] bf16, packed like q) into
+        the pools in place (``pa_append_kv``); stream-ordered."""
+        B, Hkv, D = self.batch, self.heads_kv, self.head_dim
+        dev = k_new.device
+        if dev.type != "cuda":
+            raise ValueError("tensors must be on a CUDA device")
+        for name, t, dt in (("k_new", k_new, torch.bfloat16), ("v_new", v_new, torch.bfloat16),
+                            ("k_pool", k_pool, torch.bfloat16), ("v_pool", v_pool, torch.bfloat16),
+                            ("page_table", page_table, torch.int32),
+                            ("seq_lens", seq_lens, torch.int32)):
+            if t.dtype != dt or t.device != dev or not t.is_contiguous():
+                raise ValueError("%s must be a contiguous %s tensor on %s" % (name, dt, dev))
+        if k_new.dim() != 3 or tuple(k_new.shape[1:]) != (Hkv, D) or v_new.shape != k_new.shape:
+            raise ValueError("k_new and v_new must be [T, %d, %d]" % (Hkv, D))
+        if k_pool.dim() != 4 or tuple(k_pool.shape[1:]) != (self.page_size, Hkv, D) \
+                or v_pool.shape != k_pool.shape:
+            raise ValueError("k_pool and v_pool must be [P, %d, %d, %d]" % (self.page_size, Hkv, D))
+        if tuple(page_table.shape) != (B, self.capacity) or tuple(seq_lens.shape) != (B,):
+            raise ValueError("page_table must be [%d, %d] and seq_lens [%d]" % (B, self.capacity, B))
+        if cu_q_lens is not None:
+            if (cu_q_lens.dtype != torch.int32 or tuple(cu_q_lens.shape) != (B + 1,)
+                    or cu_q_lens.device != dev or not cu_q_lens.is_contiguous()):
+                raise ValueError("cu_q_lens must be a contiguous int32 [%d] tensor" % (B + 1))
+        elif k_new.shape[0] != B:
+            raise ValueError("without cu_q_lens, k_new must hold one token per request")
+        if stream is None:
+            stream = torch.cuda.current_stream(dev).cuda_stream
+        elif isinstance(stream, torch.cuda.Stream):
+            stream = stream.cuda_stream
+        _check(self._lib.pa_append_kv(self._h, _ptr(k_new), _ptr(v_new), _ptr(k_pool),
+                                      _ptr(v_pool), _ptr(page_table), _ptr(seq_lens),
+                                      _ptr(cu_q_lens), ctypes.c_void_p(stream)))
 
     def profile_start(self, max_runs: int):
         """Record the attention kernel's duration in the next ``max_runs`` runs."""

@@ -19,6 +19,7 @@
 #include "pa_kernels.cuh"
 #include "pa_prefill.cuh"
 #include "pa_decode.cuh"
+#include "pa_append.cuh"
 
 namespace {
 
@@ -618,6 +619,52 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_err("pa_run: launch failed: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+int pa_append_kv(pa_plan* p, const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                 const int32_t* page_table, const int32_t* seq_lens, const int32_t* cu_q_lens,
+                 pa_stream_t stream) {
+  if (!p) { set_err("pa_append_kv: NULL plan"); return PA_ERR_INVALID; }
+  if (!k_new || !v_new || !k_pool || !v_pool || !page_table || !seq_lens) {
+    set_err("pa_append_kv: NULL pointer (k_new, v_new, k_pool, v_pool, page_table and "
+            "seq_lens are required)");
+    return PA_ERR_INVALID;
+  }
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool) ||
+      !aligned16(page_table) || !aligned16(seq_lens) || (cu_q_lens && !aligned16(cu_q_lens))) {
+    set_err("pa_append_kv: every pointer must be 16-byte aligned");
+    return PA_ERR_INVALID;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) {
+    set_err("pa_append_kv: current device %d is not the plan's device %d", dev, p->device);
+    return PA_ERR_INVALID;
+  }
+  pa::AppendParams ap;
+  ap.k_new = static_cast<const uint4*>(k_new);
+  ap.v_new = static_cast<const uint4*>(v_new);
+  ap.k_pool = static_cast<uint4*>(k_pool);
+  ap.v_pool = static_cast<uint4*>(v_pool);
+  ap.page_table = page_table;
+  ap.seq_lens = seq_lens;
+  ap.cu_q_lens = cu_q_lens;
+  ap.status = &p->hdr->status;
+  ap.B = p->B; ap.C = p->C; ap.ps = p->ps; ap.num_pages = p->num_pages;
+  ap.row_u4 = p->Hkv * p->D / 8;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // one warp per new token; T is known only on the device, so the grid is
+  // sized for the most tokens the batch can hold (B * C * ps), at most four
+  // CTAs of eight warps per SM
+  const long max_tok = (long)p->B * p->C * p->ps;
+  const long want = (max_tok + (pa::kAppendThreads / 32) - 1) / (pa::kAppendThreads / 32);
+  const int grid = (int)(want < 4L * p->n_sm ? want : 4L * p->n_sm);
+  pa::pa_append_kernel<<<grid, pa::kAppendThreads, 0, st>>>(ap);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_err("pa_append_kv: launch failed: %s", cudaGetErrorString(e));
     return PA_ERR_CUDA;
   }
   return PA_OK;
