@@ -64,6 +64,7 @@ typedef struct {
     const uint16_t *q, *k_pool, *v_pool;
     const int32_t *page_table, *seq_lens, *cu_q_lens;
     double scale;
+    int non_causal;       /* 0: causal mask (default); 1: every row sees all kv_b keys */
     double *out, *lse;
     /* rows to compute: either all (rows == NULL) or a list of (t, h) */
     const int32_t *row_t, *row_h;
@@ -97,6 +98,7 @@ static int one_row(const job_t *J, long t, int h, double *o_row, double *lse_out
 
     /* visible keys: j < n, with the causal limit aligned to the end of KV */
     long n = kv_b - q_b + i + 1;
+    if (J->non_causal) n = kv_b;           /* non-causal: every key of the request */
     if (n > kv_b) n = kv_b;
     if (n < 0) n = 0;
 
@@ -225,6 +227,28 @@ int oracle_paged_attention(int B, int Hq, int Hkv, int D, int ps, int C, int num
     return run_job(&J, nthreads);
 }
 
+/*
+ * The same with a mask mode.  causal = 0 drops the causal limit: every query
+ * row of request b sees all kv_b keys.  "Unified Triton kernel that doesn't
+ * distinguish between prefill + decode" (vLLM PR #16828), review thread on the
+ * masking: non-causal attention is asked for (cascade attention, MLA); the
+ * plainest reading is the same softmax over the request's whole KV.
+ */
+int oracle_paged_attention_mode(int B, int Hq, int Hkv, int D, int ps, int C, int num_pages,
+                                const uint16_t *q, const uint16_t *k_pool,
+                                const uint16_t *v_pool, const int32_t *page_table,
+                                const int32_t *seq_lens, const int32_t *cu_q_lens, double scale,
+                                int causal, double *out, double *lse, int nthreads) {
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.ps = ps; J.C = C; J.num_pages = num_pages;
+    J.q = q; J.k_pool = k_pool; J.v_pool = v_pool;
+    J.page_table = page_table; J.seq_lens = seq_lens; J.cu_q_lens = cu_q_lens;
+    J.scale = scale; J.out = out; J.lse = lse;
+    J.non_causal = causal ? 0 : 1;
+    return run_job(&J, nthreads);
+}
+
 /* Only the listed rows: row u is (token row_t[u], head row_h[u]); out is
  * [n_rows, D], lse is [n_rows].  Same return codes. */
 int oracle_paged_attention_rows(int B, int Hq, int Hkv, int D, int ps, int C, int num_pages,
@@ -296,7 +320,8 @@ void oracle_merge_states(int n, int D, const double *o_s, const double *lse_s, d
  *      num_pages > 0; negative ids always): that token only
  *   2  q_b > kv_b: the whole request
  *   4  kv_b > C * ps: the whole request
- *   8  malformed cu_q_lens (cu[0] != 0 or decreasing): nothing is written
+ *   8  malformed cu_q_lens (cu[0] != 0, decreasing, or a total past
+ *      B * C * ps): nothing is written
  */
 int oracle_append_kv(int B, int Hkv, int D, int ps, int C, int num_pages,
                      const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_pool,
@@ -305,7 +330,9 @@ int oracle_append_kv(int B, int Hkv, int D, int ps, int C, int num_pages,
     int flags = 0;
     const long row = (long)Hkv * D;   /* elements of one token's K (or V) row */
     if (cu_q_lens) {
-        if (cu_q_lens[0] != 0) return 8;
+        /* a total past B * C * ps cannot come from valid requests (q_b <= kv_b
+         * <= C * ps), so it is treated as malformed too */
+        if (cu_q_lens[0] != 0 || (long)cu_q_lens[B] > (long)B * C * ps) return 8;
         for (int b = 0; b < B; ++b)
             if (cu_q_lens[b + 1] < cu_q_lens[b]) return 8;
     }

@@ -45,6 +45,9 @@ def _declare(lib):
     lib.oracle_paged_attention_rows.argtypes = [i, i, i, i, i, i, i, P, P, P, P, P, P,
                                                 ctypes.c_double, P, P, ctypes.c_long, P, P, i]
     lib.oracle_paged_attention_rows.restype = i
+    lib.oracle_paged_attention_mode.argtypes = [i, i, i, i, i, i, i, P, P, P, P, P, P,
+                                                ctypes.c_double, i, P, P, i]
+    lib.oracle_paged_attention_mode.restype = i
     lib.oracle_merge_states.argtypes = [i, i, P, P, P, P]
     lib.oracle_merge_states.restype = None
     lib.oracle_append_kv.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P]
@@ -88,9 +91,11 @@ def default_threads() -> int:
 
 
 def paged_attention(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, scale,
-                    num_pages: int = 0, nthreads: int | None = None, lib=None):
+                    num_pages: int = 0, nthreads: int | None = None, lib=None,
+                    causal: bool = True):
     """All rows.  Shapes: q [T, Hq, D]; pools [P, ps, Hkv, D]; page_table [B, C];
     seq_lens [B]; cu_q_lens [B+1] or None (one query token per request).
+    ``causal=False`` lets every row see all of its request's keys.
     Returns (out [T, Hq, D] float64, lse [T, Hq] float64)."""
     q, k_pool, v_pool = _u16(q), _u16(k_pool), _u16(v_pool)
     page_table, seq_lens, cu_q_lens = _i32(page_table), _i32(seq_lens), _i32(cu_q_lens)
@@ -100,10 +105,17 @@ def paged_attention(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, scale,
     B, C = page_table.shape
     out = np.zeros((T, Hq, D), dtype=np.float64)
     lse = np.zeros((T, Hq), dtype=np.float64)
-    rc = (lib or _load()).oracle_paged_attention(
-        B, Hq, Hkv, D, ps, C, int(num_pages), _ptr(q), _ptr(k_pool), _ptr(v_pool),
-        _ptr(page_table), _ptr(seq_lens), _ptr(cu_q_lens), float(scale), _ptr(out), _ptr(lse),
-        int(nthreads or default_threads()))
+    L = lib or _load()
+    if causal:
+        rc = L.oracle_paged_attention(
+            B, Hq, Hkv, D, ps, C, int(num_pages), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+            _ptr(page_table), _ptr(seq_lens), _ptr(cu_q_lens), float(scale), _ptr(out),
+            _ptr(lse), int(nthreads or default_threads()))
+    else:
+        rc = L.oracle_paged_attention_mode(
+            B, Hq, Hkv, D, ps, C, int(num_pages), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+            _ptr(page_table), _ptr(seq_lens), _ptr(cu_q_lens), float(scale), 0, _ptr(out),
+            _ptr(lse), int(nthreads or default_threads()))
     if rc:
         raise ValueError("oracle: %s" % {1: "live page id out of range",
                                          2: "out of memory"}.get(rc, rc))

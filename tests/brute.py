@@ -14,7 +14,8 @@ def bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def dense_attention(q_bits, k_bits, v_bits, page_table, seq_lens, cu_q_lens, scale):
+def dense_attention(q_bits, k_bits, v_bits, page_table, seq_lens, cu_q_lens, scale,
+                    causal=True):
     q = bits_to_f64(q_bits)                      # [T, Hq, D]
     kp = bits_to_f64(k_bits)                     # [P, ps, Hkv, D]
     vp = bits_to_f64(v_bits)
@@ -40,7 +41,7 @@ def dense_attention(q_bits, k_bits, v_bits, page_table, seq_lens, cu_q_lens, sca
         # explicit mask matrix: row i (query), column j (key)
         rows = np.arange(qb)[:, None]
         cols = np.arange(kv)[None, :]
-        visible = cols <= rows + (kv - qb)
+        visible = (cols <= rows + (kv - qb)) if causal else np.ones((qb, kv), dtype=bool)
         for h in range(Hq):
             g = h // G
             S = scale * (q[t0:t1, h, :] @ K[:, g, :].T)          # [qb, kv]
