@@ -177,6 +177,25 @@ PA_API int pa_max_splits(const pa_plan *plan);
  * 256. */
 PA_API int pa_set_two_stage_prefill(pa_plan *plan, int on);
 
+/* Mask mode.  1 (default): causal, aligned to the end of each request's KV
+ * (query i of a request with q_b tokens and kv_b keys sees keys
+ * j < kv_b - q_b + i + 1).  0: every query row sees all kv_b keys of its
+ * request -- the non-causal attention asked for in the review thread of
+ * "Unified Triton kernel that doesn't distinguish between prefill + decode"
+ * (vLLM PR #16828) for cascade attention and MLA.  Takes effect at the next
+ * pa_run.  PA_ERR_INVALID for a NULL plan. */
+PA_API int pa_set_causal(pa_plan *plan, int causal);
+
+/* Row stride of page_table in int32 entries (default: capacity).  Row b of
+ * the table starts at page_table + b * row_stride, so the K plane of a
+ * [B, 2, C] table (K page ids in plane 0, V page field in plane 1) is passed
+ * without a copy as page_table = &table[0][0][0] with row_stride = 2 * C
+ * ("integrate PrimTS FMHA kernels", section "Unified page-table metadata").
+ * Both K and V pages are read through these ids.  Applies to pa_run and
+ * pa_append_kv.  PA_ERR_INVALID if row_stride < capacity or the plan is
+ * NULL. */
+PA_API int pa_set_page_table_stride(pa_plan *plan, int row_stride);
+
 /* Decode kernel choice for runs with cu_q_lens == NULL (one query token per
  * request) and at most 32 query heads per KV head.  The decode kernel computes
  * S^T = K Q^T and O^T = V^T P^T with the 128 keys of a tile as the MMA's M

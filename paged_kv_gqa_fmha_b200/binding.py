@@ -27,7 +27,8 @@ STATUS_TIMEOUT = 1 << 4
 EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_scale",
            "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
            "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc",
-           "pa_set_two_stage_prefill", "pa_set_decode_kernel", "pa_append_kv")
+           "pa_set_two_stage_prefill", "pa_set_decode_kernel", "pa_append_kv",
+           "pa_set_causal", "pa_set_page_table_stride")
 
 # Size of the library's static scratch array used by pa_run_noalloc.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -81,6 +82,10 @@ def load_library(path: str = LIB_PATH):
     lib.pa_set_decode_kernel.restype = I
     lib.pa_append_kv.argtypes = [P, P, P, P, P, P, P, P, P]
     lib.pa_append_kv.restype = I
+    lib.pa_set_causal.argtypes = [P, I]
+    lib.pa_set_causal.restype = I
+    lib.pa_set_page_table_stride.argtypes = [P, I]
+    lib.pa_set_page_table_stride.restype = I
     lib.pa_run_noalloc.argtypes = [I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P]
     lib.pa_run_noalloc.restype = I
     if path == LIB_PATH:
@@ -114,6 +119,7 @@ class Plan:
             raise PAError(PA_ERR_INVALID, last_error())
         self.batch, self.heads_q, self.heads_kv = batch, heads_q, heads_kv
         self.head_dim, self.page_size, self.capacity = head_dim, page_size, capacity
+        self._tstride = capacity
         if scale is not None:
             _check(self._lib.pa_set_scale(self._h, float(scale)))
         if num_pages:
@@ -135,6 +141,24 @@ class Plan:
         the keys-as-M decode kernel, False puts both on the one-stage kernel
         (default: head_dim 128 on the decode kernel, 256 on the one-stage)."""
         _check(self._lib.pa_set_decode_kernel(self._h, 1 if on else 0))
+
+    def set_causal(self, causal: bool):
+        """True (default): causal mask aligned to the end of KV; False: every
+        query row sees all of its request's keys."""
+        _check(self._lib.pa_set_causal(self._h, 1 if causal else 0))
+
+    def _bind_table(self, page_table):
+        """Accept a [B, C] int32 table whose rows may be strided (e.g. the K
+        plane of a [B, 2, C] tensor, row stride 2C) and pass its stride on."""
+        B = self.batch
+        if (page_table.dtype != torch.int32 or page_table.dim() != 2
+                or tuple(page_table.shape) != (B, self.capacity) or page_table.stride(1) != 1
+                or page_table.stride(0) < self.capacity):
+            raise ValueError("page_table must be an int32 [%d, %d] tensor with unit column "
+                             "stride and row stride >= %d" % (B, self.capacity, self.capacity))
+        if page_table.stride(0) != self._tstride:
+            _check(self._lib.pa_set_page_table_stride(self._h, int(page_table.stride(0))))
+            self._tstride = int(page_table.stride(0))
 
     def set_scale(self, s: float):
         _check(self._lib.pa_set_scale(self._h, float(s)))
@@ -158,10 +182,12 @@ class Plan:
             raise ValueError("tensors must be on a CUDA device")
         for name, t, dt in (("q", q, torch.bfloat16), ("k_pool", k_pool, torch.bfloat16),
                             ("v_pool", v_pool, torch.bfloat16),
-                            ("page_table", page_table, torch.int32),
                             ("seq_lens", seq_lens, torch.int32)):
             if t.dtype != dt or t.device != dev or not t.is_contiguous():
                 raise ValueError("%s must be a contiguous %s tensor on %s" % (name, dt, dev))
+        if page_table.device != dev:
+            raise ValueError("page_table must be on %s" % dev)
+        self._bind_table(page_table)
         if q.dim() != 3 or q.shape[1] != Hq or q.shape[2] != D:
             raise ValueError("q must be [T, %d, %d], got %s" % (Hq, D, tuple(q.shape)))
         if k_pool.dim() != 4 or tuple(k_pool.shape[1:]) != (self.page_size, Hkv, D):
@@ -170,8 +196,6 @@ class Plan:
         if v_pool.shape != k_pool.shape:
             raise ValueError("v_pool shape %s != k_pool shape %s"
                              % (tuple(v_pool.shape), tuple(k_pool.shape)))
-        if tuple(page_table.shape) != (B, self.capacity):
-            raise ValueError("page_table must be [%d, %d]" % (B, self.capacity))
         if tuple(seq_lens.shape) != (B,):
             raise ValueError("seq_lens must be [%d]" % B)
         if cu_q_lens is not None:
@@ -204,17 +228,19 @@ class Plan:
             raise ValueError("tensors must be on a CUDA device")
         for name, t, dt in (("k_new", k_new, torch.bfloat16), ("v_new", v_new, torch.bfloat16),
                             ("k_pool", k_pool, torch.bfloat16), ("v_pool", v_pool, torch.bfloat16),
-                            ("page_table", page_table, torch.int32),
                             ("seq_lens", seq_lens, torch.int32)):
             if t.dtype != dt or t.device != dev or not t.is_contiguous():
                 raise ValueError("%s must be a contiguous %s tensor on %s" % (name, dt, dev))
+        if page_table.device != dev:
+            raise ValueError("page_table must be on %s" % dev)
+        self._bind_table(page_table)
         if k_new.dim() != 3 or tuple(k_new.shape[1:]) != (Hkv, D) or v_new.shape != k_new.shape:
             raise ValueError("k_new and v_new must be [T, %d, %d]" % (Hkv, D))
         if k_pool.dim() != 4 or tuple(k_pool.shape[1:]) != (self.page_size, Hkv, D) \
                 or v_pool.shape != k_pool.shape:
             raise ValueError("k_pool and v_pool must be [P, %d, %d, %d]" % (self.page_size, Hkv, D))
-        if tuple(page_table.shape) != (B, self.capacity) or tuple(seq_lens.shape) != (B,):
-            raise ValueError("page_table must be [%d, %d] and seq_lens [%d]" % (B, self.capacity, B))
+        if tuple(seq_lens.shape) != (B,):
+            raise ValueError("seq_lens must be [%d]" % B)
         if cu_q_lens is not None:
             if (cu_q_lens.dtype != torch.int32 or tuple(cu_q_lens.shape) != (B + 1,)
                     or cu_q_lens.device != dev or not cu_q_lens.is_contiguous()):

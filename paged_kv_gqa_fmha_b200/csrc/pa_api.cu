@@ -89,6 +89,8 @@ struct pa_plan {
   CUtensorMap tm_q, tm_k, tm_v;
   CUtensorMap tm_o;            // out, box (32, G, 32 / G), 64-byte swizzle
   int use_dec;                 // decode kernel: -1 head_dim 128 only (default), 1 128 and 256, 0 never
+  int causal;                  // 1 (default): causal mask; 0: every row sees all of its keys
+  int tstride;                 // page-table row stride in int32 entries (default C)
   int o_tma;                   // tm_o is used (G divides 32)
   CUtensorMap tm_k2, tm_v2;   // page boxes of box_h2 rows
 };
@@ -437,6 +439,8 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->tm_ptr[0] = p->tm_ptr[1] = p->tm_ptr[2] = p->tm_ptr[3] = nullptr;
   p->o_tma = 0;
   p->use_dec = -1;
+  p->causal = 1;
+  p->tstride = p->C;
   p->tm_num_pages = -1;
   if (alloc_workspace(p) != PA_OK) {
     delete p;
@@ -554,6 +558,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.max_items = p->max_items;
   sp.B = p->B; sp.Hkv = p->Hkv; sp.G = p->G; sp.C = p->C; sp.ps = p->ps; sp.BN = p->BN;
   sp.tpb = p->tpb;
+  sp.causal = p->causal;
   sp.S_max = p->num_splits == 1 ? 1 : p->S_max;
   sp.forced_splits = p->num_splits > 1 ? p->num_splits : 0;
   // decode-only runs (one query token per request) with up to 32 query heads
@@ -579,6 +584,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.S_max = p->S_max;
   ap.tpb = p->tpb;
   ap.box_h = p->box_h;
+  ap.tstride = p->tstride;
+  ap.causal = p->causal;
   ap.o_tma = p->o_tma;
   ap.scale_log2 = p->scale * 1.4426950408889634f;
   const bool prof = p->prof_on && p->prof_n < p->prof_cap;
@@ -653,6 +660,7 @@ int pa_append_kv(pa_plan* p, const void* k_new, const void* v_new, void* k_pool,
   ap.cu_q_lens = cu_q_lens;
   ap.status = &p->hdr->status;
   ap.B = p->B; ap.C = p->C; ap.ps = p->ps; ap.num_pages = p->num_pages;
+  ap.tstride = p->tstride;
   ap.row_u4 = p->Hkv * p->D / 8;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // one warp per new token; T is known only on the device, so the grid is
@@ -667,6 +675,22 @@ int pa_append_kv(pa_plan* p, const void* k_new, const void* v_new, void* k_pool,
     set_err("pa_append_kv: launch failed: %s", cudaGetErrorString(e));
     return PA_ERR_CUDA;
   }
+  return PA_OK;
+}
+
+int pa_set_causal(pa_plan* p, int causal) {
+  if (!p) { set_err("pa_set_causal: NULL plan"); return PA_ERR_INVALID; }
+  p->causal = causal ? 1 : 0;
+  return PA_OK;
+}
+
+int pa_set_page_table_stride(pa_plan* p, int row_stride) {
+  if (!p) { set_err("pa_set_page_table_stride: NULL plan"); return PA_ERR_INVALID; }
+  if (row_stride < p->C) {
+    set_err("pa_set_page_table_stride: row stride %d must be >= capacity %d", row_stride, p->C);
+    return PA_ERR_INVALID;
+  }
+  p->tstride = row_stride;
   return PA_OK;
 }
 
@@ -919,6 +943,7 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   sp.max_items = (int)max_items;
   sp.B = batch; sp.Hkv = heads_kv; sp.G = G; sp.C = capacity; sp.ps = page_size; sp.BN = BN;
   sp.tpb = tpb;
+  sp.causal = 1;
   sp.S_max = 1;             // no KV splits on this path
   sp.forced_splits = 0;
   sp.n_ctas = attn_grid(head_dim, nd->n_sm);
@@ -940,6 +965,8 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   ap.S_max = 1;
   ap.tpb = tpb;
   ap.box_h = box_h;
+  ap.tstride = capacity;
+  ap.causal = 1;
   ap.o_tma = 0;   // no map of out here: every block stores O directly
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)head_dim);
   ap.scale_log2 = sc * 1.4426950408889634f;

@@ -34,6 +34,7 @@ struct AppendParams {
   const int* cu_q_lens;       // [B+1] or nullptr (one token per request)
   unsigned* status;
   int B, C, ps, num_pages;
+  int tstride;                // page-table row stride (>= C)
   int row_u4;                 // 16-byte units of one token's K (or V) row: Hkv * D / 8
 };
 
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kAppendThreads) pa_append_kernel(AppendParams 
       continue;
     }
     const int j = kv - qb + i;
-    const int page = __ldg(p.page_table + (size_t)b * p.C + j / p.ps);
+    const int page = __ldg(p.page_table + (size_t)b * p.tstride + j / p.ps);
     if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
       if (lane == 0) atomicOr(p.status, kStatusBadPage);
       continue;

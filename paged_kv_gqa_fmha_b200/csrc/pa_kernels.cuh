@@ -169,6 +169,8 @@ struct AttnParams {
   float* part_lse;            // [B*Hkv*S_max*128]
   unsigned* status;
   int B, Hq, Hkv, G, C, ps, num_pages, S_max, tpb, box_h;
+  int tstride;                // page-table row stride (>= C)
+  int causal;                 // 1: causal mask aligned to the end of KV; 0: all keys
   int o_tma;                  // 1: full blocks store O through the tensor map of out
   float scale_log2;
 };
@@ -219,6 +221,7 @@ struct SchedParams {
   WsHeader* hdr;
   int max_items;
   int B, Hkv, G, C, ps, BN, tpb, S_max, forced_splits, n_ctas;
+  int causal;          // 0: every row of a request sees all of its keys
 };
 
 struct ReqInfo {
@@ -254,8 +257,10 @@ __device__ __forceinline__ ReqInfo read_request(const SchedParams& p, int b) {
 }
 
 // Keys visible to the last row of query block [q0, q0 + n): the causal limit
-// aligned to the end of the request's KV, clamped to [0, kv_len].
-__device__ __forceinline__ int block_kv_hi(int q_len, int kv_len, int q0, int n) {
+// aligned to the end of the request's KV, clamped to [0, kv_len]; all of them
+// without the causal mask.
+__device__ __forceinline__ int block_kv_hi(int q_len, int kv_len, int q0, int n, int causal) {
+  if (!causal) return kv_len;
   int hi = q0 + n + (kv_len - q_len);
   return hi < 0 ? 0 : (hi > kv_len ? kv_len : hi);
 }
@@ -309,14 +314,14 @@ __device__ __forceinline__ Unit unit_of(const SchedParams& p, const int4& ri, co
     u.n_tok = q_len;
     u.split = k;
     u.kv_lo = k * per * p.BN;
-    u.kv_hi = min(block_kv_hi(q_len, kv_len, 0, q_len), (k + 1) * per * p.BN);
+    u.kv_hi = min(block_kv_hi(q_len, kv_len, 0, q_len, p.causal), (k + 1) * per * p.BN);
     u.cost = min(per, tiles - k * per);
   } else {
     u.q0 = k * p.tpb;
     u.n_tok = min(p.tpb, q_len - u.q0);
     u.split = 0;
     u.kv_lo = 0;
-    u.kv_hi = block_kv_hi(q_len, kv_len, u.q0, u.n_tok);
+    u.kv_hi = block_kv_hi(q_len, kv_len, u.q0, u.n_tok, p.causal);
     u.cost = ceil_div(u.kv_hi, p.BN);
   }
   return u;
@@ -354,7 +359,7 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
     int t = 0;
     for (int m = 0; m < nb; ++m) {
       const int q0 = m * p.tpb;
-      t += ceil_div(block_kv_hi(r.q_len, r.kv_len, q0, min(p.tpb, r.q_len - q0)), p.BN);
+      t += ceil_div(block_kv_hi(r.q_len, r.kv_len, q0, min(p.tpb, r.q_len - q0), p.causal), p.BN);
     }
     my_tiles += (unsigned long long)p.Hkv * t;
   }
@@ -391,7 +396,7 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
     if (b < p.B) {
       const ReqInfo r = read_request(p, b);
       const int nb = n_qblocks(r.q_len, p.tpb);
-      const int tiles = ceil_div(block_kv_hi(r.q_len, r.kv_len, 0, r.q_len), p.BN);
+      const int tiles = ceil_div(block_kv_hi(r.q_len, r.kv_len, 0, r.q_len, p.causal), p.BN);
       int ns = 1, per = tiles > 0 ? tiles : 1;
       if (nb == 1 && p.S_max > 1 && tiles > 1) {
         int sp = p.forced_splits > 0 ? p.forced_splits : ceil_div(tiles, chunk);
@@ -454,7 +459,7 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
       const int pair = units2 - 1 - k;
       const int q0 = 2 * pair * p.tpb;
       const int ntok = min(2 * p.tpb, ri.y - q0);
-      const int hi_kv = block_kv_hi(ri.y, ri.w, q0, ntok);
+      const int hi_kv = block_kv_hi(ri.y, ri.w, q0, ntok, p.causal);
       const int pos = u * p.Hkv;
       for (int g = 0; g < p.Hkv; ++g) {
         if (pos + g < p.max_items2) {
@@ -646,7 +651,7 @@ __device__ __forceinline__ int tile_page_id(const AttnParams& p, const WorkItem&
   const int live = min(w.kv_len - n0, BN);
   if (lane * p.box_h >= live) return 0;
   const int col = (n0 + lane * p.box_h) / p.ps;
-  return __ldg(p.page_table + (size_t)w.b * p.C + col);
+  return __ldg(p.page_table + (size_t)w.b * p.tstride + col);
 }
 
 // KV producer warp: K and V tiles in the MMA's consumption order into the slot
@@ -855,7 +860,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
     }
     // keys visible to this row: [kv_lo, lim)
     const int i_r = w.q_tok0 + r / G;
-    const int lim = min(w.kv_hi, i_r + (w.kv_len - w.q_len) + 1);
+    const int lim = p.causal ? min(w.kv_hi, i_r + (w.kv_len - w.q_len) + 1) : w.kv_hi;
     float m_run = -INFINITY, l_run = 0.f;
     for (int j = 0; j < n && ok; ++j) {
       const uint32_t g = g_base + j, sb = g & 1;

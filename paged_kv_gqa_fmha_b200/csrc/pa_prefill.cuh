@@ -69,13 +69,13 @@ struct PairShape {
   int n;          // KV tiles of the item (max of the two)
 };
 
-__device__ __forceinline__ PairShape pair_shape(const WorkItem& w, int tpb, int BN) {
+__device__ __forceinline__ PairShape pair_shape(const WorkItem& w, int tpb, int BN, int causal) {
   PairShape s;
   s.tok[0] = max(0, min(tpb, w.q_len - w.q_tok0));
   s.tok[1] = max(0, min(tpb, w.q_len - w.q_tok0 - s.tok[0]));
   for (int x = 0; x < 2; ++x) {
     const int q0 = w.q_tok0 + x * tpb;
-    int hi = q0 + s.tok[x] + (w.kv_len - w.q_len);
+    int hi = causal ? q0 + s.tok[x] + (w.kv_len - w.q_len) : w.kv_len;
     hi = hi < 0 ? 0 : (hi > w.kv_len ? w.kv_len : hi);
     s.lim[x] = hi;
     s.nt[x] = s.tok[x] > 0 ? ceil_div(hi, BN) : 0;
@@ -105,7 +105,7 @@ __device__ __forceinline__ void pair_q_loader(const CUtensorMap* tm_q, const Att
   ItemStream items(p.items, n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
-    const PairShape ps = pair_shape(w, p.tpb, C::BN);
+    const PairShape ps = pair_shape(w, p.tpb, C::BN, p.causal);
     for (int x = 0; x < 2; ++x) {
       if (ps.nt[x] == 0) continue;
       if (!warp_wait(bar0 + 8 * (C::B_QEMPTY + x), (qc[x] & 1) ^ 1, abort)) { ok = false; break; }
@@ -182,7 +182,7 @@ __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUt
   ItemStream items(p.items, n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
-    const int n = pair_shape(w, p.tpb, C::BN).n;
+    const int n = pair_shape(w, p.tpb, C::BN, p.causal).n;
     if (n == 0) {
       have_next = false;
       continue;
@@ -229,7 +229,7 @@ __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUt
           pid_k = tile_page_id(p, w, j + 1, C::BN, lane);
         } else {
           WorkItem nw;
-          if (items.peek(nw) && pair_shape(nw, p.tpb, C::BN).n > 0) {
+          if (items.peek(nw) && pair_shape(nw, p.tpb, C::BN, p.causal).n > 0) {
             pid_next = tile_page_id(p, nw, 0, C::BN, lane);
             have_next = true;
           }
@@ -298,7 +298,7 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
   };
 
   while (ok && items.next(w)) {
-    const PairShape ps = pair_shape(w, p.tpb, C::BN);
+    const PairShape ps = pair_shape(w, p.tpb, C::BN, p.causal);
     const int n = ps.n;
     if (n == 0) continue;
     for (int x = 0; x < 2 && ok; ++x)
@@ -376,7 +376,7 @@ __device__ __forceinline__ void pair_softmax(const CUtensorMap* tm_o, const Attn
   ItemStream items(p.items, n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
-    const PairShape ps = pair_shape(w, p.tpb, BN);
+    const PairShape ps = pair_shape(w, p.tpb, BN, p.causal);
     const int n = ps.n, tok = ps.tok[x], nt = ps.nt[x];
     const int n_rows = tok * G;
     const bool real = r < n_rows;
@@ -395,7 +395,7 @@ __device__ __forceinline__ void pair_softmax(const CUtensorMap* tm_o, const Attn
       continue;
     }
     const int i_r = q_first + r / G;
-    const int lim = min(ps.lim[x], i_r + (w.kv_len - w.q_len) + 1);
+    const int lim = p.causal ? min(ps.lim[x], i_r + (w.kv_len - w.q_len) + 1) : ps.lim[x];
     // the stage whose P arrival gates the first P V of the last tile cleans
     // that tile's V rows at and past kv_len
     const bool zero_v = ((n - 1) * BN + BN > w.kv_len) &&

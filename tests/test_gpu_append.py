@@ -133,3 +133,23 @@ def test_append_full_prefill_size():
     assert plan.status() == 0
     assert np.array_equal(kp.view(torch.int16).cpu().numpy().view(np.uint16), k_ref)
     assert np.array_equal(vp.view(torch.int16).cpu().numpy().view(np.uint16), v_ref)
+
+
+def test_append_with_strided_table():
+    """pa_append_kv through the K plane of a [B, 2, C] table (row stride 2C)."""
+    c = _case(51, B=5, Hkv=2, D=64, ps=16)
+    k_ref, v_ref, flags = O.append_kv(c["k_new"], c["v_new"], c["k_pool"], c["v_pool"],
+                                      c["table"], c["kv"], c["cu"])
+    assert flags == 0
+    B, C = c["table"].shape
+    t3 = np.full((B, 2, C), -777, dtype=np.int32)
+    t3[:, 0, :] = c["table"]
+    t3 = _t(t3)
+    plan = _plan(c)
+    kp = _t(c["k_pool"], torch.bfloat16)
+    vp = _t(c["v_pool"], torch.bfloat16)
+    plan.append_kv(_t(c["k_new"], torch.bfloat16), _t(c["v_new"], torch.bfloat16), kp, vp,
+                   t3[:, 0, :], _t(c["kv"]), _t(c["cu"]))
+    assert plan.status() == 0
+    assert np.array_equal(kp.view(torch.int16).cpu().numpy().view(np.uint16), k_ref)
+    assert np.array_equal(vp.view(torch.int16).cpu().numpy().view(np.uint16), v_ref)

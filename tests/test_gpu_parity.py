@@ -5,6 +5,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import oracle as O
 from paged_kv_gqa_fmha_b200 import workloads as W
 from tests.gpu_common import (compare, gpu_run, make_plan, oracle_all, oracle_rows,
                               sample_rows)
@@ -288,3 +289,43 @@ def test_full_size_config_sampled_rows(name):
     o = out[torch.from_numpy(rt).long().cuda(), torch.from_numpy(rh).long().cuda()]
     l = lse[torch.from_numpy(rt).long().cuda(), torch.from_numpy(rh).long().cuda()]
     compare(o, l, o_ref, l_ref)
+
+
+# ------------------------------------------------------------------ mask mode, table stride
+@pytest.mark.parametrize("D,ps,G,pairs,splits", [(128, 16, 4, False, 0), (64, 32, 8, False, 0),
+                                                 (256, 64, 2, False, 3), (128, 64, 1, True, 0),
+                                                 (64, 16, 3, True, 0)])
+def test_non_causal_mode(D, ps, G, pairs, splits):
+    """pa_set_causal(plan, 0): every row sees its request's whole KV, on the
+    one-stage kernel (with and without splits) and the two-stage kernel."""
+    spec = W.custom_spec("nc", 2 * G, 2, D, ps, [300, 1, 129, 77, 0], [300, 700, 400, 500, 90])
+    w = gen(spec, 80 + D + ps + G)
+    plan = make_plan(w, num_splits=splits)
+    plan.set_causal(False)
+    if pairs:
+        plan.set_two_stage_prefill(True)
+    out, lse, _ = gpu_run(w, plan)
+    assert plan.status() == 0
+    o_ref, l_ref = O.paged_attention(W.bf16_bits(w["q"]), W.bf16_bits(w["k_pool"]),
+                                     W.bf16_bits(w["v_pool"]), w["page_table_cpu"].numpy(),
+                                     w["seq_lens_cpu"].numpy(), w["cu_q_lens_cpu"].numpy(),
+                                     w["scale"], causal=False)
+    compare(out, lse, o_ref, l_ref)
+
+
+@pytest.mark.parametrize("decode_only", [False, True])
+def test_page_table_row_stride(decode_only):
+    """The K plane of a [B, 2, C] table (row stride 2C) passed without a copy;
+    plane 1 holds garbage that must never be read."""
+    q = [1] * 6 if decode_only else [40, 1, 300, 1, 17, 1]
+    spec = W.custom_spec("stride", 32, 8, 128, 16, q, [900, 1500, 300, 64, 1200, 7],
+                         decode_only=decode_only)
+    w = gen(spec, 90 + int(decode_only))
+    B, C = w["page_table_cpu"].shape
+    t3 = torch.full((B, 2, C), -12345, dtype=torch.int32)
+    t3[:, 0, :] = w["page_table_cpu"]
+    t3 = t3.cuda()
+    plan = make_plan(w)
+    out, lse, _ = gpu_run(w, plan, use_cu=not decode_only, page_table=t3[:, 0, :])
+    assert plan.status() == 0
+    compare(out, lse, *oracle_all(w))
