@@ -177,6 +177,20 @@ PA_API int pa_max_splits(const pa_plan *plan);
  * 256. */
 PA_API int pa_set_two_stage_prefill(pa_plan *plan, int on);
 
+/* Split-KV merge.  0 (default): a separate merge kernel runs after the
+ * attention kernel.  1: fused -- every softmax warp of a split item counts
+ * itself in a per-(request, KV head) counter after writing its partial state,
+ * and the warp that arrives last merges all splits of that (request, KV head)
+ * (the fused split reduction with a per-run counter that "integrate PrimTS
+ * FMHA kernels", section "Planning, preprocessing, and workspace ownership",
+ * names; here the scheduler zeroes the counters every run and no warp waits
+ * for another).  The fused form saves the merge launch but leaves one warp
+ * to merge up to 128 rows, so it is slower when a (request, KV head) has many
+ * rows and splits (0.85 against 0.30 ms per step with G = 32, D = 256).  Both
+ * compute L = ln sum_s exp(L_s), O = sum_s exp(L_s - L) O_s.  Takes effect at
+ * the next pa_run.  PA_ERR_INVALID for a NULL plan. */
+PA_API int pa_set_fused_merge(pa_plan *plan, int on);
+
 /* Mask mode.  1 (default): causal, aligned to the end of each request's KV
  * (query i of a request with q_b tokens and kv_b keys sees keys
  * j < kv_b - q_b + i + 1).  0: every query row sees all kv_b keys of its

@@ -28,7 +28,7 @@ EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_sc
            "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
            "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc",
            "pa_set_two_stage_prefill", "pa_set_decode_kernel", "pa_append_kv",
-           "pa_set_causal", "pa_set_page_table_stride")
+           "pa_set_causal", "pa_set_page_table_stride", "pa_set_fused_merge")
 
 # Size of the library's static scratch array used by pa_run_noalloc.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -84,6 +84,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_append_kv.restype = I
     lib.pa_set_causal.argtypes = [P, I]
     lib.pa_set_causal.restype = I
+    lib.pa_set_fused_merge.argtypes = [P, I]
+    lib.pa_set_fused_merge.restype = I
     lib.pa_set_page_table_stride.argtypes = [P, I]
     lib.pa_set_page_table_stride.restype = I
     lib.pa_run_noalloc.argtypes = [I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P]
@@ -141,6 +143,11 @@ class Plan:
         the keys-as-M decode kernel, False puts both on the one-stage kernel
         (default: head_dim 128 on the decode kernel, 256 on the one-stage)."""
         _check(self._lib.pa_set_decode_kernel(self._h, 1 if on else 0))
+
+    def set_fused_merge(self, on: bool):
+        """True: split-KV partials are merged by the last split warp of each
+        (request, KV head); False (default): by a separate merge kernel."""
+        _check(self._lib.pa_set_fused_merge(self._h, 1 if on else 0))
 
     def set_causal(self, causal: bool):
         """True (default): causal mask aligned to the end of KV; False: every

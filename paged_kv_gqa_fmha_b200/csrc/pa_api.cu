@@ -90,6 +90,8 @@ struct pa_plan {
   CUtensorMap tm_o;            // out, box (32, G, 32 / G), 64-byte swizzle
   int use_dec;                 // decode kernel: -1 head_dim 128 only (default), 1 128 and 256, 0 never
   int causal;                  // 1 (default): causal mask; 0: every row sees all of its keys
+  int fused_merge;             // 1: the last split warp merges; 0 (default): merge kernel
+  int* split_cnt;              // [B * Hkv] fused-merge counters (plans with splits)
   int tstride;                 // page-table row stride in int32 entries (default C)
   int o_tma;                   // tm_o is used (G divides 32)
   CUtensorMap tm_k2, tm_v2;   // page boxes of box_h2 rows
@@ -141,6 +143,8 @@ int alloc_workspace(pa_plan* p) {
   const size_t o_items2 = off; off = align_up(off + sizeof(pa::PackedItem) * (size_t)max_items2, 256);
   const size_t o_plse = off; off = align_up(off + sizeof(float) * n_part_rows, 256);
   const size_t o_po = off; off = align_up(off + sizeof(float) * n_part_rows * p->D, 256);
+  const size_t o_cnt = off;
+  off = align_up(off + (p->S_max > 1 ? sizeof(int) * (size_t)p->B * p->Hkv : 0), 256);
   void* ws = nullptr;
   cudaError_t e = cudaMalloc(&ws, off);
   if (e != cudaSuccess) {
@@ -168,6 +172,7 @@ int alloc_workspace(pa_plan* p) {
   p->max_items2 = (int)max_items2;
   p->part_lse = reinterpret_cast<float*>(c + o_plse);
   p->part_o = reinterpret_cast<float*>(c + o_po);
+  p->split_cnt = p->S_max > 1 ? reinterpret_cast<int*>(c + o_cnt) : nullptr;
   p->max_items = (int)max_items;
   return PA_OK;
 }
@@ -440,6 +445,8 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->o_tma = 0;
   p->use_dec = -1;
   p->causal = 1;
+  p->fused_merge = 0;
+  p->split_cnt = nullptr;
   p->tstride = p->C;
   p->tm_num_pages = -1;
   if (alloc_workspace(p) != PA_OK) {
@@ -560,6 +567,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.tpb = p->tpb;
   sp.causal = p->causal;
   sp.S_max = p->num_splits == 1 ? 1 : p->S_max;
+  const bool fused = p->fused_merge && sp.S_max > 1;
+  sp.split_cnt = fused ? p->split_cnt : nullptr;
   sp.forced_splits = p->num_splits > 1 ? p->num_splits : 0;
   // decode-only runs (one query token per request) with up to 32 query heads
   // per KV head go to the keys-as-M decode kernel (one CTA per SM)
@@ -587,6 +596,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.tstride = p->tstride;
   ap.causal = p->causal;
   ap.o_tma = p->o_tma;
+  ap.split_cnt = p->split_cnt;
+  ap.fused_merge = fused ? 1 : 0;
   ap.scale_log2 = p->scale * 1.4426950408889634f;
   const bool prof = p->prof_on && p->prof_n < p->prof_cap;
   if (prof) cudaEventRecord(p->prof_ev[2 * p->prof_n], st);
@@ -606,7 +617,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     cudaEventRecord(p->prof_ev[2 * p->prof_n + 1], st);
     ++p->prof_n;
   }
-  if (le == cudaSuccess && sp.S_max > 1) {
+  if (le == cudaSuccess && sp.S_max > 1 && !fused) {
     pa::MergeParams mp;
     mp.req_info = p->req_info;
     mp.split_list = p->split_list;
@@ -622,7 +633,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     set_err("pa_run: launch failed: %s", cudaGetErrorString(le));
     return PA_ERR_CUDA;
   }
-  p->last_launches = 2 + (pairs ? 1 : 0) + (sp.S_max > 1 ? 1 : 0);
+  p->last_launches = 2 + (pairs ? 1 : 0) + (sp.S_max > 1 && !fused ? 1 : 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_err("pa_run: launch failed: %s", cudaGetErrorString(e));
@@ -675,6 +686,12 @@ int pa_append_kv(pa_plan* p, const void* k_new, const void* v_new, void* k_pool,
     set_err("pa_append_kv: launch failed: %s", cudaGetErrorString(e));
     return PA_ERR_CUDA;
   }
+  return PA_OK;
+}
+
+int pa_set_fused_merge(pa_plan* p, int on) {
+  if (!p) { set_err("pa_set_fused_merge: NULL plan"); return PA_ERR_INVALID; }
+  p->fused_merge = on ? 1 : 0;
   return PA_OK;
 }
 
@@ -944,6 +961,7 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   sp.B = batch; sp.Hkv = heads_kv; sp.G = G; sp.C = capacity; sp.ps = page_size; sp.BN = BN;
   sp.tpb = tpb;
   sp.causal = 1;
+  sp.split_cnt = nullptr;
   sp.S_max = 1;             // no KV splits on this path
   sp.forced_splits = 0;
   sp.n_ctas = attn_grid(head_dim, nd->n_sm);
@@ -967,6 +985,8 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   ap.box_h = box_h;
   ap.tstride = capacity;
   ap.causal = 1;
+  ap.split_cnt = nullptr;
+  ap.fused_merge = 0;
   ap.o_tma = 0;   // no map of out here: every block stores O directly
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)head_dim);
   ap.scale_log2 = sc * 1.4426950408889634f;

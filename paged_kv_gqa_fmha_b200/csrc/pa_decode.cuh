@@ -395,6 +395,7 @@ __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, u
           else if (p.lse) p.lse[orow0 + r] = -INFINITY;
         }
       }
+      if (split && p.fused_merge) split_arrive_and_merge(p, w, D);
       continue;
     }
     float m_run[RR], l_part[RR];
@@ -527,6 +528,7 @@ __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, u
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar0 + 8 * C::B_OEMPTY);
+    if (split && p.fused_merge) split_arrive_and_merge(p, w, D);
     ++q_cnt;
   }
 }

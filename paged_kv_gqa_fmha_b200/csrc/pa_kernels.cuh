@@ -172,8 +172,84 @@ struct AttnParams {
   int tstride;                // page-table row stride (>= C)
   int causal;                 // 1: causal mask aligned to the end of KV; 0: all keys
   int o_tma;                  // 1: full blocks store O through the tensor map of out
+  int* split_cnt;             // [B * Hkv] arrivals of split softmax warps (zeroed per run)
+  int fused_merge;            // 1: the last split warp of a (request, KV head) merges
   float scale_log2;
 };
+
+constexpr int kSoftmaxWarps = 4;      // softmax warps per CTA in every attention kernel
+
+// Merge of one row's split states by one warp: L = ln sum_s exp(L_s),
+// O = sum_s exp(L_s - L) O_s, the exact identity for attention states over
+// disjoint key ranges; empty splits (L_s = -inf) have weight 0.  Partials are
+// read through L2 (ld.global.cg): in the fused path other CTAs wrote them
+// during this launch.  part rows of the split s are base + s * 128.
+__device__ __forceinline__ void merge_one_row(const float* part_o, const float* part_lse,
+                                              size_t base, int ns, int D, uint16_t* out_row,
+                                              float* lse_out) {
+  const int lane = threadIdx.x & 31;
+  const float l0 = lane < ns ? __ldcg(part_lse + base + (size_t)lane * kBM) : -INFINITY;
+  const float l1 = lane + 32 < ns ? __ldcg(part_lse + base + (size_t)(lane + 32) * kBM) : -INFINITY;
+  float m = fmaxf(l0, l1);
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float e = 0.f;
+  if (m != -INFINITY)
+    e = (l0 == -INFINITY ? 0.f : expf(l0 - m)) + (l1 == -INFINITY ? 0.f : expf(l1 - m));
+  for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+  const float L = (m == -INFINITY) ? -INFINITY : m + logf(e);
+  const float w0 = (L == -INFINITY || l0 == -INFINITY) ? 0.f : expf(l0 - L);
+  const float w1 = (L == -INFINITY || l1 == -INFINITY) ? 0.f : expf(l1 - L);
+  for (int d0 = 0; d0 < D; d0 += 128) {            // warp-uniform loop
+    const int d = d0 + lane * 4;
+    const bool act = d < D;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < ns; ++s) {
+      const float wgt = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
+      if (act) {
+        const float4 o = __ldcg(reinterpret_cast<const float4*>(part_o + (base + (size_t)s * kBM) * D + d));
+        a0 = fmaf(wgt, o.x, a0);
+        a1 = fmaf(wgt, o.y, a1);
+        a2 = fmaf(wgt, o.z, a2);
+        a3 = fmaf(wgt, o.w, a3);
+      }
+    }
+    if (act) {
+      uint2 pk;
+      pk.x = pack_bf16x2(a0, a1);
+      pk.y = pack_bf16x2(a2, a3);
+      *reinterpret_cast<uint2*>(out_row + d) = pk;
+    }
+  }
+  if (lane == 0 && lse_out) *lse_out = L;
+}
+
+// Fused split-KV reduction.  Called by every softmax warp of a CTA after it
+// wrote its share of a split item's partials (or nothing, for rows it does not
+// own): each warp publishes its writes (__threadfence) and counts itself in
+// the (request, KV head) counter; the warp that brings the count to
+// kSoftmaxWarps * n_splits has every split's partials visible and merges all
+// rows of the item into out and lse.  No warp waits for another.
+__device__ __forceinline__ void split_arrive_and_merge(const AttnParams& p, const WorkItem& w,
+                                                       int D) {
+  const int lane = threadIdx.x & 31;
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0)
+    last = atomicAdd(p.split_cnt + (size_t)w.b * p.Hkv + w.kvh, 1) ==
+           kSoftmaxWarps * w.n_splits - 1;
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+  const int n_rows = w.n_tok * p.G;
+  for (int r = 0; r < n_rows; ++r) {
+    const size_t base = ((size_t)w.b * p.Hkv + w.kvh) * p.S_max * kBM + r;
+    const size_t orow = (size_t)(w.t_base + w.q_tok0 + r / p.G) * p.Hq + w.kvh * p.G + r % p.G;
+    merge_one_row(p.part_o, p.part_lse, base, w.n_splits, D, p.out + orow * D,
+                  p.lse ? p.lse + orow : nullptr);
+  }
+}
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -222,6 +298,7 @@ struct SchedParams {
   int max_items;
   int B, Hkv, G, C, ps, BN, tpb, S_max, forced_splits, n_ctas;
   int causal;          // 0: every row of a request sees all of its keys
+  int* split_cnt;      // [B * Hkv] fused-merge counters, zeroed here every run (or nullptr)
 };
 
 struct ReqInfo {
@@ -347,6 +424,8 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
   const int tid = threadIdx.x, lane = tid & 31;
   for (int i = tid; i < kCostBuckets; i += blockDim.x) hist[i] = 0;
   if (tid == 0) { total_tiles = 0; s_flags = 0; }
+  if (p.split_cnt)
+    for (int i = tid; i < p.B * p.Hkv; i += blockDim.x) p.split_cnt[i] = 0;
   __syncthreads();
 
   // 1.
@@ -856,6 +935,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
           if (p.lse) p.lse[(size_t)t * p.Hq + h] = -INFINITY;
         }
       }
+      if (split && p.fused_merge) split_arrive_and_merge(p, w, D);
       continue;
     }
     // keys visible to this row: [kv_lo, lim)
@@ -1052,6 +1132,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar0 + 8 * C::B_OEMPTY);
+    if (split && p.fused_merge) split_arrive_and_merge(p, w, D);
     g_base += n;
     ld_base += 2 * n;
   }
@@ -1154,7 +1235,7 @@ struct MergeParams {
 __global__ void __launch_bounds__(128) pa_merge_kernel(MergeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n_req = p.hdr->n_split_reqs;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const int n_units = n_req * p.Hkv * kBM;
   for (int u = blockIdx.x * 4 + warp; u < n_units; u += gridDim.x * 4) {
     const int r = u % kBM;
@@ -1165,43 +1246,10 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(MergeParams p) {
     const int ns = ri.x;
     if (r >= ri.y * p.G) continue;
     const size_t base = ((size_t)b * p.Hkv + kvh) * p.S_max * kBM + r;   // + s * kBM
-    const float l0 = lane < ns ? p.part_lse[base + (size_t)lane * kBM] : -INFINITY;
-    const float l1 = lane + 32 < ns ? p.part_lse[base + (size_t)(lane + 32) * kBM] : -INFINITY;
-    float m = fmaxf(l0, l1);
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float e = 0.f;
-    if (m != -INFINITY)
-      e = (l0 == -INFINITY ? 0.f : expf(l0 - m)) + (l1 == -INFINITY ? 0.f : expf(l1 - m));
-    for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-    const float L = (m == -INFINITY) ? -INFINITY : m + logf(e);
-    const float w0 = (L == -INFINITY || l0 == -INFINITY) ? 0.f : expf(l0 - L);
-    const float w1 = (L == -INFINITY || l1 == -INFINITY) ? 0.f : expf(l1 - L);
     const int t = ri.z + r / p.G;
     const int h = kvh * p.G + r % p.G;
-    for (int d0 = 0; d0 < p.D; d0 += 128) {          // warp-uniform loop
-      const int d = d0 + lane * 4;
-      const bool act = d < p.D;
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
-      for (int s = 0; s < ns; ++s) {
-        const float wgt = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
-        if (act) {
-          const float4 o =
-              *reinterpret_cast<const float4*>(p.part_o + (base + (size_t)s * kBM) * p.D + d);
-          a0 = fmaf(wgt, o.x, a0);
-          a1 = fmaf(wgt, o.y, a1);
-          a2 = fmaf(wgt, o.z, a2);
-          a3 = fmaf(wgt, o.w, a3);
-        }
-      }
-      if (act) {
-        uint2 pk;
-        pk.x = pack_bf16x2(a0, a1);
-        pk.y = pack_bf16x2(a2, a3);
-        *reinterpret_cast<uint2*>(p.out + ((size_t)t * p.Hq + h) * p.D + d) = pk;
-      }
-    }
-    if (lane == 0 && p.lse) p.lse[(size_t)t * p.Hq + h] = L;
+    merge_one_row(p.part_o, p.part_lse, base, ns, p.D, p.out + ((size_t)t * p.Hq + h) * p.D,
+                  p.lse ? p.lse + (size_t)t * p.Hq + h : nullptr);
   }
 }
 

@@ -107,11 +107,15 @@ def test_two_stage_prefill_kernel(D, ps, G):
 
 
 # ------------------------------------------------------------------ split-KV (a8)
-@pytest.mark.parametrize("splits", [1, 2, 7, 0])
-def test_split_invariance(splits):
+@pytest.mark.parametrize("splits,fused", [(1, True), (2, True), (7, True), (0, True), (2, False),
+                                          (7, False), (0, False)])
+def test_split_invariance(splits, fused):
+    """Split counts give the same result, merged by the last split warp
+    (fused) or by the separate merge kernel."""
     spec = W.custom_spec("split", 16, 2, 128, 32, [1, 1, 3, 1], [3000, 1200, 2500, 64])
     w = gen(spec, 13)
     plan = make_plan(w, num_splits=splits)
+    plan.set_fused_merge(fused)
     out, lse, _ = gpu_run(w, plan)
     compare(out, lse, *oracle_all(w))
     ref_plan = make_plan(w, num_splits=1)
@@ -124,8 +128,12 @@ def test_split_long_gqa32_head_dim_256():
     spec = W.custom_spec("split256", 64, 2, 256, 128, [1, 1], [20000, 7000])
     w = gen(spec, 14)
     for splits in (0, 5):
-        out, lse, _ = gpu_run(w, make_plan(w, num_splits=splits))
-        compare(out, lse, *oracle_all(w))
+        for fused in (True, False):
+            plan = make_plan(w, num_splits=splits)
+            plan.set_fused_merge(fused)
+            out, lse, _ = gpu_run(w, plan)
+            assert plan.status() == 0
+            compare(out, lse, *oracle_all(w))
 
 
 # ------------------------------------------------------------------ invariants on the GPU path
