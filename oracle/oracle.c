@@ -65,6 +65,10 @@ typedef struct {
     const int32_t *page_table, *seq_lens, *cu_q_lens;
     double scale;
     int non_causal;       /* 0: causal mask (default); 1: every row sees all kv_b keys */
+    /* fp8 pools: when k8 is set, K and V are e4m3 codes [P, ps, Hkv, D] and
+     * the values are code * k_scale, code * v_scale */
+    const uint8_t *k8, *v8;
+    double k_scale, v_scale;
     double *out, *lse;
     /* rows to compute: either all (rows == NULL) or a list of (t, h) */
     const int32_t *row_t, *row_h;
@@ -81,6 +85,31 @@ typedef struct {
 static double pool_at(const job_t *J, const uint16_t *pool, long page, long slot, long g, long d) {
     long idx = ((page * J->ps + slot) * J->Hkv + g) * J->D + d;
     return bf16_to_double(pool[idx]);
+}
+
+/*
+ * FP8 E4M3 code -> double, from the format's definition (the OCP 8-bit
+ * floating point format, E4M3 variant): 1 sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent 0 encodes subnormals m * 2^-9; the one
+ * pattern S.1111.111 is NaN and there are no infinities (largest 448).
+ */
+static double e4m3_to_double(uint8_t c) {
+    const int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = m * ldexp(1.0, -9);
+    else v = (1.0 + m / 8.0) * ldexp(1.0, e - 7);
+    return sgn ? -v : v;
+}
+
+static double k_at(const job_t *J, long page, long slot, long g, long d) {
+    if (J->k8) return J->k_scale * e4m3_to_double(J->k8[((page * J->ps + slot) * J->Hkv + g) * J->D + d]);
+    return pool_at(J, J->k_pool, page, slot, g, d);
+}
+
+static double v_at(const job_t *J, long page, long slot, long g, long d) {
+    if (J->v8) return J->v_scale * e4m3_to_double(J->v8[((page * J->ps + slot) * J->Hkv + g) * J->D + d]);
+    return pool_at(J, J->v_pool, page, slot, g, d);
 }
 
 /* One output row: token t (global packed index), query head h.  Returns 0 or
@@ -116,7 +145,7 @@ static int one_row(const job_t *J, long t, int h, double *o_row, double *lse_out
         long slot = j % J->ps;
         double acc = 0.0;
         for (int d = 0; d < D; ++d)
-            acc += bf16_to_double(qrow[d]) * pool_at(J, J->k_pool, page, slot, g, d);
+            acc += bf16_to_double(qrow[d]) * k_at(J, page, slot, g, d);
         s[j] = J->scale * acc;
         if (s[j] > m) m = s[j];
     }
@@ -129,7 +158,7 @@ static int one_row(const job_t *J, long t, int h, double *o_row, double *lse_out
         long page = J->page_table[(long)b * J->C + j / J->ps];
         long slot = j % J->ps;
         double w = s[j] / l;
-        for (int d = 0; d < D; ++d) o_row[d] += w * pool_at(J, J->v_pool, page, slot, g, d);
+        for (int d = 0; d < D; ++d) o_row[d] += w * v_at(J, page, slot, g, d);
     }
     *lse_out = m + log(l);
     return 0;
@@ -247,6 +276,32 @@ int oracle_paged_attention_mode(int B, int Hq, int Hkv, int D, int ps, int C, in
     J.scale = scale; J.out = out; J.lse = lse;
     J.non_causal = causal ? 0 : 1;
     return run_job(&J, nthreads);
+}
+
+/*
+ * FP8 KV cache with per-tensor descales (the "fp8 KV cache with descale,
+ * bf16 output" variants that "[Perf][FA4] Warm up dense (paged) FA4 attention
+ * kernels", vLLM PR #48156, warms up): k8 / v8 are E4M3 codes laid out like
+ * the bf16 pools and K = code * k_scale, V = code * v_scale.  q stays bf16;
+ * everything else is the causal attention above, in fp64.
+ */
+int oracle_paged_attention_fp8(int B, int Hq, int Hkv, int D, int ps, int C, int num_pages,
+                               const uint16_t *q, const uint8_t *k8, const uint8_t *v8,
+                               double k_scale, double v_scale, const int32_t *page_table,
+                               const int32_t *seq_lens, const int32_t *cu_q_lens, double scale,
+                               double *out, double *lse, int nthreads) {
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.ps = ps; J.C = C; J.num_pages = num_pages;
+    J.q = q; J.k8 = k8; J.v8 = v8; J.k_scale = k_scale; J.v_scale = v_scale;
+    J.page_table = page_table; J.seq_lens = seq_lens; J.cu_q_lens = cu_q_lens;
+    J.scale = scale; J.out = out; J.lse = lse;
+    return run_job(&J, nthreads);
+}
+
+/* E4M3 decoding of n codes (exposed for the pins). */
+void oracle_e4m3_decode(const uint8_t *codes, long n, double *out) {
+    for (long i = 0; i < n; ++i) out[i] = e4m3_to_double(codes[i]);
 }
 
 /* Only the listed rows: row u is (token row_t[u], head row_h[u]); out is

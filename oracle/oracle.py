@@ -48,6 +48,11 @@ def _declare(lib):
     lib.oracle_paged_attention_mode.argtypes = [i, i, i, i, i, i, i, P, P, P, P, P, P,
                                                 ctypes.c_double, i, P, P, i]
     lib.oracle_paged_attention_mode.restype = i
+    lib.oracle_paged_attention_fp8.argtypes = [i, i, i, i, i, i, i, P, P, P, ctypes.c_double,
+                                               ctypes.c_double, P, P, P, ctypes.c_double, P, P, i]
+    lib.oracle_paged_attention_fp8.restype = i
+    lib.oracle_e4m3_decode.argtypes = [P, ctypes.c_long, P]
+    lib.oracle_e4m3_decode.restype = None
     lib.oracle_merge_states.argtypes = [i, i, P, P, P, P]
     lib.oracle_merge_states.restype = None
     lib.oracle_append_kv.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P]
@@ -173,3 +178,35 @@ def append_kv(k_new, v_new, k_pool, v_pool, page_table, seq_lens, cu_q_lens, num
                                      _ptr(k_out), _ptr(v_out), _ptr(page_table), _ptr(seq_lens),
                                      _ptr(cu))
     return k_out, v_out, int(flags)
+
+
+def e4m3_decode(codes):
+    """E4M3 codes (uint8) -> float64 values, as the oracle reads fp8 pools."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.zeros(codes.shape, dtype=np.float64)
+    _load().oracle_e4m3_decode(_ptr(codes), codes.size, _ptr(out))
+    return out
+
+
+def paged_attention_fp8(q, k8, v8, k_scale, v_scale, page_table, seq_lens, cu_q_lens, scale,
+                        num_pages: int = 0, nthreads: int | None = None, lib=None):
+    """Causal attention over E4M3 pools (uint8 codes [P, ps, Hkv, D]) with
+    per-tensor descales; q as bf16 bits.  Returns (out, lse) in float64."""
+    q = _u16(q)
+    k8 = np.ascontiguousarray(k8, dtype=np.uint8)
+    v8 = np.ascontiguousarray(v8, dtype=np.uint8)
+    page_table, seq_lens, cu_q_lens = _i32(page_table), _i32(seq_lens), _i32(cu_q_lens)
+    T, Hq, D = q.shape
+    _, ps, Hkv, D2 = k8.shape
+    assert D2 == D and v8.shape == k8.shape
+    B, C = page_table.shape
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    lse = np.zeros((T, Hq), dtype=np.float64)
+    rc = (lib or _load()).oracle_paged_attention_fp8(
+        B, Hq, Hkv, D, ps, C, int(num_pages), _ptr(q), _ptr(k8), _ptr(v8), float(k_scale),
+        float(v_scale), _ptr(page_table), _ptr(seq_lens), _ptr(cu_q_lens), float(scale),
+        _ptr(out), _ptr(lse), int(nthreads or default_threads()))
+    if rc:
+        raise ValueError("oracle: %s" % {1: "live page id out of range",
+                                         2: "out of memory"}.get(rc, rc))
+    return out, lse

@@ -16,9 +16,12 @@ def bits_to_f64(bits: np.ndarray) -> np.ndarray:
 
 def dense_attention(q_bits, k_bits, v_bits, page_table, seq_lens, cu_q_lens, scale,
                     causal=True):
-    q = bits_to_f64(q_bits)                      # [T, Hq, D]
-    kp = bits_to_f64(k_bits)                     # [P, ps, Hkv, D]
-    vp = bits_to_f64(v_bits)
+    return dense_attention_values(bits_to_f64(q_bits), bits_to_f64(k_bits), bits_to_f64(v_bits),
+                                  page_table, seq_lens, cu_q_lens, scale, causal)
+
+
+def dense_attention_values(q, kp, vp, page_table, seq_lens, cu_q_lens, scale, causal=True):
+    """The same on float64 values: q [T, Hq, D], pools [P, ps, Hkv, D]."""
     T, Hq, D = q.shape
     P, ps, Hkv, _ = kp.shape
     B = len(seq_lens)
