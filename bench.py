@@ -490,7 +490,49 @@ def per_config(peaks):
         del w
         torch.cuda.empty_cache()
     res["kv_append"] = kv_append_rates(bw)
+    res["kv_fp8_decode"] = kv_fp8_decode_rates(bw)
     return res
+
+
+def kv_fp8_decode_rates(bw):
+    """Decode over E4M3 pools (pa_set_kv_fp8) on the decode workloads: the
+    bf16 pools are quantised on the device (x4, round to nearest E4M3) and
+    read back with descales 0.25.  Bytes per launch = the bf16 formula with K
+    and V at one byte per element; per-launch CUDA events (the plan's profile
+    pairs) over 20 launches after 5 warm-up launches (pools larger than L2)."""
+    out = {}
+    for name in ("llama8b_decode", "long_gqa32_decode"):
+        w = W.generate(W.CONFIGS[name], W.default_seed(name), device="cuda")
+        c = work_counts(w)
+        k8 = torch.empty(w["k_pool"].shape, dtype=torch.uint8, device="cuda")
+        v8 = torch.empty_like(k8)
+        for src, dst in ((w["k_pool"], k8), (w["v_pool"], v8)):
+            for a in range(0, src.shape[0], 4096):     # chunks bound the fp32 temporaries
+                dst[a:a + 4096] = (src[a:a + 4096].float() * 4).to(
+                    torch.float8_e4m3fn).view(torch.uint8)
+        del w["k_pool"], w["v_pool"]
+        torch.cuda.empty_cache()
+        plan = make_plan(w)
+        plan.set_kv_fp8(True, 0.25, 0.25)
+        args = (w["q"], k8, v8, w["page_table"], w["seq_lens"], None)
+        for _ in range(5):
+            plan.run(*args)
+        torch.cuda.synchronize()
+        plan.profile_start(20)
+        for _ in range(20):
+            plan.run(*args)
+        attn_ms, n_rec, _ = plan.profile_read()
+        ms = attn_ms / max(1, n_rec)
+        nbytes = c["bytes"] - c["kv_bytes"] // 2
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"attn_kernel_ms": ms, "algorithmic_bytes": nbytes, "kernel_GBps": gbs,
+                     "hbm_frac": gbs / bw, "status_word": plan.status(),
+                     "kernel": "pa_decode_kernel<%d, %d, true>" % (
+                         w["D"], max(4, 1 << (w["Hq"] // w["Hkv"] - 1).bit_length()))}
+        plan.close()
+        del w, k8, v8
+        torch.cuda.empty_cache()
+    return out
 
 
 def kv_append_rates(bw):

@@ -222,6 +222,22 @@ PA_API int pa_set_page_table_stride(pa_plan *plan, int row_stride);
  * pa_run; no reallocation.  PA_ERR_INVALID for a NULL plan. */
 PA_API int pa_set_decode_kernel(pa_plan *plan, int on);
 
+/* E4M3 (FP8) KV pools with per-tensor descales ("[Attention] FA4
+ * integration", vLLM #32974: the fp8 KV-cache variant with descale factors
+ * and bf16 output; the format is OCP FP8 E4M3: bias 7, 3 mantissa bits,
+ * subnormals, S.1111.111 NaN, no infinities).  With on != 0 the k_pool and
+ * v_pool of the following pa_run calls are uint8 [P, ps, Hkv, D] arrays of
+ * E4M3 codes, and attention is computed as if the pools held
+ * k_scale * decode(code) and v_scale * decode(code); q stays bf16, out stays
+ * bf16, lse is the log-sum-exp of the descaled logits.  The codes are widened
+ * to fp16 on chip (exact); q and the softmax weights P are rounded to fp16 for
+ * the MMAs (q magnitudes past 65504 saturate).  Decode only: pa_run returns
+ * PA_ERR_UNSUPPORTED when cu_q_lens is not NULL while this is on.  on = 0
+ * restores bf16 pools (descales ignored).  Returns PA_ERR_INVALID for a NULL
+ * plan or a descale that is not finite and > 0, PA_ERR_UNSUPPORTED for a
+ * head_dim other than 128 or 256. */
+PA_API int pa_set_kv_fp8(pa_plan *plan, int on, float k_scale, float v_scale);
+
 /* Paged KV append: write this step's new K and V rows into the pools before
  * attention ("integrate PrimTS FMHA kernels", section "Planning,
  * preprocessing, and workspace ownership": the KV-cache append of the

@@ -28,7 +28,7 @@ EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_sc
            "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
            "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc",
            "pa_set_two_stage_prefill", "pa_set_decode_kernel", "pa_append_kv",
-           "pa_set_causal", "pa_set_page_table_stride", "pa_set_fused_merge")
+           "pa_set_causal", "pa_set_page_table_stride", "pa_set_fused_merge", "pa_set_kv_fp8")
 
 # Size of the library's static scratch array used by pa_run_noalloc.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_set_fused_merge.restype = I
     lib.pa_set_page_table_stride.argtypes = [P, I]
     lib.pa_set_page_table_stride.restype = I
+    lib.pa_set_kv_fp8.argtypes = [P, I, F, F]
+    lib.pa_set_kv_fp8.restype = I
     lib.pa_run_noalloc.argtypes = [I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P]
     lib.pa_run_noalloc.restype = I
     if path == LIB_PATH:
@@ -122,6 +124,7 @@ class Plan:
         self.batch, self.heads_q, self.heads_kv = batch, heads_q, heads_kv
         self.head_dim, self.page_size, self.capacity = head_dim, page_size, capacity
         self._tstride = capacity
+        self._kv_dtype = torch.bfloat16
         if scale is not None:
             _check(self._lib.pa_set_scale(self._h, float(scale)))
         if num_pages:
@@ -148,6 +151,13 @@ class Plan:
         """True: split-KV partials are merged by the last split warp of each
         (request, KV head); False (default): by a separate merge kernel."""
         _check(self._lib.pa_set_fused_merge(self._h, 1 if on else 0))
+
+    def set_kv_fp8(self, on: bool, k_scale: float = 1.0, v_scale: float = 1.0):
+        """True: the pools of later ``run`` calls are uint8 tensors of E4M3
+        codes, read as ``k_scale * code`` and ``v_scale * code`` (decode only:
+        cu_q_lens must be None).  False: bf16 pools."""
+        _check(self._lib.pa_set_kv_fp8(self._h, 1 if on else 0, float(k_scale), float(v_scale)))
+        self._kv_dtype = torch.uint8 if on else torch.bfloat16
 
     def set_causal(self, causal: bool):
         """True (default): causal mask aligned to the end of KV; False: every
@@ -187,8 +197,8 @@ class Plan:
         dev = q.device
         if dev.type != "cuda":
             raise ValueError("tensors must be on a CUDA device")
-        for name, t, dt in (("q", q, torch.bfloat16), ("k_pool", k_pool, torch.bfloat16),
-                            ("v_pool", v_pool, torch.bfloat16),
+        for name, t, dt in (("q", q, torch.bfloat16), ("k_pool", k_pool, self._kv_dtype),
+                            ("v_pool", v_pool, self._kv_dtype),
                             ("seq_lens", seq_lens, torch.int32)):
             if t.dtype != dt or t.device != dev or not t.is_contiguous():
                 raise ValueError("%s must be a contiguous %s tensor on %s" % (name, dt, dev))

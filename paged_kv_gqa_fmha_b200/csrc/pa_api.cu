@@ -95,6 +95,9 @@ struct pa_plan {
   int tstride;                 // page-table row stride in int32 entries (default C)
   int o_tma;                   // tm_o is used (G divides 32)
   CUtensorMap tm_k2, tm_v2;   // page boxes of box_h2 rows
+  int kv_fp8;                  // 1: the pools hold E4M3 codes (decode kernel only)
+  float k_scale, v_scale;      // their per-tensor descales
+  int tm_fp8;                  // the pool maps were encoded for E4M3 pools
 };
 
 namespace {
@@ -179,9 +182,14 @@ int alloc_workspace(pa_plan* p) {
 
 template <int D, int RR>
 cudaError_t set_decode_smem_attr() {
-  return cudaFuncSetAttribute(pa::pa_decode_kernel<D, RR>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              pa::DecCfg<D, pa::DecRows<RR>::NR>::SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(pa::pa_decode_kernel<D, RR, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       pa::DecCfg<D, pa::DecRows<RR>::NR, false>::SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(pa::pa_decode_kernel<D, RR, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pa::DecCfg<D, pa::DecRows<RR>::NR, true>::SMEM_BYTES);
+  return e;
 }
 
 template <int D>
@@ -203,11 +211,12 @@ cudaError_t set_smem_attr() {
   return e;
 }
 
-// Decode-only runs: G query rows per (request, KV head), RR = G rounded up.
-template <int D, int RR>
+// Decode-only runs: G query rows per (request, KV head), RR = G rounded up;
+// F8: E4M3 pools.
+template <int D, int RR, bool F8>
 cudaError_t launch_decode_rr(int n_sm, cudaStream_t st, const CUtensorMap& tk,
                              const CUtensorMap& tv, const pa::AttnParams& ap) {
-  using C = pa::DecCfg<D, pa::DecRows<RR>::NR>;
+  using C = pa::DecCfg<D, pa::DecRows<RR>::NR, F8>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_sm);
   cfg.blockDim = dim3(C::THREADS);
@@ -218,22 +227,25 @@ cudaError_t launch_decode_rr(int n_sm, cudaStream_t st, const CUtensorMap& tk,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, pa::pa_decode_kernel<D, RR>, tk, tv, ap);
+  return cudaLaunchKernelEx(&cfg, pa::pa_decode_kernel<D, RR, F8>, tk, tv, ap);
 }
 
-template <int D>
+template <int D, bool F8>
 cudaError_t launch_decode_d(int G, int n_sm, cudaStream_t st, const CUtensorMap& tk,
                             const CUtensorMap& tv, const pa::AttnParams& ap) {
-  if (G <= 4) return launch_decode_rr<D, 4>(n_sm, st, tk, tv, ap);
-  if (G <= 8) return launch_decode_rr<D, 8>(n_sm, st, tk, tv, ap);
-  if (G <= 16) return launch_decode_rr<D, 16>(n_sm, st, tk, tv, ap);
-  return launch_decode_rr<D, 32>(n_sm, st, tk, tv, ap);
+  if (G <= 4) return launch_decode_rr<D, 4, F8>(n_sm, st, tk, tv, ap);
+  if (G <= 8) return launch_decode_rr<D, 8, F8>(n_sm, st, tk, tv, ap);
+  if (G <= 16) return launch_decode_rr<D, 16, F8>(n_sm, st, tk, tv, ap);
+  return launch_decode_rr<D, 32, F8>(n_sm, st, tk, tv, ap);
 }
 
-cudaError_t launch_decode(int D, int G, int n_sm, cudaStream_t st, const CUtensorMap& tk,
-                          const CUtensorMap& tv, const pa::AttnParams& ap) {
-  return D == 128 ? launch_decode_d<128>(G, n_sm, st, tk, tv, ap)
-                  : launch_decode_d<256>(G, n_sm, st, tk, tv, ap);
+cudaError_t launch_decode(int D, int G, bool fp8, int n_sm, cudaStream_t st,
+                          const CUtensorMap& tk, const CUtensorMap& tv, const pa::AttnParams& ap) {
+  if (fp8)
+    return D == 128 ? launch_decode_d<128, true>(G, n_sm, st, tk, tv, ap)
+                    : launch_decode_d<256, true>(G, n_sm, st, tk, tv, ap);
+  return D == 128 ? launch_decode_d<128, false>(G, n_sm, st, tk, tv, ap)
+                  : launch_decode_d<256, false>(G, n_sm, st, tk, tv, ap);
 }
 
 template <int D>
@@ -298,14 +310,15 @@ cudaError_t launch_merge(int n_sm, cudaStream_t st, const pa::MergeParams& mp) {
 
 int encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
            const cuuint64_t* strides, const cuuint32_t* box, const char* what,
-           CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+           CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B,
+           CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     set_err("pa: cuTensorMapEncodeTiled is not available from the driver");
     return PA_ERR_CUDA;
   }
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides,
+  CUresult r = fn(m, dt, rank, const_cast<void*>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -317,7 +330,7 @@ int encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
 
 int build_maps(pa_plan* p, const void* q, const void* k, const void* v, void* out) {
   if (p->tm_ptr[0] == q && p->tm_ptr[1] == k && p->tm_ptr[2] == v && p->tm_ptr[3] == out &&
-      p->tm_num_pages == p->num_pages)
+      p->tm_num_pages == p->num_pages && p->tm_fp8 == p->kv_fp8)
     return PA_OK;
   const cuuint64_t e = 2;  // bytes per bf16
   // q [T, Hq, D]: dims (D, Hq, T bound); box (64, G, tokens per block).
@@ -338,8 +351,22 @@ int build_maps(pa_plan* p, const void* q, const void* k, const void* v, void* ou
       if (rc) return rc;
     }
   }
-  // pools [P, ps, Hkv, D]: dims (D, Hkv, ps, P); box (64, 1, box_h, 1).
-  {
+  // E4M3 pools [P, ps, Hkv, D] bytes: dims (D, Hkv, ps, P); box (D, 1, box_h, 1),
+  // no swizzle (the decode kernel widens the rows into its own layout)
+  if (p->kv_fp8) {
+    cuuint64_t P = p->num_pages > 0 ? (cuuint64_t)p->num_pages : (cuuint64_t)0x7fffffff;
+    cuuint64_t dims[4] = {(cuuint64_t)p->D, (cuuint64_t)p->Hkv, (cuuint64_t)p->ps, P};
+    cuuint64_t str[3] = {(cuuint64_t)p->D, (cuuint64_t)p->Hkv * p->D,
+                         (cuuint64_t)p->ps * p->Hkv * p->D};
+    cuuint32_t box[4] = {(cuuint32_t)p->D, 1, (cuuint32_t)p->box_h, 1};
+    int rc = encode(&p->tm_k, k, 4, dims, str, box, "k_pool (e4m3)", CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_DATA_TYPE_UINT8);
+    if (rc) return rc;
+    rc = encode(&p->tm_v, v, 4, dims, str, box, "v_pool (e4m3)", CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_DATA_TYPE_UINT8);
+    if (rc) return rc;
+  } else {
+    // pools [P, ps, Hkv, D]: dims (D, Hkv, ps, P); box (64, 1, box_h, 1).
     cuuint64_t P = p->num_pages > 0 ? (cuuint64_t)p->num_pages : (cuuint64_t)0x7fffffff;
     cuuint64_t dims[4] = {(cuuint64_t)p->D, (cuuint64_t)p->Hkv, (cuuint64_t)p->ps, P};
     cuuint64_t str[3] = {(cuuint64_t)p->D * e, (cuuint64_t)p->Hkv * p->D * e,
@@ -362,6 +389,7 @@ int build_maps(pa_plan* p, const void* q, const void* k, const void* v, void* ou
   p->tm_ptr[2] = v;
   p->tm_ptr[3] = out;
   p->tm_num_pages = p->num_pages;
+  p->tm_fp8 = p->kv_fp8;
   return PA_OK;
 }
 
@@ -448,6 +476,9 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->fused_merge = 0;
   p->split_cnt = nullptr;
   p->tstride = p->C;
+  p->kv_fp8 = 0;
+  p->k_scale = p->v_scale = 1.0f;
+  p->tm_fp8 = 0;
   p->tm_num_pages = -1;
   if (alloc_workspace(p) != PA_OK) {
     delete p;
@@ -544,6 +575,10 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     set_err("pa_run: current device %d is not the plan's device %d", dev, p->device);
     return PA_ERR_INVALID;
   }
+  if (p->kv_fp8 && cu_q_lens != nullptr) {
+    set_err("pa_run: E4M3 pools are read by the decode kernel only (cu_q_lens must be NULL)");
+    return PA_ERR_UNSUPPORTED;
+  }
   int rc = build_maps(p, q, k_pool, v_pool, out);
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -572,8 +607,10 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.forced_splits = p->num_splits > 1 ? p->num_splits : 0;
   // decode-only runs (one query token per request) with up to 32 query heads
   // per KV head go to the keys-as-M decode kernel (one CTA per SM)
+  // (E4M3 pools always take it: pa_set_kv_fp8 checked head_dim)
   const bool dec = cu_q_lens == nullptr && p->G <= 32 &&
-                   ((p->use_dec == -1 && p->D == 128) || (p->use_dec == 1 && p->D >= 128));
+                   (p->kv_fp8 || (p->use_dec == -1 && p->D == 128) ||
+                    (p->use_dec == 1 && p->D >= 128));
   sp.n_ctas = dec ? p->n_sm : attn_grid(p->D, p->n_sm);
   pa::pa_schedule_kernel<<<1, pa::kCostBuckets, 0, st>>>(sp);
 
@@ -598,7 +635,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.o_tma = p->o_tma;
   ap.split_cnt = p->split_cnt;
   ap.fused_merge = fused ? 1 : 0;
-  ap.scale_log2 = p->scale * 1.4426950408889634f;
+  ap.scale_log2 = p->scale * 1.4426950408889634f * (p->kv_fp8 ? p->k_scale : 1.0f);
+  ap.v_scale = p->kv_fp8 ? p->v_scale : 1.0f;
   const bool prof = p->prof_on && p->prof_n < p->prof_cap;
   if (prof) cudaEventRecord(p->prof_ev[2 * p->prof_n], st);
   cudaError_t le = cudaSuccess;
@@ -611,7 +649,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
                     : launch_pairs<128>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, p->tm_o, ap2);
   }
   if (le == cudaSuccess)
-    le = dec ? launch_decode(p->D, p->G, p->n_sm, st, p->tm_k, p->tm_v, ap)
+    le = dec ? launch_decode(p->D, p->G, p->kv_fp8 != 0, p->n_sm, st, p->tm_k, p->tm_v, ap)
              : launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, p->tm_o, ap);
   if (prof) {
     cudaEventRecord(p->prof_ev[2 * p->prof_n + 1], st);
@@ -708,6 +746,28 @@ int pa_set_page_table_stride(pa_plan* p, int row_stride) {
     return PA_ERR_INVALID;
   }
   p->tstride = row_stride;
+  return PA_OK;
+}
+
+int pa_set_kv_fp8(pa_plan* p, int on, float k_scale, float v_scale) {
+  if (!p) { set_err("pa_set_kv_fp8: NULL plan"); return PA_ERR_INVALID; }
+  if (!on) {
+    p->kv_fp8 = 0;
+    p->k_scale = p->v_scale = 1.0f;
+    return PA_OK;
+  }
+  if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale)) {
+    set_err("pa_set_kv_fp8: descales must be finite and > 0 (k_scale=%g v_scale=%g)",
+            (double)k_scale, (double)v_scale);
+    return PA_ERR_INVALID;
+  }
+  if (p->D != 128 && p->D != 256) {
+    set_err("pa_set_kv_fp8: head_dim %d has no E4M3 decode kernel (128 and 256 only)", p->D);
+    return PA_ERR_UNSUPPORTED;
+  }
+  p->kv_fp8 = 1;
+  p->k_scale = k_scale;
+  p->v_scale = v_scale;
   return PA_OK;
 }
 

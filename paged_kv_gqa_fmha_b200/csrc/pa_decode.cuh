@@ -22,13 +22,22 @@
 //              one issuing warp per SM does not keep HBM busy with page-sized boxes
 //   warp  5    MMA issuer (warp-collective issue)
 //   warp  6    Q loader (Q tiles of NR rows, double-buffered where room allows)
+//
+// E4M3 pools (F8): the producers' TMA boxes land in a ring of fp8 staging
+// tiles; four more warps (8-11) widen each tile to fp16 in the swizzled layout
+// the MMA reads (every E4M3 value is exact in fp16) and zero the rows past the
+// request's end in V tiles.  The products then run as fp16 MMAs: Q is rounded
+// to fp16 by the Q loader and P is written as fp16.  The K descale multiplies
+// the softmax scale and the V descale the epilogue's 1 / l, so the pools are
+// never dequantised in memory ("[Attention] FA4 integration", vLLM #32974:
+// the fp8 KV-cache variant with descale factors and bf16 output).
 #pragma once
 
 #include "pa_kernels.cuh"
 
 namespace pa {
 
-template <int D, int NR>
+template <int D, int NR, bool F8 = false>
 struct DecCfg {
   static_assert(D == 128 || D == 256, "decode kernel: head_dim 128 or 256");
   static_assert(NR == 16 || NR == 32, "decode kernel: 16 or 32 padded rows");
@@ -36,8 +45,11 @@ struct DecCfg {
   static constexpr int DCH = D / 64;                  // 128-byte column chunks of a K/V row
   static constexpr int DH = D / 128;                  // M = 128 halves of O^T
   static constexpr int SLOT_CHUNK = BN * 128;         // one 64-column chunk of a K/V tile
-  static constexpr int SLOT_BYTES = BN * D * 2;
-  static constexpr int NSLOT = (D == 128) ? 6 : 3;
+  static constexpr int SLOT_BYTES = BN * D * 2;       // 16-bit K/V tile the MMA reads
+  // 16-bit slots; with E4M3 pools fewer of them plus NST fp8 staging tiles
+  static constexpr int NSLOT = !F8 ? ((D == 128) ? 6 : 3) : ((D == 128) ? (NR == 16 ? 4 : 3) : 2);
+  static constexpr int NST = !F8 ? 0 : ((D == 128) ? (NR == 16 ? 5 : 6) : 2);
+  static constexpr int STAGE_BYTES = BN * D;          // one fp8 tile, rows of D bytes
   static constexpr int Q_CHUNK = NR * 128;            // Q tile: NR rows x 64 columns per chunk
   static constexpr int Q_BYTES = NR * D * 2;
   static constexpr int QBUF = (D == 256 && NR == 32) ? 1 : 2;   // Q tiles in flight
@@ -48,28 +60,32 @@ struct DecCfg {
   static constexpr int O_COL = 2 * NR;                // + half * NR
   static constexpr int TMEM_USED = O_COL + DH * NR;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : (TMEM_USED <= 64 ? 64 : 128);
-  static constexpr int THREADS = 256;
+  static constexpr int THREADS = F8 ? 384 : 256;
   static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5, Q_WARP = 6, PRODUCER2_WARP = 7;
+  static constexpr int CONV_WARP0 = 8;                // E4M3 widening warps 8-11
   // barriers: q_full[2], q_empty[2], kv_full[NSLOT], kv_empty[NSLOT], s_full[2],
-  //           p_full[2], pv_done[2], o_empty, drain, red[2] (row maxima), red_sum
+  //           p_full[2], pv_done[2], o_empty, drain, red[2] (row maxima), red_sum,
+  //           st_full[NST], st_empty[NST] (fp8 staging)
   static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NSLOT,
                        B_SFULL = 4 + 2 * NSLOT, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
                        B_OEMPTY = B_PVDONE + 2, B_DRAIN = B_OEMPTY + 1, B_RED = B_DRAIN + 1,
-                       B_REDSUM = B_RED + 2, NBAR = B_REDSUM + 1;
-  static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = 1024 + NSLOT * SLOT_BYTES + QBUF * Q_BYTES + 2 * P_BYTES +
-                                    RED_BYTES + BAR_BYTES;
+                       B_REDSUM = B_RED + 2, B_STFULL = B_REDSUM + 1, B_STEMPTY = B_STFULL + NST,
+                       NBAR = B_STEMPTY + NST;
+  static constexpr int BAR_BYTES = F8 ? 512 : 256;
+  static constexpr int SMEM_BYTES = 1024 + NSLOT * SLOT_BYTES + NST * STAGE_BYTES +
+                                    QBUF * Q_BYTES + 2 * P_BYTES + RED_BYTES + BAR_BYTES;
   static_assert(NBAR * 8 + 16 <= BAR_BYTES, "barrier area");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(TMEM_USED <= TMEM_COLS, "TMEM columns");
 };
 
 // Q loader: the NR-row Q tile of each item (rows past G * n_tok are left as
-// they are; they only feed columns of S^T and O^T that are never read).
-template <int D, int NR>
+// they are; they only feed columns of S^T and O^T that are never read).  For
+// E4M3 pools the tile is rounded to fp16 (the MMA's A and B share one type).
+template <int D, int NR, bool F8>
 __device__ __forceinline__ void dec_q_loader(const AttnParams& p, uint32_t sQ, uint32_t bar0,
                                              int n_items, volatile int* abort) {
-  using C = DecCfg<D, NR>;
+  using C = DecCfg<D, NR, F8>;
   const int lane = threadIdx.x & 31;
   const int G = p.G;
   uint32_t q_cnt = 0;
@@ -101,6 +117,12 @@ __device__ __forceinline__ void dec_q_loader(const AttnParams& p, uint32_t sQ, u
           const int r = u / (D / 8), c16 = u % (D / 8);
           const uint32_t dst =
               base + (c16 >> 3) * C::Q_CHUNK + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+          if constexpr (F8) {
+            v[k].x = bf16x2_to_f16x2_sat(v[k].x);
+            v[k].y = bf16x2_to_f16x2_sat(v[k].y);
+            v[k].z = bf16x2_to_f16x2_sat(v[k].z);
+            v[k].w = bf16x2_to_f16x2_sat(v[k].w);
+          }
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[k].x),
                        "r"(v[k].y), "r"(v[k].z), "r"(v[k].w)
                        : "memory");
@@ -121,11 +143,19 @@ __device__ __forceinline__ void dec_q_loader(const AttnParams& p, uint32_t sQ, u
 // needs are loaded three tiles ahead (pf0..pf2 hold tiles j..j+2 when K_j is
 // reached), and the first three tiles of the next item are loaded during the
 // current item's last K, so no table read is waited on in the loop.
-template <int D, int NR>
+// With E4M3 pools the boxes (one per page part, D bytes wide) go to the fp8
+// staging ring at `sKV` instead of the 16-bit slots.
+template <int D, int NR, bool F8>
 __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                              const AttnParams& p, uint32_t sKV, uint32_t bar0,
                                              int n_items, uint32_t which, volatile int* abort) {
-  using C = DecCfg<D, NR>;
+  using C = DecCfg<D, NR, F8>;
+  constexpr int RING = F8 ? C::NST : C::NSLOT;
+  constexpr int B_FULL = F8 ? C::B_STFULL : C::B_KVFULL;
+  constexpr int B_EMPTY = F8 ? C::B_STEMPTY : C::B_KVEMPTY;
+  constexpr int RING_BYTES = F8 ? C::STAGE_BYTES : C::SLOT_BYTES;
+  constexpr int ROW_BYTES = F8 ? D : 128;     // bytes of one box row
+  constexpr int NCH = F8 ? 1 : C::DCH;        // boxes per page part
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
@@ -166,9 +196,8 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
         page = (j == n - 1) ? pid_v_next : pid_v;
       }
       const bool mine = (ld_idx & 1u) == which;
-      const uint32_t slot = ld_idx % C::NSLOT;
-      if (mine &&
-          !warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
+      const uint32_t slot = ld_idx % RING;
+      if (mine && !warp_wait(bar0 + 8 * (B_EMPTY + slot), ((ld_idx / RING) & 1) ^ 1, abort)) {
         ok = false;
         break;
       }
@@ -177,8 +206,8 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
       // included) so that no stale shared memory meets the products
       const int live = min(w.kv_len - n0, C::BN);
       const int nbox = ceil_div(live, p.box_h);
-      const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
-      if (mine && lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
+      const uint32_t full = bar0 + 8 * (B_FULL + slot);
+      if (mine && lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * ROW_BYTES * NCH);
       __syncwarp();
       if (mine && lane < nbox) {
         const int row = (n0 + lane * p.box_h) % p.ps;
@@ -187,8 +216,8 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
           page = -1;   // out of the tensor map: the box reads as zeros
         }
         const CUtensorMap* tm = is_v ? tm_v : tm_k;
-        const uint32_t dst = sKV + slot * C::SLOT_BYTES + lane * p.box_h * 128;
-        for (int c = 0; c < C::DCH; ++c)
+        const uint32_t dst = sKV + slot * RING_BYTES + lane * p.box_h * ROW_BYTES;
+        for (int c = 0; c < NCH; ++c)
           tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, row, page);
       }
       if (!is_v && j == n - 1) {
@@ -206,9 +235,85 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
   if (!ok || *abort) {
     // wait (bounded) for this producer's copies still in flight
     if (lane == 0) {
-      const uint32_t first = ld_idx > (uint32_t)C::NSLOT ? ld_idx - C::NSLOT : 0;
+      const uint32_t first = ld_idx > (uint32_t)RING ? ld_idx - RING : 0;
       for (uint32_t k = first; k < ld_idx; ++k)
-        if ((k & 1u) == which) mbar_drain(bar0 + 8 * (C::B_KVFULL + k % C::NSLOT), (k / C::NSLOT) & 1);
+        if ((k & 1u) == which) mbar_drain(bar0 + 8 * (B_FULL + k % RING), (k / RING) & 1);
+    }
+  }
+}
+
+// E4M3 widening (warps 8-11, 128 threads).  Walks the producers' load order;
+// for load i: wait for staging tile i % NST (TMA bytes landed) and for 16-bit
+// slot i % NSLOT (the MMA released it), widen the 128 x D codes to fp16 in the
+// slot's swizzled layout, then release both.  Thread u takes 16-byte unit u of
+// the staging tile (a warp reads 512 contiguous bytes) and writes its 16
+// halves as two 16-byte units of row `row`, 64-column chunk k / 4; unit x of a
+// row sits at x ^ (row & 7), so the stores of a warp spread over all banks.
+// Rows of a V tile at and past the request's end are written as zeros (P is 0
+// there, but 0 * NaN is not).
+template <int D, int NR>
+__device__ __forceinline__ void dec_convert(const AttnParams& p, uint32_t sKV, uint32_t sST,
+                                            uint32_t bar0, int n_items, volatile int* abort) {
+  using C = DecCfg<D, NR, true>;
+  constexpr int UPR = D / 16;                        // 16-byte fp8 units per row
+  constexpr int UNITS = C::BN * UPR;
+  const int ct = threadIdx.x - 32 * C::CONV_WARP0;   // 0..127
+  const int lane = threadIdx.x & 31;
+  uint32_t ld_idx = 0;
+  bool ok = true;
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+  while (ok && items.next(w)) {
+    const int n = item_tiles(w, C::BN);
+    for (int s = 0; s < 2 * n; ++s) {
+      int j;
+      bool is_v;
+      kv_sequence(s, n, j, is_v);
+      const uint32_t st = ld_idx % C::NST, slot = ld_idx % C::NSLOT;
+      if (!warp_wait(bar0 + 8 * (C::B_STFULL + st), (ld_idx / C::NST) & 1, abort) ||
+          !warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
+        ok = false;
+        break;
+      }
+      const int n0 = w.kv_lo + j * C::BN;
+      const int zero_from = is_v ? max(0, min(C::BN, w.kv_len - n0)) : C::BN;
+      const uint32_t src0 = sST + st * C::STAGE_BYTES;
+      const uint32_t dst0 = sKV + slot * C::SLOT_BYTES;
+#pragma unroll 4
+      for (int u = ct; u < UNITS; u += 128) {
+        const int row = u / UPR, k = u % UPR;
+        uint32_t h[8];
+        if (row < zero_from) {
+          uint32_t x0, x1, x2, x3;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                       : "r"(src0 + u * 16));
+          e4m3x4_to_f16x4(x0, h[0], h[1]);
+          e4m3x4_to_f16x4(x1, h[2], h[3]);
+          e4m3x4_to_f16x4(x2, h[4], h[5]);
+          e4m3x4_to_f16x4(x3, h[6], h[7]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) h[i] = 0u;
+        }
+        const uint32_t rbase = dst0 + (k >> 2) * C::SLOT_CHUNK + row * 128;
+        const uint32_t x0 = 2 * (k & 3);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         rbase + ((x0 ^ (row & 7)) << 4)),
+                     "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         rbase + (((x0 + 1) ^ (row & 7)) << 4)),
+                     "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar0 + 8 * (C::B_KVFULL + slot));
+        mbar_arrive(bar0 + 8 * (C::B_STEMPTY + st));
+      }
+      ++ld_idx;
     }
   }
 }
@@ -216,13 +321,16 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
 // MMA issuer (all 32 lanes; one elected lane issues).  Per item of n tiles:
 //   S^T(0) | S^T(1) O^T+=V(0)^T P^T(0) | S^T(2) O^T+=V(1)^T P^T(1) | ...
 // g counts tiles over all items: S^T(g) and P^T(g) use buffer g & 1.
-template <int D, int NR>
+template <int D, int NR, bool F8>
 __device__ __forceinline__ void dec_mma(const AttnParams& p, uint32_t sQ, uint32_t sKV,
                                         uint32_t sP, uint32_t bar0, uint32_t tmem, int n_items,
                                         volatile int* abort) {
-  using C = DecCfg<D, NR>;
-  constexpr uint32_t kIdescS = idesc_bf16_f32(128, NR, false, false);
-  constexpr uint32_t kIdescO = idesc_bf16_f32(128, NR, true, false);
+  using C = DecCfg<D, NR, F8>;
+  // bf16 operands, or fp16 ones (widened E4M3 K/V, Q and P rounded to fp16)
+  constexpr uint32_t kIdescS =
+      F8 ? idesc_f16_f32(128, NR, false, false) : idesc_bf16_f32(128, NR, false, false);
+  constexpr uint32_t kIdescO =
+      F8 ? idesc_f16_f32(128, NR, true, false) : idesc_bf16_f32(128, NR, true, false);
   uint32_t ld_idx = 0, g = 0, q_cnt = 0;
   bool ok = true;
   ItemStream items(p.items, n_items, p.tpb);
@@ -359,11 +467,11 @@ __device__ __forceinline__ bool block_reduce_rows(float (&v)[RR], float* red, ui
 // of every row (identical in all threads) and its own share of the row sums.
 // A decode item is one query token: its G rows see the same keys [kv_lo, kv_hi).
 // Rows G .. RR-1 (padding) are held at -inf, so their P is 0.
-template <int D, int NR, int RR>
+template <int D, int NR, int RR, bool F8>
 __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, uint32_t sP,
                                             float* red, uint32_t bar0, uint32_t tmem,
                                             int n_items, volatile int* abort) {
-  using C = DecCfg<D, NR>;
+  using C = DecCfg<D, NR, F8>;
   constexpr int BN = C::BN;
   const int t = threadIdx.x;
   const int warp = t >> 5, lane = t & 31;
@@ -462,10 +570,11 @@ __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, u
         const float pr = ex2_approx(fmaf(s[r], p.scale_log2, -m_use));
         l_part[r] = fmaf(l_part[r], alpha[r], pr);
         asm volatile("st.shared.u16 [%0], %1;" ::"r"(pb + r * 128 + ((p_unit ^ (r & 7)) << 4)),
-                     "h"(bf16_bits(pr))
+                     "h"(F8 ? f16_bits(pr) : bf16_bits(pr))
                      : "memory");
       }
-      if (j == n - 1 && n0 + BN > w.kv_len) {
+      // (with E4M3 pools the widening warps zero these rows)
+      if (!F8 && j == n - 1 && n0 + BN > w.kv_len) {
         // rows at and past kv_len of the last V tile: tail slots or rows never
         // loaded; P is 0 there but 0 * NaN would still poison O
         const uint32_t ldv = ld_base + 2 * n - 1;
@@ -509,7 +618,7 @@ __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, u
 #pragma unroll
       for (int r = 0; r < RR; ++r) {
         if (r < G) {
-          const float inv_l = l_part[r] > 0.f ? 1.0f / l_part[r] : 0.f;
+          const float inv_l = l_part[r] > 0.f ? (F8 ? p.v_scale : 1.0f) / l_part[r] : 0.f;
           const float val = __uint_as_float(o[r]) * inv_l;
           if (split) p.part_o[(prow0 + r) * D + d] = val;
           else p.out[(orow0 + r) * D + d] = bf16_bits(val);
@@ -541,20 +650,22 @@ struct DecRows {
   static constexpr int NR = RR < 16 ? 16 : RR;
 };
 
-template <int D, int RR>
-__global__ void __launch_bounds__(256, 1)
+template <int D, int RR, bool F8 = false>
+__global__ void __launch_bounds__(DecCfg<D, DecRows<RR>::NR, F8>::THREADS, 1)
     pa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   constexpr int NR = DecRows<RR>::NR;
-  using C = DecCfg<D, NR>;
+  using C = DecCfg<D, NR, F8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t sKV = base;
-  const uint32_t sQ = sKV + C::NSLOT * C::SLOT_BYTES;
+  const uint32_t sST = sKV + C::NSLOT * C::SLOT_BYTES;          // fp8 staging (F8 only)
+  const uint32_t sQ = sST + C::NST * C::STAGE_BYTES;
   const uint32_t sP = sQ + C::QBUF * C::Q_BYTES;
-  const uint32_t off_red = C::NSLOT * C::SLOT_BYTES + C::QBUF * C::Q_BYTES + 2 * C::P_BYTES;
+  const uint32_t off_red = C::NSLOT * C::SLOT_BYTES + C::NST * C::STAGE_BYTES +
+                           C::QBUF * C::Q_BYTES + 2 * C::P_BYTES;
   float* red = reinterpret_cast<float*>(smem + off_red);
   const uint32_t bar0 = base + off_red + C::RED_BYTES;
   uint8_t* bar_ptr = smem + off_red + C::RED_BYTES;
@@ -572,8 +683,13 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(bar0 + 8 * (C::B_RED + i), 4);
     }
     for (int i = 0; i < C::NSLOT; ++i) {
-      mbar_init(bar0 + 8 * (C::B_KVFULL + i), 1);
+      // filled by TMA (one expect_tx arrival) or by the four widening warps
+      mbar_init(bar0 + 8 * (C::B_KVFULL + i), F8 ? 4 : 1);
       mbar_init(bar0 + 8 * (C::B_KVEMPTY + i), 1);
+    }
+    for (int i = 0; i < C::NST; ++i) {
+      mbar_init(bar0 + 8 * (C::B_STFULL + i), 1);
+      mbar_init(bar0 + 8 * (C::B_STEMPTY + i), 4);
     }
     mbar_init(bar0 + 8 * C::B_OEMPTY, 4);
     mbar_init(bar0 + 8 * C::B_DRAIN, 1);
@@ -599,14 +715,16 @@ __global__ void __launch_bounds__(256, 1)
   const int n_items = p.hdr->n_items;
 
   if (warp == C::PRODUCER_WARP || warp == C::PRODUCER2_WARP) {
-    dec_producer<D, NR>(&tm_k, &tm_v, p, sKV, bar0, n_items,
-                        warp == C::PRODUCER_WARP ? 0u : 1u, abort);
+    dec_producer<D, NR, F8>(&tm_k, &tm_v, p, F8 ? sST : sKV, bar0, n_items,
+                            warp == C::PRODUCER_WARP ? 0u : 1u, abort);
   } else if (warp == C::Q_WARP) {
-    dec_q_loader<D, NR>(p, sQ, bar0, n_items, abort);
+    dec_q_loader<D, NR, F8>(p, sQ, bar0, n_items, abort);
   } else if (warp == C::MMA_WARP) {
-    dec_mma<D, NR>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
+    dec_mma<D, NR, F8>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
+  } else if (warp < kSoftmaxWarps) {
+    dec_softmax<D, NR, RR, F8>(p, sKV, sP, red, bar0, tmem, n_items, abort);
   } else {
-    dec_softmax<D, NR, RR>(p, sKV, sP, red, bar0, tmem, n_items, abort);
+    if constexpr (F8) dec_convert<D, NR>(p, sKV, sST, bar0, n_items, abort);
   }
 
   tc_fence_before();

@@ -174,7 +174,8 @@ struct AttnParams {
   int o_tma;                  // 1: full blocks store O through the tensor map of out
   int* split_cnt;             // [B * Hkv] arrivals of split softmax warps (zeroed per run)
   int fused_merge;            // 1: the last split warp of a (request, KV head) merges
-  float scale_log2;
+  float scale_log2;           // softmax scale * log2(e) (times the K descale for E4M3 pools)
+  float v_scale;              // V descale of E4M3 pools (1 for bf16 pools)
 };
 
 constexpr int kSoftmaxWarps = 4;      // softmax warps per CTA in every attention kernel

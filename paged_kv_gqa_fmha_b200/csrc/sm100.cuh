@@ -252,6 +252,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// The same with A and B in fp16 (format code 0 in both fields).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16_f32(M, N, a_mn, b_mn) & ~((1u << 7) | (1u << 10));
+}
+
 // TMEM loads/stores, shape 32x32b: lane i of the warp reads/writes TMEM lane
 // (lane base + i), `N` consecutive 32-bit columns starting at the address's column.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -343,17 +348,43 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Two fp32 -> packed bf16x2, round to nearest even; `lo` goes to the low half.
 // fp32 -> bf16 bits, round to nearest even.
 __device__ __forceinline__ unsigned short bf16_bits(float x) {
   unsigned short h;
   asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(x));
   return h;
 }
+// Two fp32 -> packed bf16x2, round to nearest even; `lo` goes to the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// fp32 -> fp16 bits, round to nearest even.
+__device__ __forceinline__ unsigned short f16_bits(float x) {
+  unsigned short h;
+  asm("cvt.rn.f16.f32 %0, %1;" : "=h"(h) : "f"(x));
+  return h;
+}
+// Two bf16 (packed in one word, element 0 low) -> two fp16 in the same order,
+// round to nearest even, magnitudes past the fp16 range saturated to +-65504.
+// bf16 -> fp32 is a 16-bit shift (exact).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_sat(uint32_t w) {
+  const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Four E4M3 codes (one word, element 0 in the low byte) -> four fp16 in the
+// same order as two words.  Every E4M3 value is exact in fp16 (3 mantissa
+// bits, exponents 2^-9 .. 2^8), so this widening loses nothing.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 }  // namespace pa

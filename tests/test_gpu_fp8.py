@@ -1,0 +1,169 @@
+"""GPU parity of the E4M3 (FP8) KV decode path (pa_set_kv_fp8 + pa_run,
+through the C ABI) with the oracle's attention over fp8 pools.
+
+The pools hold E4M3 codes of N(0,1) * 4 values (torch's round-to-nearest
+quantisation); the descales are arbitrary non-powers of two so that a missing
+or misplaced descale cannot pass.  Rows of each request's last page past its
+KV length hold NaN codes: the kernel must never let them reach O."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from paged_kv_gqa_fmha_b200 import binding, workloads as W
+from tests.gpu_common import compare
+
+pytestmark = pytest.mark.gpu
+
+K_SCALE, V_SCALE = 0.22, 0.31
+NAN_CODE = 0x7F
+
+
+def _codes(shape, gen, dev):
+    x = torch.randn(shape, generator=gen, device=dev, dtype=torch.float32) * 4
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def _poison_tails(k8, v8, w):
+    """NaN codes in the rows past kv_len of every request's last page."""
+    table = w["page_table_cpu"].numpy()
+    ps = w["ps"]
+    for b, kv in enumerate(w["seq_lens_cpu"].tolist()):
+        if kv % ps:
+            page = int(table[b, (kv - 1) // ps])
+            k8[page, kv % ps:] = NAN_CODE
+            v8[page, kv % ps:] = NAN_CODE
+
+
+def _fp8_workload(spec, seed, dev="cuda"):
+    w = W.generate(spec, seed, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 7)
+    k8 = _codes(tuple(w["k_pool"].shape), g, dev)
+    v8 = _codes(tuple(w["v_pool"].shape), g, dev)
+    _poison_tails(k8, v8, w)
+    return w, k8, v8
+
+
+def _plan(w, num_splits=0):
+    plan = binding.Plan(w["B"], w["Hq"], w["Hkv"], w["D"], w["ps"], w["C"], scale=w["scale"],
+                        num_pages=w["P"], num_splits=num_splits)
+    plan.set_kv_fp8(True, K_SCALE, V_SCALE)
+    return plan
+
+
+def _oracle(w, k8, v8):
+    return O.paged_attention_fp8(W.bf16_bits(w["q"]), k8.cpu().numpy(), v8.cpu().numpy(),
+                                 K_SCALE, V_SCALE, w["page_table_cpu"].numpy(),
+                                 w["seq_lens_cpu"].numpy(), w["cu_q_lens_cpu"].numpy(),
+                                 w["scale"])
+
+
+def _run(plan, w, k8, v8):
+    out, lse = plan.run(w["q"], k8, v8, w["page_table"], w["seq_lens"], None)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    return out, lse
+
+
+GEOMS = [  # seed, D, G, ps, Hkv, B, max_kv
+    (1, 128, 4, 16, 2, 5, 700),
+    (2, 128, 8, 32, 1, 3, 1000),
+    (3, 128, 16, 64, 2, 4, 600),
+    (4, 128, 32, 16, 1, 3, 500),
+    (5, 128, 1, 128, 2, 4, 900),
+    (6, 256, 4, 16, 2, 3, 500),
+    (7, 256, 32, 64, 1, 2, 400),
+    (8, 128, 5, 32, 2, 3, 400),
+]
+
+
+@pytest.mark.parametrize("seed,D,G,ps,Hkv,B,max_kv", GEOMS)
+def test_fp8_decode_matches_oracle(seed, D, G, ps, Hkv, B, max_kv):
+    rng = np.random.default_rng(seed)
+    spec = W.random_small(rng, D=D, ps=ps, G=G, Hkv=Hkv, B=B, max_kv=max_kv, prefill=False)
+    w, k8, v8 = _fp8_workload(spec, 500 + seed)
+    out, lse = _run(_plan(w), w, k8, v8)
+    o_ref, l_ref = _oracle(w, k8, v8)
+    compare(out, lse, o_ref, l_ref)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_fp8_splits_and_tile_edges(fused):
+    """KV lengths on and next to the 128-key tile edges, forced splits, with
+    the separate merge kernel and with the fused merge."""
+    kv = [1, 127, 128, 129, 255, 256, 257, 1000]
+    spec = W.custom_spec("fp8_edges", 16, 2, 128, 32, [1] * len(kv), kv)
+    w, k8, v8 = _fp8_workload(spec, 77)
+    o_ref, l_ref = _oracle(w, k8, v8)
+    for splits in (1, 3):
+        plan = _plan(w, num_splits=splits)
+        plan.set_fused_merge(fused)
+        out, lse = _run(plan, w, k8, v8)
+        compare(out, lse, o_ref, l_ref)
+
+
+def test_fp8_descales_are_applied():
+    """The same codes with other descales: still the oracle's answer (a
+    kernel that ignored either descale could not match both)."""
+    rng = np.random.default_rng(91)
+    spec = W.random_small(rng, D=128, ps=16, G=4, Hkv=2, B=3, max_kv=300, prefill=False)
+    w, k8, v8 = _fp8_workload(spec, 91)
+    plan = _plan(w)
+    for ks, vs in ((K_SCALE, V_SCALE), (0.05, 0.9)):
+        plan.set_kv_fp8(True, ks, vs)
+        out, lse = _run(plan, w, k8, v8)
+        o_ref, l_ref = O.paged_attention_fp8(
+            W.bf16_bits(w["q"]), k8.cpu().numpy(), v8.cpu().numpy(), ks, vs,
+            w["page_table_cpu"].numpy(), w["seq_lens_cpu"].numpy(),
+            w["cu_q_lens_cpu"].numpy(), w["scale"])
+        compare(out, lse, o_ref, l_ref)
+
+
+def test_fp8_rejections():
+    rng = np.random.default_rng(3)
+    spec = W.random_small(rng, D=128, ps=16, G=4, Hkv=2, B=2, max_kv=100, prefill=True)
+    w, k8, v8 = _fp8_workload(spec, 3)
+    plan = _plan(w)
+    with pytest.raises(binding.PAError) as e:
+        plan.run(w["q"], k8, v8, w["page_table"], w["seq_lens"], w["cu_q_lens"])
+    assert e.value.code == binding.PA_ERR_UNSUPPORTED
+    with pytest.raises(binding.PAError) as e:
+        plan.set_kv_fp8(True, 0.0, 1.0)
+    assert e.value.code == binding.PA_ERR_INVALID
+    p64 = binding.Plan(2, 8, 2, 64, 16, 8)
+    with pytest.raises(binding.PAError) as e:
+        p64.set_kv_fp8(True, 1.0, 1.0)
+    assert e.value.code == binding.PA_ERR_UNSUPPORTED
+
+
+def test_fp8_full_size_llama_decode_sampled():
+    """The Llama-3.1-8B decode shape at full size (the timed launch), fp8 pools
+    quantised on the device; eight requests checked against the oracle on a
+    compact copy of their pages."""
+    w = W.generate(W.CONFIGS["llama8b_decode"], W.default_seed("llama8b_decode"), device="cuda")
+    k8 = (w["k_pool"].float() * 4).to(torch.float8_e4m3fn).view(torch.uint8)
+    v8 = (w["v_pool"].float() * 4).to(torch.float8_e4m3fn).view(torch.uint8)
+    del w["k_pool"], w["v_pool"]
+    plan = _plan(w)
+    out, lse = _run(plan, w, k8, v8)
+    rng = np.random.default_rng(5)
+    reqs = sorted(int(b) for b in rng.choice(w["B"], size=8, replace=False))
+    table = w["page_table_cpu"].numpy()
+    seq = w["seq_lens_cpu"].numpy()
+    ps = w["ps"]
+    pages = sorted(set(int(p) for b in reqs for p in table[b, : -(-int(seq[b]) // ps)]))
+    remap = {p: i for i, p in enumerate(pages)}
+    idx = torch.tensor(pages, dtype=torch.long, device="cuda")
+    ks = k8.index_select(0, idx).cpu().numpy()
+    vs = v8.index_select(0, idx).cpu().numpy()
+    t2 = np.full((len(reqs), table.shape[1]), -1, dtype=np.int32)
+    for i, b in enumerate(reqs):
+        n = -(-int(seq[b]) // ps)
+        t2[i, :n] = [remap[int(p)] for p in table[b, :n]]
+    q = W.bf16_bits(w["q"])[reqs]
+    cu = np.arange(len(reqs) + 1, dtype=np.int32)
+    o_ref, l_ref = O.paged_attention_fp8(q, ks, vs, K_SCALE, V_SCALE, t2, seq[reqs], cu,
+                                         w["scale"])
+    sel = torch.tensor(reqs, dtype=torch.long, device="cuda")
+    compare(out.index_select(0, sel), lse.index_select(0, sel), o_ref, l_ref)
