@@ -351,18 +351,18 @@ int build_maps(pa_plan* p, const void* q, const void* k, const void* v, void* ou
       if (rc) return rc;
     }
   }
-  // E4M3 pools [P, ps, Hkv, D] bytes: dims (D, Hkv, ps, P); box (D, 1, box_h, 1),
-  // no swizzle (the decode kernel widens the rows into its own layout)
+  // E4M3 pools [P, ps, Hkv, D] bytes: dims (D, Hkv, ps, P); box (128, 1, box_h, 1),
+  // 128-byte swizzle (D / 128 boxes per page part)
   if (p->kv_fp8) {
     cuuint64_t P = p->num_pages > 0 ? (cuuint64_t)p->num_pages : (cuuint64_t)0x7fffffff;
     cuuint64_t dims[4] = {(cuuint64_t)p->D, (cuuint64_t)p->Hkv, (cuuint64_t)p->ps, P};
     cuuint64_t str[3] = {(cuuint64_t)p->D, (cuuint64_t)p->Hkv * p->D,
                          (cuuint64_t)p->ps * p->Hkv * p->D};
-    cuuint32_t box[4] = {(cuuint32_t)p->D, 1, (cuuint32_t)p->box_h, 1};
-    int rc = encode(&p->tm_k, k, 4, dims, str, box, "k_pool (e4m3)", CU_TENSOR_MAP_SWIZZLE_NONE,
+    cuuint32_t box[4] = {128, 1, (cuuint32_t)p->box_h, 1};
+    int rc = encode(&p->tm_k, k, 4, dims, str, box, "k_pool (e4m3)", CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_DATA_TYPE_UINT8);
     if (rc) return rc;
-    rc = encode(&p->tm_v, v, 4, dims, str, box, "v_pool (e4m3)", CU_TENSOR_MAP_SWIZZLE_NONE,
+    rc = encode(&p->tm_v, v, 4, dims, str, box, "v_pool (e4m3)", CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_DATA_TYPE_UINT8);
     if (rc) return rc;
   } else {

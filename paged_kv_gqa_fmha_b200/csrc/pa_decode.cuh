@@ -24,10 +24,14 @@
 //   warp  6    Q loader (Q tiles of NR rows, double-buffered where room allows)
 //
 // E4M3 pools (F8): the producers' TMA boxes land in a ring of fp8 staging
-// tiles; four more warps (8-11) widen each tile to fp16 in the swizzled layout
-// the MMA reads (every E4M3 value is exact in fp16) and zero the rows past the
-// request's end in V tiles.  The products then run as fp16 MMAs: Q is rounded
-// to fp16 by the Q loader and P is written as fp16.  The K descale multiplies
+// tiles (128-byte swizzled rows); four more warps (8-11) widen each tile to
+// fp16 (every E4M3 value is exact in fp16).  A K tile is widened straight into
+// tensor memory, thread t writing key t's row into TMEM lane t, and S^T takes
+// its A operand from there; a V tile is widened into the swizzled shared-memory
+// slot the O^T product reads MN-major, with the rows past the request's end
+// zeroed.  Shared-memory traffic per key is then the fp8 tile written and read
+// once plus one fp16 V row written and read once.  The products run as fp16
+// MMAs: Q is rounded to fp16 by the Q loader and P is written as fp16.  The K descale multiplies
 // the softmax scale and the V descale the epilogue's 1 / l, so the pools are
 // never dequantised in memory ("[Attention] FA4 integration", vLLM #32974:
 // the fp8 KV-cache variant with descale factors and bf16 output).
@@ -46,10 +50,11 @@ struct DecCfg {
   static constexpr int DH = D / 128;                  // M = 128 halves of O^T
   static constexpr int SLOT_CHUNK = BN * 128;         // one 64-column chunk of a K/V tile
   static constexpr int SLOT_BYTES = BN * D * 2;       // 16-bit K/V tile the MMA reads
-  // 16-bit slots; with E4M3 pools fewer of them plus NST fp8 staging tiles
+  // 16-bit K/V slots; with E4M3 pools V slots only, plus NST fp8 staging
+  // tiles (D / 128 chunks of BN rows x 128 bytes, 128-byte swizzle)
   static constexpr int NSLOT = !F8 ? ((D == 128) ? 6 : 3) : ((D == 128) ? (NR == 16 ? 4 : 3) : 2);
   static constexpr int NST = !F8 ? 0 : ((D == 128) ? (NR == 16 ? 5 : 6) : 2);
-  static constexpr int STAGE_BYTES = BN * D;          // one fp8 tile, rows of D bytes
+  static constexpr int STAGE_BYTES = BN * D;
   static constexpr int Q_CHUNK = NR * 128;            // Q tile: NR rows x 64 columns per chunk
   static constexpr int Q_BYTES = NR * D * 2;
   static constexpr int QBUF = (D == 256 && NR == 32) ? 1 : 2;   // Q tiles in flight
@@ -58,20 +63,26 @@ struct DecCfg {
   static constexpr int RED_BYTES = 3 * 4 * NR * 4;    // row maxima of 4 warps (two tiles), row sums
   static constexpr int S_COL = 0;                     // + buffer * NR
   static constexpr int O_COL = 2 * NR;                // + half * NR
-  static constexpr int TMEM_USED = O_COL + DH * NR;
-  static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : (TMEM_USED <= 64 ? 64 : 128);
+  // widened K tiles (F8): NKB buffers of D / 2 columns (fp16 pairs), A of S^T
+  static constexpr int NKB = (D == 128) ? 4 : 2;
+  static constexpr int K_COL = D;
+  static constexpr int TMEM_USED = F8 ? K_COL + NKB * D / 2 : O_COL + DH * NR;
+  static constexpr int TMEM_COLS =
+      TMEM_USED <= 32 ? 32 : (TMEM_USED <= 64 ? 64 : (TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512)));
   static constexpr int THREADS = F8 ? 384 : 256;
   static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5, Q_WARP = 6, PRODUCER2_WARP = 7;
   static constexpr int CONV_WARP0 = 8;                // E4M3 widening warps 8-11
   // barriers: q_full[2], q_empty[2], kv_full[NSLOT], kv_empty[NSLOT], s_full[2],
   //           p_full[2], pv_done[2], o_empty, drain, red[2] (row maxima), red_sum,
-  //           st_full[NST], st_empty[NST] (fp8 staging)
+  //           st_full[NST], st_empty[NST] (fp8 staging), k_full[NKB], k_empty[NKB]
+  //           (widened K in TMEM); with F8 kv_full / kv_empty guard the V slots
   static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NSLOT,
                        B_SFULL = 4 + 2 * NSLOT, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
                        B_OEMPTY = B_PVDONE + 2, B_DRAIN = B_OEMPTY + 1, B_RED = B_DRAIN + 1,
                        B_REDSUM = B_RED + 2, B_STFULL = B_REDSUM + 1, B_STEMPTY = B_STFULL + NST,
-                       NBAR = B_STEMPTY + NST;
-  static constexpr int BAR_BYTES = F8 ? 512 : 256;
+                       B_KFULL = B_STEMPTY + NST, B_KEMPTY = B_KFULL + NKB,
+                       NBAR = B_KFULL + (F8 ? 2 * NKB : 0);
+  static constexpr int BAR_BYTES = F8 ? 384 : 256;
   static constexpr int SMEM_BYTES = 1024 + NSLOT * SLOT_BYTES + NST * STAGE_BYTES +
                                     QBUF * Q_BYTES + 2 * P_BYTES + RED_BYTES + BAR_BYTES;
   static_assert(NBAR * 8 + 16 <= BAR_BYTES, "barrier area");
@@ -143,8 +154,8 @@ __device__ __forceinline__ void dec_q_loader(const AttnParams& p, uint32_t sQ, u
 // needs are loaded three tiles ahead (pf0..pf2 hold tiles j..j+2 when K_j is
 // reached), and the first three tiles of the next item are loaded during the
 // current item's last K, so no table read is waited on in the loop.
-// With E4M3 pools the boxes (one per page part, D bytes wide) go to the fp8
-// staging ring at `sKV` instead of the 16-bit slots.
+// With E4M3 pools the boxes (128-byte column chunks) go to the fp8 staging
+// ring at `sKV` instead of the 16-bit slots.
 template <int D, int NR, bool F8>
 __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                              const AttnParams& p, uint32_t sKV, uint32_t bar0,
@@ -154,8 +165,8 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
   constexpr int B_FULL = F8 ? C::B_STFULL : C::B_KVFULL;
   constexpr int B_EMPTY = F8 ? C::B_STEMPTY : C::B_KVEMPTY;
   constexpr int RING_BYTES = F8 ? C::STAGE_BYTES : C::SLOT_BYTES;
-  constexpr int ROW_BYTES = F8 ? D : 128;     // bytes of one box row
-  constexpr int NCH = F8 ? 1 : C::DCH;        // boxes per page part
+  constexpr int NCH = F8 ? D / 128 : C::DCH;  // boxes (128-byte column chunks) per page part
+  constexpr int CH_ELEMS = F8 ? 128 : 64;     // elements of one chunk
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
@@ -207,7 +218,7 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
       const int live = min(w.kv_len - n0, C::BN);
       const int nbox = ceil_div(live, p.box_h);
       const uint32_t full = bar0 + 8 * (B_FULL + slot);
-      if (mine && lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * ROW_BYTES * NCH);
+      if (mine && lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * NCH);
       __syncwarp();
       if (mine && lane < nbox) {
         const int row = (n0 + lane * p.box_h) % p.ps;
@@ -216,9 +227,9 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
           page = -1;   // out of the tensor map: the box reads as zeros
         }
         const CUtensorMap* tm = is_v ? tm_v : tm_k;
-        const uint32_t dst = sKV + slot * RING_BYTES + lane * p.box_h * ROW_BYTES;
+        const uint32_t dst = sKV + slot * RING_BYTES + lane * p.box_h * 128;
         for (int c = 0; c < NCH; ++c)
-          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, row, page);
+          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * CH_ELEMS, w.kvh, row, page);
       }
       if (!is_v && j == n - 1) {
         WorkItem nw;
@@ -243,23 +254,30 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
 }
 
 // E4M3 widening (warps 8-11, 128 threads).  Walks the producers' load order;
-// for load i: wait for staging tile i % NST (TMA bytes landed) and for 16-bit
-// slot i % NSLOT (the MMA released it), widen the 128 x D codes to fp16 in the
-// slot's swizzled layout, then release both.  Thread u takes 16-byte unit u of
-// the staging tile (a warp reads 512 contiguous bytes) and writes its 16
-// halves as two 16-byte units of row `row`, 64-column chunk k / 4; unit x of a
-// row sits at x ^ (row & 7), so the stores of a warp spread over all banks.
-// Rows of a V tile at and past the request's end are written as zeros (P is 0
-// there, but 0 * NaN is not).
+// staging tile i % NST holds load i as D / 128 chunks of 128 rows x 128 bytes,
+// 16-byte unit x of row r stored at x ^ (r & 7) (the TMA 128-byte swizzle).
+//   K tile of tile g: thread t widens key t's row and stores it to TMEM lane
+//     t, columns K_COL + (g % NKB) * D / 2 onwards (fp16 pairs, element 2c in the
+//     low half of column c); reading unit x of rows t..t+7 hits 8 distinct
+//     bank groups thanks to the swizzle.
+//   V tile of tile g: 16-bit slot g % NSLOT, thread u taking unit u (a warp
+//     reads 512 contiguous bytes) and writing its 16 halves as two 16-byte
+//     units of the slot's swizzled row; units k < 4 and k >= 4 of a row store
+//     their even / odd unit first, so every 8-lane phase of a store covers all
+//     8 bank groups.  Rows at and past the request's end are written as zeros
+//     (P is 0 there, but 0 * NaN is not).
 template <int D, int NR>
 __device__ __forceinline__ void dec_convert(const AttnParams& p, uint32_t sKV, uint32_t sST,
-                                            uint32_t bar0, int n_items, volatile int* abort) {
+                                            uint32_t bar0, uint32_t tmem, int n_items,
+                                            volatile int* abort) {
   using C = DecCfg<D, NR, true>;
   constexpr int UPR = D / 16;                        // 16-byte fp8 units per row
   constexpr int UNITS = C::BN * UPR;
   const int ct = threadIdx.x - 32 * C::CONV_WARP0;   // 0..127
   const int lane = threadIdx.x & 31;
-  uint32_t ld_idx = 0;
+  // this warp's TMEM lanes (warp 8 + i owns lanes 32 i .. 32 i + 31)
+  const uint32_t tl = tmem + (static_cast<uint32_t>((ct >> 5) * 32) << 16);
+  uint32_t ld_idx = 0, g = 0;
   bool ok = true;
   ItemStream items(p.items, n_items, p.tpb);
   WorkItem w;
@@ -269,68 +287,124 @@ __device__ __forceinline__ void dec_convert(const AttnParams& p, uint32_t sKV, u
       int j;
       bool is_v;
       kv_sequence(s, n, j, is_v);
-      const uint32_t st = ld_idx % C::NST, slot = ld_idx % C::NSLOT;
-      if (!warp_wait(bar0 + 8 * (C::B_STFULL + st), (ld_idx / C::NST) & 1, abort) ||
-          !warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
+      const uint32_t st = ld_idx % C::NST, tile = g + j;
+      if (!warp_wait(bar0 + 8 * (C::B_STFULL + st), (ld_idx / C::NST) & 1, abort)) {
         ok = false;
         break;
       }
-      const int n0 = w.kv_lo + j * C::BN;
-      const int zero_from = is_v ? max(0, min(C::BN, w.kv_len - n0)) : C::BN;
       const uint32_t src0 = sST + st * C::STAGE_BYTES;
-      const uint32_t dst0 = sKV + slot * C::SLOT_BYTES;
-#pragma unroll 4
-      for (int u = ct; u < UNITS; u += 128) {
-        const int row = u / UPR, k = u % UPR;
-        uint32_t h[8];
-        if (row < zero_from) {
-          uint32_t x0, x1, x2, x3;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
-                       : "r"(src0 + u * 16));
-          e4m3x4_to_f16x4(x0, h[0], h[1]);
-          e4m3x4_to_f16x4(x1, h[2], h[3]);
-          e4m3x4_to_f16x4(x2, h[4], h[5]);
-          e4m3x4_to_f16x4(x3, h[6], h[7]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) h[i] = 0u;
+      if (!is_v) {
+        const uint32_t kb = tile % C::NKB;
+        if (!warp_wait(bar0 + 8 * (C::B_KEMPTY + kb), ((tile / C::NKB) & 1) ^ 1, abort)) {
+          ok = false;
+          break;
         }
-        const uint32_t rbase = dst0 + (k >> 2) * C::SLOT_CHUNK + row * 128;
-        const uint32_t x0 = 2 * (k & 3);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         rbase + ((x0 ^ (row & 7)) << 4)),
-                     "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         rbase + (((x0 + 1) ^ (row & 7)) << 4)),
-                     "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
-                     : "memory");
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar0 + 8 * (C::B_KVFULL + slot));
-        mbar_arrive(bar0 + 8 * (C::B_STEMPTY + st));
+        tc_fence_after();
+        const uint32_t row_src = src0 + ct * 128;
+        const uint32_t col0 = tl + C::K_COL + kb * (D / 2);
+        // all of the row's loads first (8 units per pass), then widen and store
+#pragma unroll
+        for (int k0 = 0; k0 < UPR; k0 += 8) {
+          uint32_t x[8][4];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int k = k0 + e;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(x[e][0]), "=r"(x[e][1]), "=r"(x[e][2]), "=r"(x[e][3])
+                         : "r"(row_src + (k >> 3) * C::SLOT_CHUNK + (((k & 7) ^ (ct & 7)) << 4)));
+          }
+#pragma unroll
+          for (int e2 = 0; e2 < 8; e2 += 2) {
+            uint32_t h[16];
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                e4m3x4_to_f16x4(x[e2 + e][q], h[8 * e + 2 * q], h[8 * e + 2 * q + 1]);
+            tmem_st16(col0 + (k0 + e2) * 8, h);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar0 + 8 * (C::B_KFULL + kb));
+          mbar_arrive(bar0 + 8 * (C::B_STEMPTY + st));
+        }
+      } else {
+        const uint32_t slot = tile % C::NSLOT;
+        if (!warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((tile / C::NSLOT) & 1) ^ 1, abort)) {
+          ok = false;
+          break;
+        }
+        const int n0 = w.kv_lo + j * C::BN;
+        const int zero_from = max(0, min(C::BN, w.kv_len - n0));
+        const uint32_t dst0 = sKV + slot * C::SLOT_BYTES;
+        // 8 units per pass: every load of the pass before any store
+#pragma unroll
+        for (int u0 = 0; u0 < UNITS; u0 += 8 * 128) {
+          uint32_t x[8][4];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int u = u0 + e * 128 + ct;
+            const int row = u / UPR, k = u % UPR;
+            if (row < zero_from) {
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(x[e][0]), "=r"(x[e][1]), "=r"(x[e][2]), "=r"(x[e][3])
+                           : "r"(src0 + (k >> 3) * C::SLOT_CHUNK + row * 128 +
+                                 (((k & 7) ^ (row & 7)) << 4)));
+            } else {
+              x[e][0] = x[e][1] = x[e][2] = x[e][3] = 0u;   // E4M3 code 0 is +0
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int u = u0 + e * 128 + ct;
+            const int row = u / UPR, k = u % UPR;
+            uint32_t h[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) e4m3x4_to_f16x4(x[e][q], h[2 * q], h[2 * q + 1]);
+            const uint32_t rbase = dst0 + (k >> 2) * C::SLOT_CHUNK + row * 128;
+            const uint32_t odd = (k >> 2) & 1;        // store the odd unit first
+            const uint32_t xa = 2 * (k & 3) + odd, xb = 2 * (k & 3) + (odd ^ 1);
+            // unit 2(k & 3) holds halves 0-7, unit 2(k & 3) + 1 halves 8-15
+            const uint32_t e0 = odd ? h[4] : h[0], e1 = odd ? h[5] : h[1],
+                           e2 = odd ? h[6] : h[2], e3 = odd ? h[7] : h[3];
+            const uint32_t f0 = odd ? h[0] : h[4], f1 = odd ? h[1] : h[5],
+                           f2 = odd ? h[2] : h[6], f3 = odd ? h[3] : h[7];
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             rbase + ((xa ^ (row & 7)) << 4)),
+                         "r"(e0), "r"(e1), "r"(e2), "r"(e3)
+                         : "memory");
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             rbase + ((xb ^ (row & 7)) << 4)),
+                         "r"(f0), "r"(f1), "r"(f2), "r"(f3)
+                         : "memory");
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar0 + 8 * (C::B_KVFULL + slot));
+          mbar_arrive(bar0 + 8 * (C::B_STEMPTY + st));
+        }
       }
       ++ld_idx;
     }
+    g += n;
   }
 }
 
 // MMA issuer (all 32 lanes; one elected lane issues).  Per item of n tiles:
 //   S^T(0) | S^T(1) O^T+=V(0)^T P^T(0) | S^T(2) O^T+=V(1)^T P^T(1) | ...
 // g counts tiles over all items: S^T(g) and P^T(g) use buffer g & 1.
-template <int D, int NR, bool F8>
+template <int D, int NR>
 __device__ __forceinline__ void dec_mma(const AttnParams& p, uint32_t sQ, uint32_t sKV,
                                         uint32_t sP, uint32_t bar0, uint32_t tmem, int n_items,
                                         volatile int* abort) {
-  using C = DecCfg<D, NR, F8>;
-  // bf16 operands, or fp16 ones (widened E4M3 K/V, Q and P rounded to fp16)
-  constexpr uint32_t kIdescS =
-      F8 ? idesc_f16_f32(128, NR, false, false) : idesc_bf16_f32(128, NR, false, false);
-  constexpr uint32_t kIdescO =
-      F8 ? idesc_f16_f32(128, NR, true, false) : idesc_bf16_f32(128, NR, true, false);
+  using C = DecCfg<D, NR>;
+  constexpr uint32_t kIdescS = idesc_bf16_f32(128, NR, false, false);
+  constexpr uint32_t kIdescO = idesc_bf16_f32(128, NR, true, false);
   uint32_t ld_idx = 0, g = 0, q_cnt = 0;
   bool ok = true;
   ItemStream items(p.items, n_items, p.tpb);
@@ -402,6 +476,85 @@ __device__ __forceinline__ void dec_mma(const AttnParams& p, uint32_t sQ, uint32
     }
     g += n;
     ld_idx += 2 * n;
+    ++q_cnt;
+  }
+  tc_commit_w(bar0 + 8 * C::B_DRAIN);
+  if ((threadIdx.x & 31) == 0) mbar_drain(bar0 + 8 * C::B_DRAIN, 0);
+  __syncwarp();
+}
+
+// MMA issuer for E4M3 pools: the same order as dec_mma, with S^T's A operand
+// (the widened K tile of tile g) read from TMEM buffer g % NKB and the V tile of
+// tile g from 16-bit slot g % NSLOT; fp16 operands.
+template <int D, int NR>
+__device__ __forceinline__ void dec_mma_f8(const AttnParams& p, uint32_t sQ, uint32_t sKV,
+                                           uint32_t sP, uint32_t bar0, uint32_t tmem,
+                                           int n_items, volatile int* abort) {
+  using C = DecCfg<D, NR, true>;
+  constexpr uint32_t kIdescS = idesc_f16_f32(128, NR, false, false);
+  constexpr uint32_t kIdescO = idesc_f16_f32(128, NR, true, false);
+  uint32_t g = 0, q_cnt = 0;
+  bool ok = true;
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+
+  // S^T(gs) = K Q^T: A = widened K in TMEM (128 lanes = keys, 8 columns per
+  // 16 of D), B = Q tile (K-major, NR rows)
+  auto issue_s = [&](uint32_t gs, uint32_t sQb) -> bool {
+    const uint32_t kb = gs % C::NKB, sb = gs & 1;
+    if (!warp_wait(bar0 + 8 * (C::B_KFULL + kb), (gs / C::NKB) & 1, abort)) return false;
+    tc_fence_after();
+    const uint32_t a0 = tmem + C::K_COL + kb * (D / 2);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t bd = smem_desc_sw128(sQb + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024);
+      mma_ts_w(tmem + C::S_COL + sb * NR, a0 + kk * 8, bd, kIdescS, kk > 0 ? 1u : 0u);
+    }
+    tc_commit_w(bar0 + 8 * (C::B_SFULL + sb));
+    tc_commit_w(bar0 + 8 * (C::B_KEMPTY + kb));
+    return true;
+  };
+  // O^T += V^T P^T(gp): A = V tile read MN-major, B = P^T (K-major)
+  auto issue_o = [&](uint32_t gp, bool first) -> bool {
+    const uint32_t slot = gp % C::NSLOT;
+    if (!warp_wait(bar0 + 8 * (C::B_KVFULL + slot), (gp / C::NSLOT) & 1, abort)) return false;
+    if (!warp_wait(bar0 + 8 * (C::B_PFULL + (gp & 1)), (gp >> 1) & 1, abort)) return false;
+    if (first && !warp_wait(bar0 + 8 * C::B_OEMPTY, (q_cnt & 1) ^ 1, abort)) return false;
+    tc_fence_after();
+    const uint32_t slot_addr = sKV + slot * C::SLOT_BYTES;
+    const uint32_t pb = sP + (gp & 1) * C::P_BYTES;
+#pragma unroll
+    for (int kk = 0; kk < C::BN / 16; ++kk) {
+      const uint64_t bd = smem_desc_sw128(pb + (kk >> 2) * C::P_CHUNK + (kk & 3) * 32, 16, 1024);
+#pragma unroll
+      for (int hh = 0; hh < C::DH; ++hh) {
+        const uint64_t ad = smem_desc_sw128(slot_addr + 2 * hh * C::SLOT_CHUNK + kk * 16 * 128,
+                                            C::SLOT_CHUNK, 1024);
+        mma_ss_w(tmem + C::O_COL + hh * NR, ad, bd, kIdescO, (!first || kk > 0) ? 1u : 0u);
+      }
+    }
+    tc_commit_w(bar0 + 8 * (C::B_PVDONE + (gp & 1)));
+    tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + slot));
+    return true;
+  };
+
+  while (ok && items.next(w)) {
+    const int n = item_tiles(w, C::BN);
+    if (n == 0) continue;
+    const uint32_t qb = q_cnt % C::QBUF;
+    const uint32_t sQb = sQ + qb * C::Q_BYTES;
+    if (!warp_wait(bar0 + 8 * (C::B_QFULL + qb), (q_cnt / C::QBUF) & 1, abort)) { ok = false; break; }
+    tc_fence_after();
+    if (!issue_s(g, sQb)) { ok = false; break; }
+    if (n == 1) tc_commit_w(bar0 + 8 * (C::B_QEMPTY + qb));
+    for (int j = 0; j < n && ok; ++j) {
+      if (j + 1 < n) {
+        if (!issue_s(g + j + 1, sQb)) { ok = false; break; }
+        if (j + 2 == n) tc_commit_w(bar0 + 8 * (C::B_QEMPTY + qb));
+      }
+      if (!issue_o(g + j, j == 0)) { ok = false; break; }
+    }
+    g += n;
     ++q_cnt;
   }
   tc_commit_w(bar0 + 8 * C::B_DRAIN);
@@ -691,6 +844,12 @@ __global__ void __launch_bounds__(DecCfg<D, DecRows<RR>::NR, F8>::THREADS, 1)
       mbar_init(bar0 + 8 * (C::B_STFULL + i), 1);
       mbar_init(bar0 + 8 * (C::B_STEMPTY + i), 4);
     }
+    if (F8) {
+      for (int i = 0; i < C::NKB; ++i) {
+        mbar_init(bar0 + 8 * (C::B_KFULL + i), 4);
+        mbar_init(bar0 + 8 * (C::B_KEMPTY + i), 1);
+      }
+    }
     mbar_init(bar0 + 8 * C::B_OEMPTY, 4);
     mbar_init(bar0 + 8 * C::B_DRAIN, 1);
     mbar_init(bar0 + 8 * C::B_REDSUM, 4);
@@ -720,11 +879,12 @@ __global__ void __launch_bounds__(DecCfg<D, DecRows<RR>::NR, F8>::THREADS, 1)
   } else if (warp == C::Q_WARP) {
     dec_q_loader<D, NR, F8>(p, sQ, bar0, n_items, abort);
   } else if (warp == C::MMA_WARP) {
-    dec_mma<D, NR, F8>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
+    if constexpr (F8) dec_mma_f8<D, NR>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
+    else dec_mma<D, NR>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
   } else if (warp < kSoftmaxWarps) {
     dec_softmax<D, NR, RR, F8>(p, sKV, sP, red, bar0, tmem, n_items, abort);
   } else {
-    if constexpr (F8) dec_convert<D, NR>(p, sKV, sST, bar0, n_items, abort);
+    if constexpr (F8) dec_convert<D, NR>(p, sKV, sST, bar0, tmem, n_items, abort);
   }
 
   tc_fence_before();
