@@ -350,7 +350,7 @@ def attention_kernel_name(w, decode_only: bool) -> str:
         rr = 4
         while rr < G:
             rr *= 2
-        return "pa_decode_kernel<128, %d>" % rr
+        return "pa_decode_kernel<128, %d, false>" % rr
     return "pa_attention_kernel<%d>" % w["D"]
 
 
@@ -363,7 +363,12 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip per-config, e2e and CPU legs")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(W.CONFIGS),
                     help="workload of the timed steps (default: the headline decode)")
+    ap.add_argument("--kv-fp8", action="store_true",
+                    help="E4M3 pools (decode workloads; implies --no-extra): the metric "
+                         "then counts one byte per K/V element")
     args = ap.parse_args()
+    if args.kv_fp8:
+        args.no_extra = True
     if args.warmup < 3:
         args.warmup = 3
 
@@ -417,6 +422,16 @@ def main():
     w = W.generate(spec, W.default_seed(args.workload), device="cuda")
     counts = work_counts(w)
     plan = make_plan(w)
+    kernel = attention_kernel_name(w, spec.decode_only)
+    if args.kv_fp8:
+        if not spec.decode_only:
+            raise SystemExit("--kv-fp8: E4M3 pools are read by the decode kernel only")
+        to_fp8_pools(w)
+        plan.set_kv_fp8(True, FP8_DESCALE, FP8_DESCALE)
+        counts["bytes"] -= counts["kv_bytes"] // 2
+        counts["kv_bytes"] //= 2
+        kernel = "pa_decode_kernel<%d, %d, true>" % (
+            w["D"], max(4, 1 << (w["Hq"] // w["Hkv"] - 1).bit_length()))
     clocks = ClockSampler(local)
     clocks.start()
     ms, attn_ms, per_run, status = time_headline(w, plan, args.steps, args.warmup, dist_on)
@@ -428,18 +443,20 @@ def main():
 
     achieved = counts["bytes"] / (attn_ms * 1e-3) / 1e9
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    traffic = ncu_traffic(args.workload)
+    traffic = ncu_traffic(args.workload + ("_fp8" if args.kv_fp8 else ""))
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": config_desc(w),
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 KV, bf16 q/out, fp16 MMAs" if args.kv_fp8 else "bf16",
+        "data": "synthetic",
+        "config": {"workload": config_desc(w) + (", E4M3 pools" if args.kv_fp8 else ""),
                    "l2": "inputs larger than L2 (%.2f GB of KV), no flush" % (counts["kv_bytes"] / 1e9),
                    "value_counts": "K+V bytes of every visible key per KV head",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": attention_kernel_name(w, spec.decode_only),
+                     "kernel": kernel,
                      "algorithmic_bytes_per_launch": counts["bytes"],
                      "kernel_ms": attn_ms, "peak_source": "%s hbm_gbs" % peak_kind},
         "gpu_launches": per_run * args.steps,
@@ -494,6 +511,25 @@ def per_config(peaks):
     return res
 
 
+FP8_DESCALE = 0.25
+
+
+def to_fp8_pools(w):
+    """Replace the workload's bf16 pools by E4M3 codes of 4x their values
+    (round to nearest on the device, in chunks that bound the fp32 temporaries);
+    read back with descales FP8_DESCALE the values are the bf16 ones rounded to
+    E4M3."""
+    for key in ("k_pool", "v_pool"):
+        src = w[key]
+        dst = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+        for a in range(0, src.shape[0], 4096):
+            dst[a:a + 4096] = (src[a:a + 4096].float() * 4).to(torch.float8_e4m3fn).view(
+                torch.uint8)
+        w[key] = dst
+        del src
+    torch.cuda.empty_cache()
+
+
 def kv_fp8_decode_rates(bw):
     """Decode over E4M3 pools (pa_set_kv_fp8) on the decode workloads: the
     bf16 pools are quantised on the device (x4, round to nearest E4M3) and
@@ -504,17 +540,10 @@ def kv_fp8_decode_rates(bw):
     for name in ("llama8b_decode", "long_gqa32_decode"):
         w = W.generate(W.CONFIGS[name], W.default_seed(name), device="cuda")
         c = work_counts(w)
-        k8 = torch.empty(w["k_pool"].shape, dtype=torch.uint8, device="cuda")
-        v8 = torch.empty_like(k8)
-        for src, dst in ((w["k_pool"], k8), (w["v_pool"], v8)):
-            for a in range(0, src.shape[0], 4096):     # chunks bound the fp32 temporaries
-                dst[a:a + 4096] = (src[a:a + 4096].float() * 4).to(
-                    torch.float8_e4m3fn).view(torch.uint8)
-        del w["k_pool"], w["v_pool"]
-        torch.cuda.empty_cache()
+        to_fp8_pools(w)
         plan = make_plan(w)
-        plan.set_kv_fp8(True, 0.25, 0.25)
-        args = (w["q"], k8, v8, w["page_table"], w["seq_lens"], None)
+        plan.set_kv_fp8(True, FP8_DESCALE, FP8_DESCALE)
+        args = (w["q"], w["k_pool"], w["v_pool"], w["page_table"], w["seq_lens"], None)
         for _ in range(5):
             plan.run(*args)
         torch.cuda.synchronize()
@@ -530,7 +559,7 @@ def kv_fp8_decode_rates(bw):
                      "kernel": "pa_decode_kernel<%d, %d, true>" % (
                          w["D"], max(4, 1 << (w["Hq"] // w["Hkv"] - 1).bit_length()))}
         plan.close()
-        del w, k8, v8
+        del w
         torch.cuda.empty_cache()
     return out
 
