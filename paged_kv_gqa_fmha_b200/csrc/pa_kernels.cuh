@@ -724,20 +724,12 @@ __device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const Att
   }
 }
 
-// Page id of this lane's box in tile j of item w (0 for lanes without a box).
-__device__ __forceinline__ int tile_page_id(const AttnParams& p, const WorkItem& w, int j, int BN,
-                                            int lane) {
-  const int n0 = w.kv_lo + j * BN;
-  const int live = min(w.kv_len - n0, BN);
-  if (lane * p.box_h >= live) return 0;
-  const int col = (n0 + lane * p.box_h) / p.ps;
-  return __ldg(p.page_table + (size_t)w.b * p.tstride + col);
-}
-
 // KV producer warp: K and V tiles in the MMA's consumption order into the slot
 // ring.  One TMA box is one page (or the part of a page inside the tile) of
-// one KV head; lane k issues box k.  The page ids of tile j+1 are fetched
-// right after tile j's K is issued, so the table read is off the critical path.
+// one KV head; lane k issues box k.  Both producers walk the order; this one
+// issues the loads whose index has parity `which` and skips the others.  Each
+// lane reads its page id from the table right before its box (a loop-carried
+// look-ahead of the ids made every producer wait on every load's table read).
 template <int D>
 __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const AttnParams& p, uint32_t sKV, uint32_t bar0,
@@ -746,34 +738,17 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
-  int pid_next = 0;
-  bool have_next = false;
   ItemStream items(p.items, n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = item_tiles(w, C::BN);
-    if (n == 0) {
-      have_next = false;
-      continue;
-    }
-    // Page ids are loop-carried so that no load result is used in the
-    // iteration that issues it: pid_k holds tile j's ids when K_j is issued
-    // (loaded one K-step earlier), pid_v holds tile j-1's for V_{j-1}, and
-    // pid_v_next keeps tile j's for V_j.  Tile 0 was fetched during the
-    // previous item when possible.
-    int pid_k = have_next ? pid_next : tile_page_id(p, w, 0, C::BN, lane);
-    int pid_v = 0, pid_v_next = 0;
-    have_next = false;
-    for (int s = 0; s < 2 * n; ++s) {
+    for (int s = 0; s < 2 * n; ++s, ++ld_idx) {
+      if ((ld_idx & 1u) != which) continue;
       int j;
       bool is_v;
       kv_sequence(s, n, j, is_v);
-      // both producers walk the whole order; this one issues the loads whose
-      // index has parity `which`
-      const bool mine = (ld_idx & 1u) == which;
       const uint32_t slot = ld_idx % C::NSLOT;
-      if (mine &&
-          !warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
+      if (!warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
         ok = false;
         break;
       }
@@ -783,18 +758,11 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
       const int live = min(w.kv_len - n0, C::BN);
       const int nbox = ceil_div(live, p.box_h);
       const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
-      if (mine && lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
+      if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
       __syncwarp();
-      int page;
-      if (!is_v) {
-        pid_v = pid_v_next;
-        pid_v_next = pid_k;
-        page = pid_k;
-      } else {
-        page = (j == n - 1) ? pid_v_next : pid_v;
-      }
-      if (mine && lane < nbox) {
-        const int row = (n0 + lane * p.box_h) % p.ps;
+      if (lane < nbox) {
+        const int r = n0 + lane * p.box_h;     // < kv_len <= C * ps
+        int page = __ldg(p.page_table + (size_t)w.b * p.tstride + r / p.ps);
         if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
           atomicOr(p.status, kStatusBadPage);
           page = -1;   // out of the tensor map: the box reads as zeros
@@ -802,20 +770,8 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
         const CUtensorMap* tm = is_v ? tm_v : tm_k;
         const uint32_t dst = sKV + slot * C::SLOT_BYTES + lane * p.box_h * 128;
         for (int c = 0; c < C::DCH; ++c)
-          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, row, page);
+          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, r % p.ps, page);
       }
-      if (!is_v) {
-        if (j + 1 < n) {
-          pid_k = tile_page_id(p, w, j + 1, C::BN, lane);
-        } else {
-          WorkItem nw;
-          if (items.peek(nw) && item_tiles(nw, C::BN) > 0) {
-            pid_next = tile_page_id(p, nw, 0, C::BN, lane);
-            have_next = true;
-          }
-        }
-      }
-      ++ld_idx;
     }
   }
   if (!ok || *abort) {

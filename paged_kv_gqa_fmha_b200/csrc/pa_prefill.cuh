@@ -168,7 +168,8 @@ __device__ __forceinline__ void pair_q_loader(const CUtensorMap* tm_q, const Att
 
 // K/V producer: the tiles of an item in the MMA's consumption order
 // (kv_sequence: K0 K1 V0 K2 V1 ... V(n-1)); every live row of a tile is
-// loaded.  Page ids are loop-carried exactly as in the one-stage producer.
+// loaded.  Each lane reads its page id right before its box, as in the
+// one-stage producer.
 template <int D>
 __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const AttnParams& p, uint32_t sKV, uint32_t bar0,
@@ -177,20 +178,11 @@ __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUt
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
-  int pid_next = 0;
-  bool have_next = false;
   ItemStream items(p.items, n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = pair_shape(w, p.tpb, C::BN, p.causal).n;
-    if (n == 0) {
-      have_next = false;
-      continue;
-    }
-    int pid_k = have_next ? pid_next : tile_page_id(p, w, 0, C::BN, lane);
-    int pid_v = 0, pid_v_next = 0;
-    have_next = false;
-    for (int s = 0; s < 2 * n; ++s) {
+    for (int s = 0; s < 2 * n; ++s, ++ld_idx) {
       int j;
       bool is_v;
       kv_sequence(s, n, j, is_v);
@@ -205,16 +197,9 @@ __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUt
       const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
       if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
       __syncwarp();
-      int page;
-      if (!is_v) {
-        pid_v = pid_v_next;
-        pid_v_next = pid_k;
-        page = pid_k;
-      } else {
-        page = (j == n - 1) ? pid_v_next : pid_v;
-      }
       if (lane < nbox) {
-        const int row = (n0 + lane * p.box_h) % p.ps;
+        const int r = n0 + lane * p.box_h;     // < kv_len <= C * ps
+        int page = __ldg(p.page_table + (size_t)w.b * p.tstride + r / p.ps);
         if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
           atomicOr(p.status, kStatusBadPage);
           page = -1;   // out of the tensor map: the box reads as zeros
@@ -222,20 +207,8 @@ __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUt
         const CUtensorMap* tm = is_v ? tm_v : tm_k;
         const uint32_t dst = sKV + slot * C::SLOT_BYTES + lane * p.box_h * 128;
         for (int c = 0; c < C::DCH; ++c)
-          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, row, page);
+          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, r % p.ps, page);
       }
-      if (!is_v) {
-        if (j + 1 < n) {
-          pid_k = tile_page_id(p, w, j + 1, C::BN, lane);
-        } else {
-          WorkItem nw;
-          if (items.peek(nw) && pair_shape(nw, p.tpb, C::BN, p.causal).n > 0) {
-            pid_next = tile_page_id(p, nw, 0, C::BN, lane);
-            have_next = true;
-          }
-        }
-      }
-      ++ld_idx;
     }
   }
   if (!ok || *abort) {
