@@ -614,7 +614,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.n_ctas = dec ? p->n_sm : attn_grid(p->D, p->n_sm);
   pa::pa_schedule_kernel<<<1, pa::kCostBuckets, 0, st>>>(sp);
 
-  pa::AttnParams ap;
+  pa::AttnParams ap = {};
   ap.q = static_cast<const uint16_t*>(q);
   ap.page_table = page_table;
   ap.cu_q_lens = cu_q_lens;
@@ -630,6 +630,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.S_max = p->S_max;
   ap.tpb = p->tpb;
   ap.box_h = p->box_h;
+  ap.ps_log2 = __builtin_ctz((unsigned)p->ps);
+  ap.box_log2 = __builtin_ctz((unsigned)p->box_h);
   ap.tstride = p->tstride;
   ap.causal = p->causal;
   ap.o_tma = p->o_tma;
@@ -645,6 +647,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     pa::AttnParams ap2 = ap;
     ap2.items = p->items2;
     ap2.box_h = p->box_h2;
+    ap2.box_log2 = __builtin_ctz((unsigned)p->box_h2);
     le = p->D == 64 ? launch_pairs<64>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, p->tm_o, ap2)
                     : launch_pairs<128>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, p->tm_o, ap2);
   }
@@ -1027,7 +1030,7 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   sp.n_ctas = attn_grid(head_dim, nd->n_sm);
   pa::pa_schedule_kernel<<<1, pa::kCostBuckets, 0, st>>>(sp);
 
-  pa::AttnParams ap;
+  pa::AttnParams ap = {};
   ap.q = static_cast<const uint16_t*>(q);
   ap.page_table = page_table;
   ap.cu_q_lens = cu_q_lens;
@@ -1043,6 +1046,9 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   ap.S_max = 1;
   ap.tpb = tpb;
   ap.box_h = box_h;
+  ap.ps_log2 = __builtin_ctz((unsigned)page_size);
+  ap.box_log2 = __builtin_ctz((unsigned)box_h);
+  ap.v_scale = 1.0f;
   ap.tstride = capacity;
   ap.causal = 1;
   ap.split_cnt = nullptr;

@@ -188,13 +188,13 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
       // every live row of the tile is loaded (rows past the item's range
       // included) so that no stale shared memory meets the products
       const int live = min(w.kv_len - n0, C::BN);
-      const int nbox = ceil_div(live, p.box_h);
+      const int nbox = (live + p.box_h - 1) >> p.box_log2;
       const uint32_t full = bar0 + 8 * (B_FULL + slot);
       if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * NCH);
       __syncwarp();
       if (lane < nbox) {
         const int r = n0 + lane * p.box_h;     // < kv_len <= C * ps
-        int page = __ldg(p.page_table + (size_t)w.b * p.tstride + r / p.ps);
+        int page = __ldg(p.page_table + (size_t)w.b * p.tstride + (r >> p.ps_log2));
         if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
           atomicOr(p.status, kStatusBadPage);
           page = -1;   // out of the tensor map: the box reads as zeros
@@ -202,7 +202,7 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
         const CUtensorMap* tm = is_v ? tm_v : tm_k;
         const uint32_t dst = sKV + slot * RING_BYTES + lane * p.box_h * 128;
         for (int c = 0; c < NCH; ++c)
-          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * CH_ELEMS, w.kvh, r % p.ps, page);
+          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * CH_ELEMS, w.kvh, r & (p.ps - 1), page);
       }
     }
   }

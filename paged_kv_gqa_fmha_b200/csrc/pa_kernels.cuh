@@ -169,6 +169,7 @@ struct AttnParams {
   float* part_lse;            // [B*Hkv*S_max*128]
   unsigned* status;
   int B, Hq, Hkv, G, C, ps, num_pages, S_max, tpb, box_h;
+  int ps_log2, box_log2;      // log2 of ps and box_h (both powers of two)
   int tstride;                // page-table row stride (>= C)
   int causal;                 // 1: causal mask aligned to the end of KV; 0: all keys
   int o_tma;                  // 1: full blocks store O through the tensor map of out
@@ -756,13 +757,13 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
       // every live row of the tile is loaded (rows past the item's causal limit
       // included) so that no stale shared memory meets P * V
       const int live = min(w.kv_len - n0, C::BN);
-      const int nbox = ceil_div(live, p.box_h);
+      const int nbox = (live + p.box_h - 1) >> p.box_log2;
       const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
       if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
       __syncwarp();
       if (lane < nbox) {
         const int r = n0 + lane * p.box_h;     // < kv_len <= C * ps
-        int page = __ldg(p.page_table + (size_t)w.b * p.tstride + r / p.ps);
+        int page = __ldg(p.page_table + (size_t)w.b * p.tstride + (r >> p.ps_log2));
         if (page < 0 || (p.num_pages > 0 && page >= p.num_pages)) {
           atomicOr(p.status, kStatusBadPage);
           page = -1;   // out of the tensor map: the box reads as zeros
@@ -770,7 +771,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
         const CUtensorMap* tm = is_v ? tm_v : tm_k;
         const uint32_t dst = sKV + slot * C::SLOT_BYTES + lane * p.box_h * 128;
         for (int c = 0; c < C::DCH; ++c)
-          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, r % p.ps, page);
+          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, r & (p.ps - 1), page);
       }
     }
   }
