@@ -153,8 +153,10 @@ PA_API int pa_set_scale(pa_plan *plan, float scale);
 PA_API int pa_set_num_pages(pa_plan *plan, int num_pages);
 
 /* KV splits for requests whose packed query rows fit one 128-row tile
- * (decode-like requests): 0 = automatic (default), 1 = never split,
- * n > 1 = split every such request into min(n, its KV tiles) chunks.
+ * (decode-like requests): 0 = automatic (default: chunks sized so that
+ * the whole run is about four work items per CTA, at most
+ * ceil(8 * SMs / (batch * heads_kv)) and 64 chunks per request), 1 = never
+ * split, n > 1 = split every such request into min(n, its KV tiles) chunks.
  * May reallocate the workspace; call it outside graph capture. */
 PA_API int pa_set_num_splits(pa_plan *plan, int num_splits);
 

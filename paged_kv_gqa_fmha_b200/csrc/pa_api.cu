@@ -115,7 +115,7 @@ int attn_grid(int D, int n_sm) {
 
 int auto_smax(int B, int Hkv, int n_sm) {
   const long units = (long)B * Hkv;
-  long s = (4L * n_sm + units - 1) / units;
+  long s = (8L * n_sm + units - 1) / units;
   if (s > pa::kMaxSplits) s = pa::kMaxSplits;
   if (s < 1) s = 1;
   return (int)s;

@@ -201,27 +201,42 @@ __device__ __forceinline__ void merge_one_row(const float* part_o, const float* 
   const float L = (m == -INFINITY) ? -INFINITY : m + logf(e);
   const float w0 = (L == -INFINITY || l0 == -INFINITY) ? 0.f : expf(l0 - L);
   const float w1 = (L == -INFINITY || l1 == -INFINITY) ? 0.f : expf(l1 - L);
-  for (int d0 = 0; d0 < D; d0 += 128) {            // warp-uniform loop
-    const int d = d0 + lane * 4;
-    const bool act = d < D;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
-    for (int s = 0; s < ns; ++s) {
-      const float wgt = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
-      if (act) {
-        const float4 o = __ldcg(reinterpret_cast<const float4*>(part_o + (base + (size_t)s * kBM) * D + d));
-        a0 = fmaf(wgt, o.x, a0);
-        a1 = fmaf(wgt, o.y, a1);
-        a2 = fmaf(wgt, o.z, a2);
-        a3 = fmaf(wgt, o.w, a3);
-      }
+  // lane owns columns 4 lane .. 4 lane + 3 of each 128-wide chunk (D <= 256:
+  // at most two chunks); both chunks of a split are loaded in the same pass,
+  // eight splits per unrolled step, so up to 16 loads per lane are in flight
+  const int d_a = lane * 4, d_b = 128 + lane * 4;
+  const bool act_a = d_a < D, act_b = d_b < D;
+  float4 acc_a = make_float4(0.f, 0.f, 0.f, 0.f), acc_b = acc_a;
+#pragma unroll 8
+  for (int s = 0; s < ns; ++s) {
+    const float wgt = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
+    const float* row = part_o + (base + (size_t)s * kBM) * D;
+    if (act_a) {
+      const float4 o = __ldcg(reinterpret_cast<const float4*>(row + d_a));
+      acc_a.x = fmaf(wgt, o.x, acc_a.x);
+      acc_a.y = fmaf(wgt, o.y, acc_a.y);
+      acc_a.z = fmaf(wgt, o.z, acc_a.z);
+      acc_a.w = fmaf(wgt, o.w, acc_a.w);
     }
-    if (act) {
-      uint2 pk;
-      pk.x = pack_bf16x2(a0, a1);
-      pk.y = pack_bf16x2(a2, a3);
-      *reinterpret_cast<uint2*>(out_row + d) = pk;
+    if (act_b) {
+      const float4 o = __ldcg(reinterpret_cast<const float4*>(row + d_b));
+      acc_b.x = fmaf(wgt, o.x, acc_b.x);
+      acc_b.y = fmaf(wgt, o.y, acc_b.y);
+      acc_b.z = fmaf(wgt, o.z, acc_b.z);
+      acc_b.w = fmaf(wgt, o.w, acc_b.w);
     }
+  }
+  if (act_a) {
+    uint2 pk;
+    pk.x = pack_bf16x2(acc_a.x, acc_a.y);
+    pk.y = pack_bf16x2(acc_a.z, acc_a.w);
+    *reinterpret_cast<uint2*>(out_row + d_a) = pk;
+  }
+  if (act_b) {
+    uint2 pk;
+    pk.x = pack_bf16x2(acc_b.x, acc_b.y);
+    pk.y = pack_bf16x2(acc_b.z, acc_b.w);
+    *reinterpret_cast<uint2*>(out_row + d_b) = pk;
   }
   if (lane == 0 && lse_out) *lse_out = L;
 }
@@ -454,7 +469,9 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
   }
   __syncthreads();
   if (tid == 0) {
-    const unsigned long long target = (unsigned long long)p.n_ctas * 2ull;
+    // about four items per CTA: with the longest-first order that balances
+    // uneven requests without making the split merge too long
+    const unsigned long long target = (unsigned long long)p.n_ctas * 4ull;
     const unsigned long long c = (total_tiles + target - 1) / target;
     s_chunk = (int)(c < 4 ? 4 : (c > (1ull << 30) ? (1ull << 30) : c));
     if (s_flags) atomicOr(&p.hdr->status, s_flags);
@@ -1194,10 +1211,13 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(MergeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n_req = p.hdr->n_split_reqs;
   const int warp = threadIdx.x >> 5;
-  const int n_units = n_req * p.Hkv * kBM;
+  // row-major over (request, KV head): unit u is row u / n_kh of block u % n_kh,
+  // so the live rows (r < q_len * G) come first and spread over all warps
+  const int n_kh = n_req * p.Hkv;
+  const int n_units = n_kh * kBM;
   for (int u = blockIdx.x * 4 + warp; u < n_units; u += gridDim.x * 4) {
-    const int r = u % kBM;
-    const int kh = u / kBM;
+    const int r = u / n_kh;
+    const int kh = u % n_kh;
     const int kvh = kh % p.Hkv;
     const int b = p.split_list[kh / p.Hkv];
     const int4 ri = p.req_info[b];
