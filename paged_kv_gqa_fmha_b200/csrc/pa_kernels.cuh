@@ -818,14 +818,14 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
     if (n == 0) continue;
     const uint32_t qb = q_cnt % C::QBUF;
     const uint32_t sQb = sQ + qb * C::Q_BYTES;
-    if (!mbar_wait(bar0 + 8 * (C::B_QFULL + qb), (q_cnt / C::QBUF) & 1, abort)) { ok = false; break; }
+    if (!warp_wait(bar0 + 8 * (C::B_QFULL + qb), (q_cnt / C::QBUF) & 1, abort)) { ok = false; break; }
     tc_fence_after();
     for (int s = 0; s < 2 * n; ++s) {
       int j;
       bool is_v;
       kv_sequence(s, n, j, is_v);
       const uint32_t slot = ld_idx % C::NSLOT;
-      if (!mbar_wait(bar0 + 8 * (C::B_KVFULL + slot), (ld_idx / C::NSLOT) & 1, abort)) {
+      if (!warp_wait(bar0 + 8 * (C::B_KVFULL + slot), (ld_idx / C::NSLOT) & 1, abort)) {
         ok = false;
         break;
       }
@@ -839,14 +839,14 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
           const uint64_t ad = smem_desc_sw128(sQb + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024);
           const uint64_t bd =
               smem_desc_sw128(slot_addr + (kk >> 2) * C::SLOT_CHUNK + (kk & 3) * 32, 16, 1024);
-          mma_ss(tmem + sb * C::BN, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss_w(tmem + sb * C::BN, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar0 + 8 * (C::B_SFULL + sb));
-        tc_commit(bar0 + 8 * (C::B_KVEMPTY + slot));
-        if (j == n - 1) tc_commit(bar0 + 8 * (C::B_QEMPTY + qb));
+        tc_commit_w(bar0 + 8 * (C::B_SFULL + sb));
+        tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + slot));
+        if (j == n - 1) tc_commit_w(bar0 + 8 * (C::B_QEMPTY + qb));
       } else {
-        if (!mbar_wait(bar0 + 8 * (C::B_PFULL + sb), (g >> 1) & 1, abort)) { ok = false; break; }
-        if (j == 0 && !mbar_wait(bar0 + 8 * C::B_OEMPTY, (q_cnt & 1) ^ 1, abort)) {
+        if (!warp_wait(bar0 + 8 * (C::B_PFULL + sb), (g >> 1) & 1, abort)) { ok = false; break; }
+        if (j == 0 && !warp_wait(bar0 + 8 * C::B_OEMPTY, (q_cnt & 1) ^ 1, abort)) {
           ok = false;
           break;
         }
@@ -856,20 +856,21 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           const uint64_t bd = smem_desc_sw128(slot_addr + kk * 16 * 128, C::SLOT_CHUNK, 1024);
-          mma_ts(tmem + C::O_COL, tmem + sb * C::BN + kk * 8, bd, kIdescPV,
+          mma_ts_w(tmem + C::O_COL, tmem + sb * C::BN + kk * 8, bd, kIdescPV,
                  (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar0 + 8 * (C::B_PVDONE + sb));
-        tc_commit(bar0 + 8 * (C::B_KVEMPTY + slot));
+        tc_commit_w(bar0 + 8 * (C::B_PVDONE + sb));
+        tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + slot));
       }
       ++ld_idx;
     }
     g_base += n;
     ++q_cnt;
   }
-  // all MMAs issued by this thread complete before TMEM is released
-  tc_commit(bar0 + 8 * C::B_DRAIN);
-  mbar_drain(bar0 + 8 * C::B_DRAIN, 0);
+  // all MMAs issued by this warp complete before TMEM is released
+  tc_commit_w(bar0 + 8 * C::B_DRAIN);
+  if ((threadIdx.x & 31) == 0) mbar_drain(bar0 + 8 * C::B_DRAIN, 0);
+  __syncwarp();
 }
 
 template <int D>
@@ -1176,8 +1177,7 @@ __global__ void __maxnreg__(TileCfg<D>::MAXREG)
   } else if (warp == kQWarp) {
     q_loader_role<D>(&tm_q, p, sQ, bar0, n_items, abort);
   } else if (warp == kMmaWarp) {
-    if ((threadIdx.x & 31) == 0) mma_role<D>(p, sQ, sKV, bar0, tmem, n_items, abort);
-    __syncwarp();
+    mma_role<D>(p, sQ, sKV, bar0, tmem, n_items, abort);   // all 32 lanes
   } else {
     softmax_role<D>(&tm_o, p, sKV, sEpi, bar0, tmem, n_items, abort);
   }

@@ -136,6 +136,25 @@ def test_split_long_gqa32_head_dim_256():
             compare(out, lse, *oracle_all(w))
 
 
+@pytest.mark.parametrize("D,decode_kernel", [(128, True), (128, False), (256, False)])
+def test_up_to_64_splits(D, decode_kernel):
+    """One long request on one KV head: the automatic split count reaches its
+    cap of 64 (the merge's second LSE lane, splits 33..64, is in use); the
+    result must match the oracle and the unsplit run."""
+    spec = W.custom_spec("split64", 8, 1, D, 64, [1], [60000])
+    w = gen(spec, 15)
+    plan = make_plan(w)
+    plan.set_decode_kernel(decode_kernel)
+    assert plan.max_splits == 64
+    out, lse, _ = gpu_run(w, plan, use_cu=False)
+    assert plan.status() == 0
+    compare(out, lse, *oracle_all(w))
+    one = make_plan(w, num_splits=1)
+    out1, lse1, _ = gpu_run(w, one, use_cu=False)
+    assert torch.max(torch.abs(out.float() - out1.float())).item() <= 1e-2
+    assert torch.max(torch.abs(lse - lse1)).item() <= 1e-3
+
+
 # ------------------------------------------------------------------ invariants on the GPU path
 def test_page_permutation_invariance_gpu():
     spec = W.custom_spec("perm", 16, 4, 64, 16, [1, 40, 1], [500, 300, 77])
