@@ -54,6 +54,22 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
 
+// What the scheduler writes and the attention and merge kernels of the same
+// run read.  Two sets, used by alternate runs: a run's scheduler may start
+// (as a programmatic dependent) while the previous run's kernels still read
+// the other set; it waits for them before it exits.
+struct SchedBufs {
+  pa::WsHeader* hdr;          // n_items, n_split_reqs, n_items2 (status is in set 0)
+  int4* req_info;
+  int4* req_aux;
+  int* unit_off;
+  int* split_list;
+  pa::PackedItem* items;
+  int* unit_off2;
+  pa::PackedItem* items2;
+  int* split_cnt;             // [B * Hkv] fused-merge counters (plans with splits)
+};
+
 struct pa_plan {
   int B, Hq, Hkv, D, ps, C, G;
   int device, n_sm;
@@ -66,14 +82,9 @@ struct pa_plan {
   // workspace
   void* ws;
   size_t ws_bytes;
-  pa::WsHeader* hdr;
-  int4* req_info;
-  int4* req_aux;
-  int* unit_off;
-  int* split_list;
-  int* unit_off2;
-  pa::PackedItem* items;
-  pa::PackedItem* items2;     // query-block pairs (two-stage prefill kernel)
+  pa::WsHeader* hdr;           // set 0's header: holds the status word of every run
+  SchedBufs sb[2];
+  unsigned run_par;            // set used by the next pa_run
   int max_items2;
   bool use_pairs;             // head_dim <= 128: prefill runs on the two-stage kernel
   int last_launches;          // kernels the last pa_run enqueued
@@ -91,7 +102,6 @@ struct pa_plan {
   int use_dec;                 // decode kernel: -1 head_dim 128 only (default), 1 128 and 256, 0 never
   int causal;                  // 1 (default): causal mask; 0: every row sees all of its keys
   int fused_merge;             // 1: the last split warp merges; 0 (default): merge kernel
-  int* split_cnt;              // [B * Hkv] fused-merge counters (plans with splits)
   int tstride;                 // page-table row stride in int32 entries (default C)
   int o_tma;                   // tm_o is used (G divides 32)
   CUtensorMap tm_k2, tm_v2;   // page boxes of box_h2 rows
@@ -136,25 +146,31 @@ int alloc_workspace(pa_plan* p) {
   const long max_items2 = p->use_pairs ? (long)p->B * p->Hkv * ((blocks_per_req + 1) / 2) : 0;
   const size_t n_part_rows = p->S_max > 1 ? (size_t)p->B * p->Hkv * p->S_max * pa::kBM : 0;
   size_t off = 0;
-  const size_t o_hdr = off; off = align_up(off + sizeof(pa::WsHeader), 256);
-  const size_t o_req = off; off = align_up(off + sizeof(int4) * (size_t)p->B, 256);
-  const size_t o_aux = off; off = align_up(off + sizeof(int4) * (size_t)p->B, 256);
-  const size_t o_uoff = off; off = align_up(off + sizeof(int) * (size_t)(p->B + 1), 256);
-  const size_t o_split = off; off = align_up(off + sizeof(int) * (size_t)p->B, 256);
-  const size_t o_items = off; off = align_up(off + sizeof(pa::PackedItem) * (size_t)max_items, 256);
-  const size_t o_uoff2 = off; off = align_up(off + sizeof(int) * (size_t)(p->B + 1), 256);
-  const size_t o_items2 = off; off = align_up(off + sizeof(pa::PackedItem) * (size_t)max_items2, 256);
+  size_t o_hdr[2], o_req[2], o_aux[2], o_uoff[2], o_split[2], o_items[2], o_uoff2[2],
+      o_items2[2], o_cnt[2];
+  o_hdr[0] = off; off = align_up(off + sizeof(pa::WsHeader), 256);
+  o_hdr[1] = off; off = align_up(off + sizeof(pa::WsHeader), 256);
+  const size_t zero_bytes = off;   // both headers start zeroed
+  for (int k = 0; k < 2; ++k) {
+    o_req[k] = off; off = align_up(off + sizeof(int4) * (size_t)p->B, 256);
+    o_aux[k] = off; off = align_up(off + sizeof(int4) * (size_t)p->B, 256);
+    o_uoff[k] = off; off = align_up(off + sizeof(int) * (size_t)(p->B + 1), 256);
+    o_split[k] = off; off = align_up(off + sizeof(int) * (size_t)p->B, 256);
+    o_items[k] = off; off = align_up(off + sizeof(pa::PackedItem) * (size_t)max_items, 256);
+    o_uoff2[k] = off; off = align_up(off + sizeof(int) * (size_t)(p->B + 1), 256);
+    o_items2[k] = off; off = align_up(off + sizeof(pa::PackedItem) * (size_t)max_items2, 256);
+    o_cnt[k] = off;
+    off = align_up(off + (p->S_max > 1 ? sizeof(int) * (size_t)p->B * p->Hkv : 0), 256);
+  }
   const size_t o_plse = off; off = align_up(off + sizeof(float) * n_part_rows, 256);
   const size_t o_po = off; off = align_up(off + sizeof(float) * n_part_rows * p->D, 256);
-  const size_t o_cnt = off;
-  off = align_up(off + (p->S_max > 1 ? sizeof(int) * (size_t)p->B * p->Hkv : 0), 256);
   void* ws = nullptr;
   cudaError_t e = cudaMalloc(&ws, off);
   if (e != cudaSuccess) {
     set_err("pa: cudaMalloc of %zu workspace bytes failed: %s", off, cudaGetErrorString(e));
     return PA_ERR_CUDA;
   }
-  e = cudaMemset(ws, 0, o_req);
+  e = cudaMemset(ws, 0, zero_bytes);
   if (e != cudaSuccess) {
     cudaFree(ws);
     set_err("pa: cudaMemset failed: %s", cudaGetErrorString(e));
@@ -164,18 +180,23 @@ int alloc_workspace(pa_plan* p) {
   p->ws = ws;
   p->ws_bytes = off;
   char* c = static_cast<char*>(ws);
-  p->hdr = reinterpret_cast<pa::WsHeader*>(c + o_hdr);
-  p->req_info = reinterpret_cast<int4*>(c + o_req);
-  p->req_aux = reinterpret_cast<int4*>(c + o_aux);
-  p->unit_off = reinterpret_cast<int*>(c + o_uoff);
-  p->split_list = reinterpret_cast<int*>(c + o_split);
-  p->items = reinterpret_cast<pa::PackedItem*>(c + o_items);
-  p->unit_off2 = reinterpret_cast<int*>(c + o_uoff2);
-  p->items2 = reinterpret_cast<pa::PackedItem*>(c + o_items2);
+  for (int k = 0; k < 2; ++k) {
+    SchedBufs& b = p->sb[k];
+    b.hdr = reinterpret_cast<pa::WsHeader*>(c + o_hdr[k]);
+    b.req_info = reinterpret_cast<int4*>(c + o_req[k]);
+    b.req_aux = reinterpret_cast<int4*>(c + o_aux[k]);
+    b.unit_off = reinterpret_cast<int*>(c + o_uoff[k]);
+    b.split_list = reinterpret_cast<int*>(c + o_split[k]);
+    b.items = reinterpret_cast<pa::PackedItem*>(c + o_items[k]);
+    b.unit_off2 = reinterpret_cast<int*>(c + o_uoff2[k]);
+    b.items2 = reinterpret_cast<pa::PackedItem*>(c + o_items2[k]);
+    b.split_cnt = p->S_max > 1 ? reinterpret_cast<int*>(c + o_cnt[k]) : nullptr;
+  }
+  p->hdr = p->sb[0].hdr;
+  p->run_par = 0;
   p->max_items2 = (int)max_items2;
   p->part_lse = reinterpret_cast<float*>(c + o_plse);
   p->part_o = reinterpret_cast<float*>(c + o_po);
-  p->split_cnt = p->S_max > 1 ? reinterpret_cast<int*>(c + o_cnt) : nullptr;
   p->max_items = (int)max_items;
   return PA_OK;
 }
@@ -292,6 +313,25 @@ cudaError_t launch_attention_d(int D, int n_sm, cudaStream_t st, const CUtensorM
     case 128: return launch_attention<128>(n_sm, st, tq, tk, tv, to, ap);
     default: return launch_attention<256>(n_sm, st, tq, tk, tv, to, ap);
   }
+}
+
+// The scheduler is a programmatic dependent of the kernel before it (the
+// previous run's attention or merge kernel): it builds this run's work list in
+// the other set of buffers while that kernel finishes, and waits for it
+// (griddepcontrol.wait) before it exits, so everything launched after the
+// scheduler is ordered after the previous run.
+cudaError_t launch_schedule(cudaStream_t st, const pa::SchedParams& sp) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(pa::kCostBuckets);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pa::pa_schedule_kernel, sp);
 }
 
 cudaError_t launch_merge(int n_sm, cudaStream_t st, const pa::MergeParams& mp) {
@@ -474,7 +514,6 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->use_dec = -1;
   p->causal = 1;
   p->fused_merge = 0;
-  p->split_cnt = nullptr;
   p->tstride = p->C;
   p->kv_fp8 = 0;
   p->k_scale = p->v_scale = 1.0f;
@@ -583,27 +622,30 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
+  // this run's set of scheduler outputs (the previous run may still read the other)
+  const SchedBufs& bufs = p->sb[p->run_par & 1u];
   pa::SchedParams sp;
   sp.seq_lens = seq_lens;
   sp.cu_q_lens = cu_q_lens;
-  sp.items = p->items;
-  sp.req_info = p->req_info;
-  sp.req_aux = p->req_aux;
-  sp.unit_off = p->unit_off;
-  sp.split_list = p->split_list;
+  sp.items = bufs.items;
+  sp.req_info = bufs.req_info;
+  sp.req_aux = bufs.req_aux;
+  sp.unit_off = bufs.unit_off;
+  sp.split_list = bufs.split_list;
   // without cu_q_lens every request is one decode token: no query-block pairs
   const bool pairs = p->use_pairs && cu_q_lens != nullptr;
-  sp.items2 = pairs ? p->items2 : nullptr;
-  sp.unit_off2 = p->unit_off2;
+  sp.items2 = pairs ? bufs.items2 : nullptr;
+  sp.unit_off2 = bufs.unit_off2;
   sp.max_items2 = p->max_items2;
-  sp.hdr = p->hdr;
+  sp.hdr = bufs.hdr;
+  sp.status = &p->hdr->status;
   sp.max_items = p->max_items;
   sp.B = p->B; sp.Hkv = p->Hkv; sp.G = p->G; sp.C = p->C; sp.ps = p->ps; sp.BN = p->BN;
   sp.tpb = p->tpb;
   sp.causal = p->causal;
   sp.S_max = p->num_splits == 1 ? 1 : p->S_max;
   const bool fused = p->fused_merge && sp.S_max > 1;
-  sp.split_cnt = fused ? p->split_cnt : nullptr;
+  sp.split_cnt = fused ? bufs.split_cnt : nullptr;
   sp.forced_splits = p->num_splits > 1 ? p->num_splits : 0;
   // decode-only runs (one query token per request) with up to 32 query heads
   // per KV head go to the keys-as-M decode kernel (one CTA per SM)
@@ -612,7 +654,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
                    (p->kv_fp8 || (p->use_dec == -1 && p->D == 128) ||
                     (p->use_dec == 1 && p->D >= 128));
   sp.n_ctas = dec ? p->n_sm : attn_grid(p->D, p->n_sm);
-  pa::pa_schedule_kernel<<<1, pa::kCostBuckets, 0, st>>>(sp);
+  cudaError_t le = launch_schedule(st, sp);
 
   pa::AttnParams ap = {};
   ap.q = static_cast<const uint16_t*>(q);
@@ -620,8 +662,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.cu_q_lens = cu_q_lens;
   ap.out = static_cast<uint16_t*>(out);
   ap.lse = lse;
-  ap.items = p->items;
-  ap.hdr = p->hdr;
+  ap.items = bufs.items;
+  ap.hdr = bufs.hdr;
   ap.part_o = p->part_o;
   ap.part_lse = p->part_lse;
   ap.status = &p->hdr->status;
@@ -635,17 +677,16 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   ap.tstride = p->tstride;
   ap.causal = p->causal;
   ap.o_tma = p->o_tma;
-  ap.split_cnt = p->split_cnt;
+  ap.split_cnt = bufs.split_cnt;
   ap.fused_merge = fused ? 1 : 0;
   ap.scale_log2 = p->scale * 1.4426950408889634f * (p->kv_fp8 ? p->k_scale : 1.0f);
   ap.v_scale = p->kv_fp8 ? p->v_scale : 1.0f;
   const bool prof = p->prof_on && p->prof_n < p->prof_cap;
   if (prof) cudaEventRecord(p->prof_ev[2 * p->prof_n], st);
-  cudaError_t le = cudaSuccess;
-  if (pairs) {
+  if (le == cudaSuccess && pairs) {
     // query-block pairs (prefill) first, on the two-stage kernel
     pa::AttnParams ap2 = ap;
-    ap2.items = p->items2;
+    ap2.items = bufs.items2;
     ap2.box_h = p->box_h2;
     ap2.box_log2 = __builtin_ctz((unsigned)p->box_h2);
     le = p->D == 64 ? launch_pairs<64>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, p->tm_o, ap2)
@@ -660,9 +701,9 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   }
   if (le == cudaSuccess && sp.S_max > 1 && !fused) {
     pa::MergeParams mp;
-    mp.req_info = p->req_info;
-    mp.split_list = p->split_list;
-    mp.hdr = p->hdr;
+    mp.req_info = bufs.req_info;
+    mp.split_list = bufs.split_list;
+    mp.hdr = bufs.hdr;
     mp.part_o = p->part_o;
     mp.part_lse = p->part_lse;
     mp.out = static_cast<uint16_t*>(out);
@@ -675,6 +716,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     return PA_ERR_CUDA;
   }
   p->last_launches = 2 + (pairs ? 1 : 0) + (sp.S_max > 1 && !fused ? 1 : 0);
+  p->run_par ^= 1u;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_err("pa_run: launch failed: %s", cudaGetErrorString(e));
@@ -1020,6 +1062,7 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   sp.req_aux = reinterpret_cast<int4*>(base + o_aux);
   sp.unit_off = reinterpret_cast<int*>(base + o_uoff);
   sp.hdr = hdr;
+  sp.status = &hdr->status;
   sp.max_items = (int)max_items;
   sp.B = batch; sp.Hkv = heads_kv; sp.G = G; sp.C = capacity; sp.ps = page_size; sp.BN = BN;
   sp.tpb = tpb;

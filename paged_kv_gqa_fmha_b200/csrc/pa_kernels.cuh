@@ -311,7 +311,8 @@ struct SchedParams {
   int4* req_info;      // [B] {n_splits, q_len, t_base, kv_len}
   int4* req_aux;       // [B] {units, tiles per split, KV tiles of the single block, 0}
   int* unit_off;       // [B + 1] exclusive prefix sum of units
-  WsHeader* hdr;
+  WsHeader* hdr;        // this run's header (n_items, n_split_reqs, n_items2)
+  unsigned* status;     // the plan's status word
   int max_items;
   int B, Hkv, G, C, ps, BN, tpb, S_max, forced_splits, n_ctas;
   int causal;          // 0: every row of a request sees all of its keys
@@ -423,7 +424,7 @@ __device__ __forceinline__ Unit unit_of(const SchedParams& p, const int4& ri, co
 
 // One CTA of 1024 threads.
 //   1. validate every request, count the KV tiles of all work;
-//   2. choose splits (about two waves of CTAs over all work, or the forced
+//   2. choose splits (about four items per CTA over all work, or the forced
 //      count) for requests whose packed rows fit one 128-row tile; count the
 //      units (query blocks or splits) of each request and prefix-sum them;
 //   3. histogram of unit costs, scanned in descending cost order;
@@ -474,7 +475,7 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
     const unsigned long long target = (unsigned long long)p.n_ctas * 4ull;
     const unsigned long long c = (total_tiles + target - 1) / target;
     s_chunk = (int)(c < 4 ? 4 : (c > (1ull << 30) ? (1ull << 30) : c));
-    if (s_flags) atomicOr(&p.hdr->status, s_flags);
+    if (s_flags) atomicOr(p.status, s_flags);
   }
   __syncthreads();
   const int chunk = s_chunk;
@@ -663,6 +664,10 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
       }
     }
   }
+  // this kernel may have started while the previous run's kernels were still
+  // running (it only wrote the other set of buffers); finishing only after
+  // them orders every later kernel after the previous run as well
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // =========================================================================== attention
