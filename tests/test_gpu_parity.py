@@ -155,6 +155,23 @@ def test_up_to_64_splits(D, decode_kernel):
     assert torch.max(torch.abs(lse - lse1)).item() <= 1e-3
 
 
+@pytest.mark.parametrize("G,splits,fused", [(4, 0, False), (8, 3, False), (4, 3, True),
+                                            (32, 0, False)])
+def test_mixed_batch_splits_and_edges(G, splits, fused):
+    """Mixed batch: single-token requests long enough to be split (merge
+    kernel or fused merge), a single key, a tile edge, prefill requests of one
+    and of several query blocks, two tokens over two keys."""
+    q = [1, 200, 1, 1, 37, 1, 130, 1, 2]
+    kv = [3000, 600, 129, 1, 500, 2048, 130, 77, 2]
+    spec = W.custom_spec("mixed_edges", 2 * G, 2, 128, 32, q, kv)
+    w = gen(spec, 17 + G + splits)
+    plan = make_plan(w, num_splits=splits)
+    plan.set_fused_merge(fused)
+    out, lse, _ = gpu_run(w, plan)
+    assert plan.status() == 0
+    compare(out, lse, *oracle_all(w))
+
+
 # ------------------------------------------------------------------ invariants on the GPU path
 def test_page_permutation_invariance_gpu():
     spec = W.custom_spec("perm", 16, 4, 64, 16, [1, 40, 1], [500, 300, 77])
