@@ -125,9 +125,12 @@ PA_API pa_plan *pa_create_plan(int batch, int heads_q, int heads_kv, int head_di
  * the request's KV; decode sees every key).  Query head h reads KV head
  * h / G.  All pointers must be 16-byte aligned.
  *
- * Enqueues at most three kernels (scheduler, attention, split merge); does
- * not allocate, does not synchronise and reads no device data on the host,
- * so it can be captured in a CUDA graph.  Returns PA_OK, PA_ERR_INVALID
+ * Enqueues at most four kernels (scheduler, two-stage prefill when enabled,
+ * attention, split merge); does not allocate, does not synchronise and reads
+ * no device data on the host, so it can be captured in a CUDA graph.  The
+ * scheduler may start while the previous pa_run on the same plan and stream
+ * is still finishing (it writes the other of two work-list buffers) and ends
+ * only after that run, so consecutive runs keep stream order.  Returns PA_OK, PA_ERR_INVALID
  * (NULL or misaligned pointer) or PA_ERR_CUDA (launch failure).  Problems in
  * the device-side request data are recorded in the status word instead.
  */
