@@ -223,12 +223,11 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
 //     t, columns K_COL + (g % NKB) * D / 2 onwards (fp16 pairs, element 2c in the
 //     low half of column c); reading unit x of rows t..t+7 hits 8 distinct
 //     bank groups thanks to the swizzle.
-//   V tile of tile g: 16-bit slot g % NSLOT, thread u taking unit u (a warp
-//     reads 512 contiguous bytes) and writing its 16 halves as two 16-byte
-//     units of the slot's swizzled row; units k < 4 and k >= 4 of a row store
-//     their even / odd unit first, so every 8-lane phase of a store covers all
-//     8 bank groups.  Rows at and past the request's end are written as zeros
-//     (P is 0 there, but 0 * NaN is not).
+//   V tile of tile g: 16-bit slot g % NSLOT; the 8 lanes of a phase take one
+//     16-byte unit of 8 consecutive rows, whose swizzled places (staging and
+//     slot alike) fall in 8 distinct bank groups, and write its 16 halves as
+//     two 16-byte units of the slot's swizzled rows.  Rows at and past the
+//     request's end are written as zeros (P is 0 there, but 0 * NaN is not).
 template <int D, int NR>
 __device__ __forceinline__ void dec_convert(const AttnParams& p, uint32_t sKV, uint32_t sST,
                                             uint32_t bar0, uint32_t tmem, int n_items,
@@ -303,14 +302,18 @@ __device__ __forceinline__ void dec_convert(const AttnParams& p, uint32_t sKV, u
         const int n0 = w.kv_lo + j * C::BN;
         const int zero_from = max(0, min(C::BN, w.kv_len - n0));
         const uint32_t dst0 = sKV + slot * C::SLOT_BYTES;
-        // 8 units per pass: every load of the pass before any store
+        // 8 units per pass: every load of the pass before any store.  Unit u
+        // is row (u & 7) + 8 (u / (8 UPR)), column unit (u / 8) % UPR: the 8
+        // lanes of a phase take 8 consecutive rows at one unit, so both the
+        // swizzled staging loads and the swizzled fp16 stores hit 8 distinct
+        // bank groups
 #pragma unroll
         for (int u0 = 0; u0 < UNITS; u0 += 8 * 128) {
           uint32_t x[8][4];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int u = u0 + e * 128 + ct;
-            const int row = u / UPR, k = u % UPR;
+            const int row = (u & 7) + 8 * (u / (8 * UPR)), k = (u >> 3) % UPR;
             if (row < zero_from) {
               asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                            : "=r"(x[e][0]), "=r"(x[e][1]), "=r"(x[e][2]), "=r"(x[e][3])
@@ -323,25 +326,21 @@ __device__ __forceinline__ void dec_convert(const AttnParams& p, uint32_t sKV, u
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int u = u0 + e * 128 + ct;
-            const int row = u / UPR, k = u % UPR;
+            const int row = (u & 7) + 8 * (u / (8 * UPR)), k = (u >> 3) % UPR;
             uint32_t h[8];
 #pragma unroll
             for (int q = 0; q < 4; ++q) e4m3x4_to_f16x4(x[e][q], h[2 * q], h[2 * q + 1]);
+            // halves 0-7 go to 16-byte unit 2 (k & 3) of the 64-column chunk
+            // k / 4, halves 8-15 to the next unit (x stored at x ^ (row & 7))
             const uint32_t rbase = dst0 + (k >> 2) * C::SLOT_CHUNK + row * 128;
-            const uint32_t odd = (k >> 2) & 1;        // store the odd unit first
-            const uint32_t xa = 2 * (k & 3) + odd, xb = 2 * (k & 3) + (odd ^ 1);
-            // unit 2(k & 3) holds halves 0-7, unit 2(k & 3) + 1 halves 8-15
-            const uint32_t e0 = odd ? h[4] : h[0], e1 = odd ? h[5] : h[1],
-                           e2 = odd ? h[6] : h[2], e3 = odd ? h[7] : h[3];
-            const uint32_t f0 = odd ? h[0] : h[4], f1 = odd ? h[1] : h[5],
-                           f2 = odd ? h[2] : h[6], f3 = odd ? h[3] : h[7];
+            const uint32_t x0 = 2 * (k & 3);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             rbase + ((xa ^ (row & 7)) << 4)),
-                         "r"(e0), "r"(e1), "r"(e2), "r"(e3)
+                             rbase + ((x0 ^ (row & 7)) << 4)),
+                         "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
                          : "memory");
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             rbase + ((xb ^ (row & 7)) << 4)),
-                         "r"(f0), "r"(f1), "r"(f2), "r"(f3)
+                             rbase + (((x0 + 1) ^ (row & 7)) << 4)),
+                         "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
                          : "memory");
           }
         }
