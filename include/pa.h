@@ -227,6 +227,18 @@ PA_API int pa_set_page_table_stride(pa_plan *plan, int row_stride);
  * pa_run; no reallocation.  PA_ERR_INVALID for a NULL plan. */
 PA_API int pa_set_decode_kernel(pa_plan *plan, int on);
 
+/* Self-test of the bounded waits every kernel uses (no plan needed).  Runs
+ * one CTA on the current device in which one warp waits on an mbarrier that
+ * nothing arrives at, with a limit of limit_us microseconds (1 .. 1000000):
+ * it gives up, sets the CTA's abort flag and PA_STATUS_TIMEOUT; a second warp
+ * waiting on another such barrier with the production limit (2 s) must leave
+ * through the abort flag soon after.  Writes the status word to *status_out
+ * and the two waits' durations in microseconds to elapsed_us_out[0..1].
+ * Synchronous (allocates 12 bytes, synchronises the device).  Returns PA_OK,
+ * PA_ERR_INVALID (NULL argument, limit out of range) or PA_ERR_CUDA. */
+PA_API int pa_selftest_wait_timeout(uint32_t limit_us, uint32_t *status_out,
+                                    uint32_t *elapsed_us_out);
+
 /* E4M3 (FP8) KV pools with per-tensor descales ("[Attention] FA4
  * integration", vLLM #32974: the fp8 KV-cache variant with descale factors
  * and bf16 output; the format is OCP FP8 E4M3: bias 7, 3 mantissa bits,

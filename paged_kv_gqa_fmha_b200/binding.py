@@ -28,7 +28,8 @@ EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_sc
            "pa_set_num_pages", "pa_set_num_splits", "pa_get_status", "pa_workspace_bytes",
            "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc",
            "pa_set_two_stage_prefill", "pa_set_decode_kernel", "pa_append_kv",
-           "pa_set_causal", "pa_set_page_table_stride", "pa_set_fused_merge", "pa_set_kv_fp8")
+           "pa_set_causal", "pa_set_page_table_stride", "pa_set_fused_merge", "pa_set_kv_fp8",
+           "pa_selftest_wait_timeout")
 
 # Size of the library's static scratch array used by pa_run_noalloc.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -90,6 +91,9 @@ def load_library(path: str = LIB_PATH):
     lib.pa_set_page_table_stride.restype = I
     lib.pa_set_kv_fp8.argtypes = [P, I, F, F]
     lib.pa_set_kv_fp8.restype = I
+    lib.pa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.POINTER(ctypes.c_uint32),
+                                             ctypes.POINTER(ctypes.c_uint32)]
+    lib.pa_selftest_wait_timeout.restype = I
     lib.pa_run_noalloc.argtypes = [I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P]
     lib.pa_run_noalloc.restype = I
     if path == LIB_PATH:
@@ -302,6 +306,17 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def selftest_wait_timeout(limit_us: int):
+    """Run the bounded-wait self-test (pa_selftest_wait_timeout): returns
+    (status word, microseconds the short-limit wait took, microseconds the
+    production-limit wait took before the abort flag released it)."""
+    lib = load_library()
+    st = ctypes.c_uint32(0)
+    el = (ctypes.c_uint32 * 2)()
+    _check(lib.pa_selftest_wait_timeout(int(limit_us), ctypes.byref(st), el))
+    return int(st.value), int(el[0]), int(el[1])
 
 
 def run_noalloc(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, out, lse, *, heads_kv,

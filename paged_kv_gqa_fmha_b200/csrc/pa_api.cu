@@ -794,6 +794,37 @@ int pa_set_page_table_stride(pa_plan* p, int row_stride) {
   return PA_OK;
 }
 
+int pa_selftest_wait_timeout(uint32_t limit_us, uint32_t* status_out,
+                             uint32_t* elapsed_us_out) {
+  if (!status_out || !elapsed_us_out) {
+    set_err("pa_selftest_wait_timeout: NULL argument");
+    return PA_ERR_INVALID;
+  }
+  if (limit_us < 1 || limit_us > 1000000) {
+    set_err("pa_selftest_wait_timeout: limit_us %u outside [1, 1000000]", limit_us);
+    return PA_ERR_INVALID;
+  }
+  unsigned* d = nullptr;   // [0] status, [1..2] elapsed microseconds of warps 1 and 2
+  cudaError_t e = cudaMalloc(&d, 3 * sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaMemset(d, 0, 3 * sizeof(unsigned));
+  if (e == cudaSuccess) {
+    pa::pa_selftest_wait_kernel<<<1, 96>>>(d, (uint64_t)limit_us * 1000u, d + 1);
+    e = cudaGetLastError();
+  }
+  unsigned h[3] = {0, 0, 0};
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(h, d, sizeof h, cudaMemcpyDeviceToHost);
+  if (d) cudaFree(d);
+  if (e != cudaSuccess) {
+    set_err("pa_selftest_wait_timeout: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  *status_out = h[0];
+  elapsed_us_out[0] = h[1];
+  elapsed_us_out[1] = h[2];
+  return PA_OK;
+}
+
 int pa_set_kv_fp8(pa_plan* p, int on, float k_scale, float v_scale) {
   if (!p) { set_err("pa_set_kv_fp8: NULL plan"); return PA_ERR_INVALID; }
   if (!on) {

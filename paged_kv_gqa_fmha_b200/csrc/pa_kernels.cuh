@@ -1236,4 +1236,37 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(MergeParams p) {
   }
 }
 
+// Self-test of the bounded waits (pa_selftest_wait_timeout).  One CTA of
+// three warps and two mbarriers that nothing ever arrives at.  Warp 1 waits on
+// the first with a short limit, gives up, sets the CTA's abort flag and the
+// timeout status bit; warp 2 waits on the second with the production limit
+// and must leave through the abort shortcut long before that limit.  Both
+// record how long they waited (microseconds of global time).
+__global__ void __launch_bounds__(96) pa_selftest_wait_kernel(unsigned* status, uint64_t limit_ns,
+                                                               unsigned* elapsed_us) {
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars[0]), 1);
+    mbar_init(smem_u32(&bars[1]), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abort = &abort_flag;
+  if (warp == 1 || warp == 2) {
+    const uint64_t t0 = global_timer_ns();
+    const bool ok = __all_sync(0xffffffffu,
+                               mbar_wait_for(smem_u32(&bars[warp - 1]), 0, abort,
+                                             warp == 1 ? limit_ns : kWaitTimeoutNs));
+    const uint64_t dt = global_timer_ns() - t0;
+    if (lane == 0) {
+      elapsed_us[warp - 1] = (unsigned)(dt / 1000u);
+      if (!ok) atomicOr(status, kStatusTimeout);
+    }
+  }
+  __syncthreads();
+}
+
 }  // namespace pa

@@ -373,3 +373,21 @@ def test_page_table_row_stride(decode_only):
     out, lse, _ = gpu_run(w, plan, use_cu=not decode_only, page_table=t3[:, 0, :])
     assert plan.status() == 0
     compare(out, lse, *oracle_all(w))
+
+
+# ------------------------------------------------------------------ bounded waits
+@pytest.mark.parametrize("limit_us", [500, 5000])
+def test_wait_timeout_sets_status_and_releases_other_roles(limit_us):
+    """A wait on an mbarrier that nothing arrives at gives up after its limit
+    and sets PA_STATUS_TIMEOUT; a second wait with the production limit (2 s)
+    leaves through the abort flag right after; the context stays usable."""
+    from paged_kv_gqa_fmha_b200 import binding
+    status, t_short, t_long = binding.selftest_wait_timeout(limit_us)
+    assert status & binding.STATUS_TIMEOUT
+    assert limit_us <= t_short < limit_us + 50000
+    assert t_long < t_short + 50000          # far below the 2 s production limit
+    spec = W.custom_spec("after_timeout", 8, 2, 128, 16, [1, 1], [100, 300])
+    w = gen(spec, 19)
+    out, lse, plan = gpu_run(w, use_cu=False)
+    assert plan.status() == 0
+    compare(out, lse, *oracle_all(w))
