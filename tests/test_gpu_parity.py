@@ -106,6 +106,28 @@ def test_two_stage_prefill_kernel(D, ps, G):
     compare(out, lse, *oracle_all(w))
 
 
+@pytest.mark.parametrize("scale_q", [1.0, 30.0])
+def test_two_stage_long_requests(scale_q):
+    """The two-stage kernel over many 128-key tiles per item (the slot ring
+    wraps many times), a chunked-prefill request whose keys start far before
+    its queries, and (q x 30) a peaked softmax that rescales O in TMEM."""
+    spec = W.custom_spec("pairs_long", 16, 4, 128, 64, [1024, 200, 33], [1024, 1500, 2100])
+    w = gen(spec, 41)
+    if scale_q != 1.0:
+        w["q"] = (w["q"].float() * scale_q).to(torch.bfloat16)
+    plan = make_plan(w)
+    plan.set_two_stage_prefill(True)
+    out, lse, _ = gpu_run(w, plan)
+    assert plan.status() == 0
+    o_ref, l_ref = oracle_all(w)
+    if scale_q == 1.0:
+        compare(out, lse, o_ref, l_ref)
+    else:
+        vmax = float(w["v_pool"].float().abs().max())
+        compare(out, lse, o_ref, l_ref, tol_o=2.0 ** -8 * vmax,
+                tol_l=1e-3 * max(1.0, float(np.max(np.abs(l_ref)))))
+
+
 # ------------------------------------------------------------------ split-KV (a8)
 @pytest.mark.parametrize("splits,fused", [(1, True), (2, True), (7, True), (0, True), (2, False),
                                           (7, False), (0, False)])
@@ -320,11 +342,14 @@ def test_large_logits_gpu():
 
 
 # ------------------------------------------------------------------ full-size configs, sampled rows
-@pytest.mark.parametrize("name", ["llama8b_decode", "llama8b_causal_prefill", "unified_mixed",
-                                  "long_gqa32_decode"])
-def test_full_size_config_sampled_rows(name):
+@pytest.mark.parametrize("name,pairs", [("llama8b_decode", False), ("llama8b_causal_prefill", False),
+                                        ("unified_mixed", False), ("long_gqa32_decode", False),
+                                        ("llama8b_causal_prefill", True), ("unified_mixed", True)])
+def test_full_size_config_sampled_rows(name, pairs):
     w = gen(W.CONFIGS[name], W.default_seed(name))
     plan = make_plan(w)
+    if pairs:
+        plan.set_two_stage_prefill(True)
     out, lse, _ = gpu_run(w, plan, use_cu=not W.CONFIGS[name].decode_only)
     assert plan.status() == 0
     assert torch.isfinite(out.float()).all()
