@@ -110,7 +110,8 @@ def test_two_stage_prefill_kernel(D, ps, G):
 def test_two_stage_long_requests(scale_q):
     """The two-stage kernel over many 128-key tiles per item (the slot ring
     wraps many times), a chunked-prefill request whose keys start far before
-    its queries, and (q x 30) a peaked softmax that rescales O in TMEM."""
+    its queries, and (q x 30) a peaked softmax that rescales O in TMEM (bound
+    of the large-logit test below)."""
     spec = W.custom_spec("pairs_long", 16, 4, 128, 64, [1024, 200, 33], [1024, 1500, 2100])
     w = gen(spec, 41)
     if scale_q != 1.0:
@@ -124,7 +125,7 @@ def test_two_stage_long_requests(scale_q):
         compare(out, lse, o_ref, l_ref)
     else:
         vmax = float(w["v_pool"].float().abs().max())
-        compare(out, lse, o_ref, l_ref, tol_o=2.0 ** -8 * vmax,
+        compare(out, lse, o_ref, l_ref, tol_o=2.0 ** -7 * vmax,
                 tol_l=1e-3 * max(1.0, float(np.max(np.abs(l_ref)))))
 
 
@@ -327,17 +328,19 @@ def test_zero_query_closed_form_gpu():
 
 def test_large_logits_gpu():
     """q x 30: a very peaked softmax must neither overflow nor lose accuracy
-    beyond what bf16 allows.  With P rounded to bf16 (relative error <= 2^-9
-    per weight) and O rounded to bf16 (<= 2^-9 |O|), |O - O_ref| is bounded by
-    2^-8 max|V|; N(0,1) inputs with moderate logits stay far below that, but a
-    one-hot softmax reaches it."""
+    beyond what bf16 allows.  bf16 carries an 8-bit significand, so rounding
+    to nearest has relative error <= 2^-8: with P rounded to bf16 for P V
+    (the row sum keeps fp32 P) the weighted sum moves by <= 2^-8 max|V|, and
+    rounding O to bf16 adds <= 2^-8 |O| <= 2^-8 max|V|, so |O - O_ref| is
+    bounded by 2^-7 max|V|; N(0,1) inputs with moderate logits stay far below
+    that, but a one-hot softmax comes near it."""
     spec = W.custom_spec("big", 16, 4, 128, 32, [64, 1], [700, 900])
     w = gen(spec, 23)
     w["q"] = (w["q"].float() * 30.0).to(torch.bfloat16)
     out, lse, _ = gpu_run(w)
     o_ref, l_ref = oracle_all(w)
     vmax = float(w["v_pool"].float().abs().max())
-    compare(out, lse, o_ref, l_ref, tol_o=2.0 ** -8 * vmax,
+    compare(out, lse, o_ref, l_ref, tol_o=2.0 ** -7 * vmax,
             tol_l=1e-3 * max(1.0, float(np.max(np.abs(l_ref)))))
 
 
