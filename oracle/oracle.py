@@ -128,7 +128,8 @@ def paged_attention(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, scale,
 
 
 def paged_attention_rows(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, scale,
-                         row_t, row_h, num_pages: int = 0, nthreads: int | None = None):
+                         row_t, row_h, num_pages: int = 0, nthreads: int | None = None,
+                         lib=None):
     """Only the rows (row_t[u], row_h[u]).  Returns (out [n, D], lse [n])."""
     q, k_pool, v_pool = _u16(q), _u16(k_pool), _u16(v_pool)
     page_table, seq_lens, cu_q_lens = _i32(page_table), _i32(seq_lens), _i32(cu_q_lens)
@@ -139,7 +140,7 @@ def paged_attention_rows(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, sca
     n = int(row_t.shape[0])
     out = np.zeros((n, D), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
-    rc = _load().oracle_paged_attention_rows(
+    rc = (lib or _load()).oracle_paged_attention_rows(
         B, Hq, Hkv, D, ps, C, int(num_pages), _ptr(q), _ptr(k_pool), _ptr(v_pool),
         _ptr(page_table), _ptr(seq_lens), _ptr(cu_q_lens), float(scale), _ptr(row_t),
         _ptr(row_h), n, _ptr(out), _ptr(lse), int(nthreads or default_threads()))
