@@ -317,6 +317,59 @@ def cpu_oracle_rate(w, target_s=10.0, max_reps=50, request_subset=None):
                 seconds=dt)
 
 
+# Requests each workload's CPU-oracle sample takes: whole workloads where one
+# pass takes seconds, otherwise a subset with the workload's own mix (the
+# causal prefill's requests are all alike; the mixed batch keeps its ratio of
+# one prefill request to 31 decode requests).
+CPU_SAMPLE = {
+    "tiny_decode": None,
+    "llama8b_decode": None,
+    "llama8b_causal_prefill": [0],
+    "unified_mixed": [0] + list(range(8, 39)),
+    "long_gqa32_decode": None,
+}
+
+
+def cpu_oracle_config(w, reqs=None, target_s=4.0, max_reps=200):
+    """The CPU oracle, as it stands, on all host cores over the requests
+    ``reqs`` of the workload (all of them when None), repeated until about
+    ``target_s`` seconds.  Rates use the same algorithmic counts as the GPU
+    rows; ``est_seconds_full`` scales the per-pass time to the whole workload
+    by FLOPs (the oracle's cost is one dot product over D per visible
+    (query, key) pair and one weighted V row)."""
+    from oracle import oracle as O
+    B = w["B"]
+    idx = list(range(B)) if reqs is None else [b for b in reqs if b < B]
+    cu = w["cu_q_lens_cpu"].numpy()
+    q_all = W.bf16_bits(w["q"])
+    q = np.concatenate([q_all[cu[b]:cu[b + 1]] for b in idx], 0)
+    q_lens = [int(cu[b + 1] - cu[b]) for b in idx]
+    cu_s = np.zeros(len(idx) + 1, dtype=np.int32)
+    cu_s[1:] = np.cumsum(q_lens)
+    table = w["page_table_cpu"].numpy()[idx]
+    seq = w["seq_lens_cpu"].numpy()[idx]
+    k = W.bf16_bits(w["k_pool"])
+    v = W.bf16_bits(w["v_pool"])
+    threads = O.default_threads()
+    sub = dict(q_lens=q_lens, kv_lens=[int(x) for x in seq], Hq=w["Hq"], Hkv=w["Hkv"],
+               D=w["D"], ps=w["ps"])
+    c_sub, c_all = work_counts(sub), work_counts(w)
+    O.paged_attention(q[:1], k, v, table[:1], seq[:1], np.array([0, 1], np.int32),
+                      w["scale"], nthreads=threads)   # load + build outside the timing
+    reps, t0 = 0, time.time()
+    while reps < max_reps:
+        O.paged_attention(q, k, v, table, seq, cu_s, w["scale"], nthreads=threads)
+        reps += 1
+        if time.time() - t0 >= target_s:
+            break
+    dt = (time.time() - t0) / reps
+    return {"kind": "oracle", "cores": threads, "seconds_per_pass": dt,
+            "GBps": c_sub["bytes"] / dt / 1e9, "TFLOPs": c_sub["flops"] / dt / 1e12,
+            "est_seconds_full": dt * c_all["flops"] / max(1, c_sub["flops"]),
+            "sample": "%d of %d requests (all %d query heads, full KV), %d passes"
+                      % (len(idx), B, w["Hq"], reps)}
+
+
 # ----------------------------------------------------------------------------- main
 def config_desc(w) -> str:
     q, kv = w["q_lens"], w["kv_lens"]
@@ -484,7 +537,7 @@ def main():
         torch.distributed.destroy_process_group()
 
 
-def per_config(peaks):
+def per_config(peaks, cpu=True):
     res = {}
     bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -509,6 +562,8 @@ def per_config(peaks):
         t_fl = c["flops"] / (tf * 1e12)
         r["roofline_ms_max_form"] = max(t_bw, t_fl) * 1e3
         r["roofline_frac_max_form"] = max(t_bw, t_fl) / (attn_ms * 1e-3)
+        if cpu:
+            r["cpu_baseline"] = cpu_oracle_config(w, CPU_SAMPLE.get(name))
         res[name] = r
         del w
         torch.cuda.empty_cache()

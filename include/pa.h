@@ -239,10 +239,12 @@ PA_API int pa_set_decode_kernel(pa_plan *plan, int on);
 PA_API int pa_selftest_wait_timeout(uint32_t limit_us, uint32_t *status_out,
                                     uint32_t *elapsed_us_out);
 
-/* E4M3 (FP8) KV pools with per-tensor descales ("[Attention] FA4
- * integration", vLLM #32974: the fp8 KV-cache variant with descale factors
- * and bf16 output; the format is OCP FP8 E4M3: bias 7, 3 mantissa bits,
- * subnormals, S.1111.111 NaN, no infinities).  With on != 0 the k_pool and
+/* E4M3 (FP8) KV pools with per-tensor descales ("[Perf][FA4] Warm up dense
+ * (paged) FA4 attention kernels", vLLM PR #48156: the Summary's fp8-descale
+ * variants of the dense decode and prefill kernels when the KV cache is fp8,
+ * and the review thread on the per-arch selector, where the fp8 kernel is
+ * SM100-only and writes a bf16 output; the format is OCP FP8 E4M3: bias 7,
+ * 3 mantissa bits, subnormals, S.1111.111 NaN, no infinities).  With on != 0 the k_pool and
  * v_pool of the following pa_run calls are uint8 [P, ps, Hkv, D] arrays of
  * E4M3 codes, and attention is computed as if the pools held
  * k_scale * decode(code) and v_scale * decode(code); q stays bf16, out stays
@@ -295,13 +297,13 @@ PA_API int pa_profile_read(pa_plan *plan, float *attn_ms, int *n_runs, int *laun
  * point exists for integration, not for the method.)
  *
  * Some callers cannot call cudaMalloc at the point where they run attention:
- * a region being captured into a CUDA graph in global capture mode (device
- * allocation is not allowed there), an engine whose device memory is fully
- * budgeted by its own allocator (a raw cudaMalloc would bypass its accounting
- * and can fail late), or a loop where a synchronous allocation would stall
- * the device.  pa_create_plan allocates a workspace, so such callers use this
- * entry point instead: no plan, no cudaMalloc, no cudaFree, no allocating
- * library routine.  The caller still passes every input and output.
+ * an engine whose device memory is fully budgeted by its own allocator (a raw
+ * cudaMalloc would bypass its accounting and can fail late, or take memory
+ * the engine has promised elsewhere), or a serving loop where a synchronous
+ * allocation would stall the device.  pa_create_plan allocates a workspace,
+ * so such callers use this entry point instead: no plan, no cudaMalloc, no
+ * cudaFree, no allocating library routine.  The caller still passes every
+ * input and output.
  *
  * Scratch: the work list and the status word live in one file-scope device
  * array of PA_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU which loads the
@@ -310,7 +312,9 @@ PA_API int pa_profile_read(pa_plan *plan, float *attn_ms, int *n_runs, int *laun
  * items of 32 bytes, plus 44 bytes per request and a small header) is
  * rejected with PA_ERR_UNSUPPORTED and a message saying so.  KV splitting is
  * not used on this path (each (request, KV head, query block) is one item),
- * so there is no split merge and no partial-state storage.
+ * so there is no split merge and no partial-state storage.  The pools are
+ * bf16 only: nothing in the arguments says whether they hold E4M3 codes, so
+ * an fp8 pool passed here would be read as bf16 without an error.
  *
  * All calls share the array and it keeps the last call's contents; each call
  * clears the header it relies on (status word, item count) on `stream` before
@@ -325,7 +329,10 @@ PA_API int pa_profile_read(pa_plan *plan, float *attn_ms, int *n_runs, int *laun
  * Arguments are those of pa_create_plan followed by those of pa_run, plus
  *   num_pages  pool size P for page-id checks (0 = trust the table)
  *   scale      softmax scale (> 0), or 0 for 1/sqrt(head_dim)
- * Returns PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED or PA_ERR_CUDA.
+ * Returns PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED or PA_ERR_CUDA.  Bad
+ * request data found on the device (PA_STATUS_* bits, as for pa_run) is
+ * recorded in the array's status word: read it with pa_noalloc_get_status
+ * before the next pa_run_noalloc on the device, which clears it.
  */
 #define PA_NOALLOC_SCRATCH_BYTES (8u << 20)
 PA_API int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_size,
@@ -333,6 +340,13 @@ PA_API int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, in
                           const void *k_pool, const void *v_pool, const int32_t *page_table,
                           const int32_t *seq_lens, const int32_t *cu_q_lens, void *out,
                           float *lse, pa_stream_t stream);
+
+/* Status word of the last pa_run_noalloc on the current device (no paper
+ * counterpart either): synchronises `stream`, copies the PA_STATUS_* bits to
+ * *status and, if clear != 0, resets them.  Allocates nothing.  Must be read
+ * before the next pa_run_noalloc on the device, which clears the word.
+ * Returns PA_OK, PA_ERR_INVALID (NULL status) or PA_ERR_CUDA. */
+PA_API int pa_noalloc_get_status(pa_stream_t stream, uint32_t *status, int clear);
 
 #ifdef __cplusplus
 }

@@ -29,7 +29,7 @@ EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_sc
            "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc",
            "pa_set_two_stage_prefill", "pa_set_decode_kernel", "pa_append_kv",
            "pa_set_causal", "pa_set_page_table_stride", "pa_set_fused_merge", "pa_set_kv_fp8",
-           "pa_selftest_wait_timeout")
+           "pa_selftest_wait_timeout", "pa_noalloc_get_status")
 
 # Size of the library's static scratch array used by pa_run_noalloc.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -96,6 +96,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_selftest_wait_timeout.restype = I
     lib.pa_run_noalloc.argtypes = [I, I, I, I, I, I, I, F, P, P, P, P, P, P, P, P, P]
     lib.pa_run_noalloc.restype = I
+    lib.pa_noalloc_get_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), I]
+    lib.pa_noalloc_get_status.restype = I
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -322,11 +324,14 @@ def selftest_wait_timeout(limit_us: int):
 def run_noalloc(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, out, lse, *, heads_kv,
                 page_size, capacity, num_pages=0, scale=0.0, stream=None):
     """Call ``pa_run_noalloc``: the attention pass for callers that cannot
-    allocate device memory (the library's static scratch array replaces the
-    plan's workspace).  Every output tensor is passed in; nothing is allocated
-    here or in the library.  The first call on a device does a one-time set-up
-    there, so make it before any stream capture.  Calls that overlap on the GPU
-    race on the shared scratch."""
+    allocate device memory (an engine whose device memory is budgeted by its
+    own allocator, a loop that must not stall on an allocation); the
+    library's static scratch array replaces the plan's workspace.  Every
+    output tensor is passed in; nothing is allocated here or in the library.
+    The first call on a device does a one-time set-up there, so make it
+    before any stream capture.  Calls that overlap on the GPU race on the
+    shared scratch.  Pools are bf16 only.  Read the status word with
+    ``noalloc_status`` before the next call, which clears it."""
     lib = load_library()
     B = seq_lens.shape[0]
     Hq, D = q.shape[1], q.shape[2]
@@ -338,3 +343,16 @@ def run_noalloc(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, out, lse, *,
                               float(scale), _ptr(q), _ptr(k_pool), _ptr(v_pool),
                               _ptr(page_table), _ptr(seq_lens), _ptr(cu_q_lens), _ptr(out),
                               _ptr(lse), ctypes.c_void_p(stream)))
+
+
+def noalloc_status(clear: bool = True, stream=None) -> int:
+    """Synchronise ``stream`` and read (then clear) the status word of the last
+    ``pa_run_noalloc`` on the current device (pa_noalloc_get_status)."""
+    lib = load_library()
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    elif isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    v = ctypes.c_uint32(0)
+    _check(lib.pa_noalloc_get_status(ctypes.c_void_p(stream), ctypes.byref(v), 1 if clear else 0))
+    return int(v.value)

@@ -988,6 +988,29 @@ int noalloc_setup(int dev, NoallocDevice** out) {
 
 }  // namespace
 
+int pa_noalloc_get_status(pa_stream_t stream, uint32_t* status, int clear) {
+  if (!status) { set_err("pa_noalloc_get_status: NULL status"); return PA_ERR_INVALID; }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_err("pa_noalloc_get_status: no current CUDA device");
+    return PA_ERR_CUDA;
+  }
+  NoallocDevice* nd = nullptr;
+  int rc = noalloc_setup(dev, &nd);
+  if (rc) return rc;
+  pa::WsHeader* hdr = static_cast<pa::WsHeader*>(nd->scratch);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(status, &hdr->status, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && clear) e = cudaMemset(&hdr->status, 0, sizeof(uint32_t));
+  if (e != cudaSuccess) {
+    set_err("pa_noalloc_get_status: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
 int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_size,
                    int capacity, int num_pages, float scale, const void* q, const void* k_pool,
                    const void* v_pool, const int32_t* page_table, const int32_t* seq_lens,

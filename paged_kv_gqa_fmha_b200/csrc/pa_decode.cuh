@@ -33,8 +33,9 @@
 // once plus one fp16 V row written and read once.  The products run as fp16
 // MMAs: Q is rounded to fp16 by the Q loader and P is written as fp16.  The K descale multiplies
 // the softmax scale and the V descale the epilogue's 1 / l, so the pools are
-// never dequantised in memory ("[Attention] FA4 integration", vLLM #32974:
-// the fp8 KV-cache variant with descale factors and bf16 output).
+// never dequantised in memory (the fp8-descale variants with a bf16 output of
+// "[Perf][FA4] Warm up dense (paged) FA4 attention kernels", vLLM PR #48156,
+// Summary and the review thread on the per-arch selector).
 #pragma once
 
 #include "pa_kernels.cuh"
