@@ -358,6 +358,29 @@ __device__ __forceinline__ void dec_convert(const AttnParams& p, uint32_t sKV, u
   }
 }
 
+// Compensated O^T product of a request with fewer than kCompKeys keys (one
+// tile, keys kCompKeys .. BN - 1 masked): the softmax stored P_lo^T, the
+// rounding remainder of the 16-bit P^T of key t, at key position t + 64 of
+// the P^T buffer (the second 64-key chunk, unused by such a tile).  The
+// regular product already multiplied that chunk by V rows 64 .. 127, which are
+// zeros past the request's end; this adds V rows 0 .. 63 times P_lo^T.
+template <int D, int NR>
+__device__ __forceinline__ void dec_issue_o_lo(uint32_t tmem, uint32_t slot_addr, uint32_t pb,
+                                               uint32_t idesc) {
+  using C = DecCfg<D, NR>;
+  static_assert(kCompKeys == 64 && C::BN == 128, "P_lo^T uses the second 64-key chunk");
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint64_t bd = smem_desc_sw128(pb + C::P_CHUNK + kk * 32, 16, 1024);
+#pragma unroll
+    for (int hh = 0; hh < C::DH; ++hh) {
+      const uint64_t ad = smem_desc_sw128(slot_addr + 2 * hh * C::SLOT_CHUNK + kk * 16 * 128,
+                                          C::SLOT_CHUNK, 1024);
+      mma_ss_w(tmem + C::O_COL + hh * NR, ad, bd, idesc, 1u);
+    }
+  }
+}
+
 // MMA issuer (all 32 lanes; one elected lane issues).  Per item of n tiles:
 //   S^T(0) | S^T(1) O^T+=V(0)^T P^T(0) | S^T(2) O^T+=V(1)^T P^T(1) | ...
 // g counts tiles over all items: S^T(g) and P^T(g) use buffer g & 1.
@@ -393,7 +416,7 @@ __device__ __forceinline__ void dec_mma(const AttnParams& p, uint32_t sQ, uint32
   };
   // O^T += V^T P^T(gp): A = V tile read MN-major (M = 128 columns of D),
   // B = P^T (K-major, NR rows x 128 keys)
-  auto issue_o = [&](uint32_t gp, uint32_t v_idx, bool first) {
+  auto issue_o = [&](uint32_t gp, uint32_t v_idx, bool first, bool comp) {
     const uint32_t slot_addr = sKV + (v_idx % C::NSLOT) * C::SLOT_BYTES;
     const uint32_t pb = sP + (gp & 1) * C::P_BYTES;
 #pragma unroll
@@ -406,6 +429,7 @@ __device__ __forceinline__ void dec_mma(const AttnParams& p, uint32_t sQ, uint32
         mma_ss_w(tmem + C::O_COL + hh * NR, ad, bd, kIdescO, (!first || kk > 0) ? 1u : 0u);
       }
     }
+    if (comp) dec_issue_o_lo<D, NR>(tmem, slot_addr, pb, kIdescO);
     tc_commit_w(bar0 + 8 * (C::B_PVDONE + (gp & 1)));
   };
 
@@ -434,7 +458,7 @@ __device__ __forceinline__ void dec_mma(const AttnParams& p, uint32_t sQ, uint32
       if (!warp_wait(bar0 + 8 * (C::B_PFULL + (gp & 1)), (gp >> 1) & 1, abort)) { ok = false; break; }
       if (j == 0 && !warp_wait(bar0 + 8 * C::B_OEMPTY, (q_cnt & 1) ^ 1, abort)) { ok = false; break; }
       tc_fence_after();
-      issue_o(gp, v_idx, j == 0);
+      issue_o(gp, v_idx, j == 0, w.kv_len < kCompKeys);
       tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + v_idx % C::NSLOT));
     }
     g += n;
@@ -478,7 +502,7 @@ __device__ __forceinline__ void dec_mma_f8(const AttnParams& p, uint32_t sQ, uin
     return true;
   };
   // O^T += V^T P^T(gp): A = V tile read MN-major, B = P^T (K-major)
-  auto issue_o = [&](uint32_t gp, bool first) -> bool {
+  auto issue_o = [&](uint32_t gp, bool first, bool comp) -> bool {
     const uint32_t slot = gp % C::NSLOT;
     if (!warp_wait(bar0 + 8 * (C::B_KVFULL + slot), (gp / C::NSLOT) & 1, abort)) return false;
     if (!warp_wait(bar0 + 8 * (C::B_PFULL + (gp & 1)), (gp >> 1) & 1, abort)) return false;
@@ -496,6 +520,7 @@ __device__ __forceinline__ void dec_mma_f8(const AttnParams& p, uint32_t sQ, uin
         mma_ss_w(tmem + C::O_COL + hh * NR, ad, bd, kIdescO, (!first || kk > 0) ? 1u : 0u);
       }
     }
+    if (comp) dec_issue_o_lo<D, NR>(tmem, slot_addr, pb, kIdescO);
     tc_commit_w(bar0 + 8 * (C::B_PVDONE + (gp & 1)));
     tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + slot));
     return true;
@@ -515,7 +540,7 @@ __device__ __forceinline__ void dec_mma_f8(const AttnParams& p, uint32_t sQ, uin
         if (!issue_s(g + j + 1, sQb)) { ok = false; break; }
         if (j + 2 == n) tc_commit_w(bar0 + 8 * (C::B_QEMPTY + qb));
       }
-      if (!issue_o(g + j, j == 0)) { ok = false; break; }
+      if (!issue_o(g + j, j == 0, w.kv_len < kCompKeys)) { ok = false; break; }
     }
     g += n;
     ++q_cnt;
@@ -678,16 +703,28 @@ __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, u
         }
         tmem_st_wait();
       }
-      // P^T[r][t] (bf16) into buffer sb: row r of the B operand of O^T
+      // P^T[r][t] (bf16) into buffer sb: row r of the B operand of O^T.  A
+      // request with fewer than kCompKeys keys also gets P_lo^T (the rounding
+      // remainder) at key position t + 64, which its masked keys leave free:
+      // threads t >= 64 (P = 0 there) skip their store
       const uint32_t pb = sP + sb * C::P_BYTES + p_col;
+      const bool comp = w.kv_len < kCompKeys;
+      if (!comp || t < kCompKeys) {
 #pragma unroll
-      for (int r = 0; r < RR; ++r) {
-        const float m_use = m_run[r] == -INFINITY ? 0.f : m_run[r];
-        const float pr = ex2_approx(fmaf(s[r], p.scale_log2, -m_use));
-        l_part[r] = fmaf(l_part[r], alpha[r], pr);
-        asm volatile("st.shared.u16 [%0], %1;" ::"r"(pb + r * 128 + ((p_unit ^ (r & 7)) << 4)),
-                     "h"(F8 ? f16_bits(pr) : bf16_bits(pr))
-                     : "memory");
+        for (int r = 0; r < RR; ++r) {
+          const float m_use = m_run[r] == -INFINITY ? 0.f : m_run[r];
+          const float pr = ex2_approx(fmaf(s[r], p.scale_log2, -m_use));
+          l_part[r] = fmaf(l_part[r], alpha[r], pr);
+          const uint32_t a = pb + r * 128 + ((p_unit ^ (r & 7)) << 4);
+          const unsigned short hi = F8 ? f16_bits(pr) : bf16_bits(pr);
+          asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(hi) : "memory");
+          if (comp) {
+            const float lo = pr - (F8 ? f16_to_f32(hi) : bf16_to_f32(hi));
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(a + C::P_CHUNK),
+                         "h"(F8 ? f16_bits(lo) : bf16_bits(lo))
+                         : "memory");
+          }
+        }
       }
       // (with E4M3 pools the widening warps zero these rows)
       if (!F8 && j == n - 1 && n0 + BN > w.kv_len) {

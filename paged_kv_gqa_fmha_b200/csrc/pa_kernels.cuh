@@ -117,6 +117,17 @@ constexpr int kCostBuckets = 1024;
 constexpr int kSchedSmemReqs = 4096;  // unit offsets of up to this many requests live in smem
 constexpr int kMaxSplits = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows > 2^8
+// Compensated P * V.  The softmax weights feed the P V product as 16-bit
+// values; rounding them costs up to 2^-9 of sum_j P_j |V_j| per row.  With
+// many keys these errors average out, but a row that sees only a few keys
+// can have |O| of 2 to 4, where this error plus the final bf16 rounding of O
+// (up to 2^-8 |O|) can pass 1e-2.  Items holding a row that sees fewer than
+// kCompKeys keys in total therefore also multiply the rounding remainder
+// P_lo = 16-bit(P - P_hi) by V into the same accumulator (P_hi + P_lo
+// carries P to about 2^-17), leaving only the final rounding of O.  Only the
+// first query blocks of each request qualify, so the extra products are a
+// small fraction of the work.
+constexpr int kCompKeys = 64;
 
 // Tile configuration per head dimension.  D = 64 and 128 run two CTAs per SM
 // (64-key tiles, 256 TMEM columns, ~100 KB of shared memory each): two
@@ -269,6 +280,14 @@ __device__ __forceinline__ void split_arrive_and_merge(const AttnParams& p, cons
 }
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Does item w hold a row that sees fewer than kCompKeys keys (all of its keys
+// from key 0, whatever the item's own key range)?  The row with the fewest is
+// the item's first query row: causal limit kv_len - q_len + q_tok0 + 1.
+__device__ __forceinline__ bool item_compensated(const WorkItem& w, int causal) {
+  const int vis0 = causal ? min(w.kv_len, w.kv_len - w.q_len + w.q_tok0 + 1) : w.kv_len;
+  return vis0 < kCompKeys;
+}
 
 __device__ __forceinline__ int item_tiles(const WorkItem& w, int BN) {
   return w.kv_hi > w.kv_lo ? ceil_div(w.kv_hi - w.kv_lo, BN) : 0;
@@ -823,6 +842,7 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
     if (n == 0) continue;
     const uint32_t qb = q_cnt % C::QBUF;
     const uint32_t sQb = sQ + qb * C::Q_BYTES;
+    const bool comp = item_compensated(w, p.causal);
     if (!warp_wait(bar0 + 8 * (C::B_QFULL + qb), (q_cnt / C::QBUF) & 1, abort)) { ok = false; break; }
     tc_fence_after();
     for (int s = 0; s < 2 * n; ++s) {
@@ -864,6 +884,15 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
           mma_ts_w(tmem + C::O_COL, tmem + sb * C::BN + kk * 8, bd, kIdescPV,
                  (j > 0 || kk > 0) ? 1u : 0u);
         }
+        if (comp) {
+          // O += P_lo V: the rounding remainder of P sits in the second half of
+          // the S buffer (columns BN / 2 .. BN - 1)
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            const uint64_t bd = smem_desc_sw128(slot_addr + kk * 16 * 128, C::SLOT_CHUNK, 1024);
+            mma_ts_w(tmem + C::O_COL, tmem + sb * C::BN + C::BN / 2 + kk * 8, bd, kIdescPV, 1u);
+          }
+        }
         tc_commit_w(bar0 + 8 * (C::B_PVDONE + sb));
         tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + slot));
       }
@@ -876,6 +905,39 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
   tc_commit_w(bar0 + 8 * C::B_DRAIN);
   if ((threadIdx.x & 31) == 0) mbar_drain(bar0 + 8 * C::B_DRAIN, 0);
   __syncwarp();
+}
+
+// P = exp2(s * scale_log2 - m) of one row of a BN-key tile, packed as bf16
+// pairs into TMEM columns [taddr, taddr + BN/2); with COMP the rounding
+// remainder P_lo = bf16(P - P_hi) goes to [taddr + BN/2, taddr + BN).  Returns
+// the row sum of the fp32 P.  (The caller waits for the stores.)
+template <int BN, bool COMP>
+__device__ __forceinline__ float write_p(float (&s)[BN], float scale_log2, float m_use,
+                                         uint32_t taddr) {
+  float rowsum = 0.f;
+  uint32_t pk[BN / 2];
+#pragma unroll
+  for (int c = 0; c < BN; c += 2) {
+    const float p0 = ex2_approx(fmaf(s[c], scale_log2, -m_use));
+    const float p1 = ex2_approx(fmaf(s[c + 1], scale_log2, -m_use));
+    rowsum += p0 + p1;
+    pk[c >> 1] = pack_bf16x2(p0, p1);
+    if constexpr (COMP) {
+      s[c] = p0;
+      s[c + 1] = p1;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) tmem_st16(taddr + c * 16, pk + c * 16);
+  if constexpr (COMP) {
+#pragma unroll
+    for (int c = 0; c < BN; c += 2)
+      pk[c >> 1] = pack_bf16x2(s[c] - bf16_to_f32(pk[c >> 1] & 0xffffu),
+                               s[c + 1] - bf16_to_f32(pk[c >> 1] >> 16));
+#pragma unroll
+    for (int c = 0; c < BN / 32; ++c) tmem_st16(taddr + BN / 2 + c * 16, pk + c * 16);
+  }
+  return rowsum;
 }
 
 template <int D>
@@ -902,6 +964,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
     const int t = w.t_base + w.q_tok0 + r / G;
     const int h = w.kvh * G + r % G;
     const bool split = w.n_splits > 1;
+    const bool comp = item_compensated(w, p.causal);
     const size_t prow = ((((size_t)w.b * p.Hkv + w.kvh) * p.S_max + w.split) * kBM + r);
     if (n == 0) {
       // no key is visible to any row of the block: O = 0, LSE = -inf
@@ -985,19 +1048,11 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
           m_run = m_new;
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        float rowsum = 0.f;
-        uint32_t pk[BN / 2];
-#pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_use));
-          const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_use));
-          rowsum += p0 + p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-        }
-        l_run += rowsum;
         // P overwrites the first BN/2 columns of the S buffer it came from
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_st16(trow + sb * BN + c * 16, pk + c * 16);
+        // (compensated items: P_lo the other BN/2); item-uniform branch, each
+        // side its own instance so the common one stays as lean as before
+        l_run += comp ? write_p<BN, true>(s, p.scale_log2, m_use, trow + sb * BN)
+                      : write_p<BN, false>(s, p.scale_log2, m_use, trow + sb * BN);
         tmem_st_wait();
       }
       if (j == n - 1) {

@@ -258,7 +258,8 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
     tc_commit_w(bar0 + 8 * (C::B_SFULL + 2 * x + (gx & 1)));
   };
   // O_X += P_X(gx) V, P read from the first BN/2 columns of its S buffer
-  auto issue_pv = [&](int x, uint32_t gx, uint32_t v_idx, bool first) {
+  // (compensated items: O_X += P_lo V as well, P_lo in the other BN/2 columns)
+  auto issue_pv = [&](int x, uint32_t gx, uint32_t v_idx, bool first, bool comp) {
     const uint32_t slot_addr = sKV + (v_idx % C::NSLOT) * C::SLOT_BYTES;
     const uint32_t p_col = tmem + C::S_COL + (2 * x + (gx & 1)) * C::BN;
 #pragma unroll
@@ -267,6 +268,13 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
       mma_ts_w(tmem + C::O_COL + x * D, p_col + kk * 8, bd, kIdescPV,
                (!first || kk > 0) ? 1u : 0u);
     }
+    if (comp) {
+#pragma unroll
+      for (int kk = 0; kk < C::BN / 16; ++kk) {
+        const uint64_t bd = smem_desc_sw128(slot_addr + kk * 16 * 128, C::SLOT_CHUNK, 1024);
+        mma_ts_w(tmem + C::O_COL + x * D, p_col + C::BN / 2 + kk * 8, bd, kIdescPV, 1u);
+      }
+    }
     tc_commit_w(bar0 + 8 * (C::B_PVDONE + 2 * x + (gx & 1)));
   };
 
@@ -274,6 +282,7 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
     const PairShape ps = pair_shape(w, p.tpb, C::BN, p.causal);
     const int n = ps.n;
     if (n == 0) continue;
+    const bool comp = item_compensated(w, p.causal);   // stage A's first row
     for (int x = 0; x < 2 && ok; ++x)
       if (ps.nt[x] > 0 && !warp_wait(bar0 + 8 * (C::B_QFULL + x), itc[x] & 1, abort)) ok = false;
     if (!ok) break;
@@ -311,7 +320,7 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
           break;
         }
         tc_fence_after();
-        issue_pv(x, gx, v_idx, j == 0);
+        issue_pv(x, gx, v_idx, j == 0, comp);
       }
       if (!ok) break;
       tc_commit_w(bar0 + 8 * (C::B_KVEMPTY + v_idx % C::NSLOT));
@@ -351,6 +360,7 @@ __device__ __forceinline__ void pair_softmax(const CUtensorMap* tm_o, const Attn
   while (ok && items.next(w)) {
     const PairShape ps = pair_shape(w, p.tpb, BN, p.causal);
     const int n = ps.n, tok = ps.tok[x], nt = ps.nt[x];
+    const bool comp = item_compensated(w, p.causal);   // stage A's first row
     const int n_rows = tok * G;
     const bool real = r < n_rows;
     const bool warp_active = warp * 32 < n_rows;
@@ -445,9 +455,19 @@ __device__ __forceinline__ void pair_softmax(const CUtensorMap* tm_o, const Attn
             rs0 += p0;
             rs1 += p1;
             pk[e >> 1] = pack_bf16x2(p0, p1);
+            sc[c * 32 + e] = p0;
+            sc[c * 32 + e + 1] = p1;
           }
           // P overwrites the first BN/2 columns of the S buffer it came from
           tmem_st16(trow + s_col + c * 16, pk);
+          if (comp) {
+            // P_lo = bf16(P - P_hi) into the other BN/2 columns
+#pragma unroll
+            for (int e = 0; e < 32; e += 2)
+              pk[e >> 1] = pack_bf16x2(sc[c * 32 + e] - bf16_to_f32(pk[e >> 1] & 0xffffu),
+                                       sc[c * 32 + e + 1] - bf16_to_f32(pk[e >> 1] >> 16));
+            tmem_st16(trow + s_col + BN / 2 + c * 16, pk);
+          }
         }
         l_run += rs0 + rs1;
         tmem_st_wait();

@@ -365,6 +365,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// bf16 bits -> fp32 (exact: the bf16 bits are the high half of a binary32).
+__device__ __forceinline__ float bf16_to_f32(uint32_t bits) { return __uint_as_float(bits << 16); }
+// fp16 bits -> fp32 (exact).
+__device__ __forceinline__ float f16_to_f32(unsigned short h) {
+  float f;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
+  return f;
+}
 // fp32 -> fp16 bits, round to nearest even.
 __device__ __forceinline__ unsigned short f16_bits(float x) {
   unsigned short h;

@@ -346,6 +346,67 @@ def test_large_logits_gpu():
             tol_l=1e-3 * np.maximum(1.0, np.abs(l_ref)))
 
 
+# ------------------------------------------------------------------ rows with few keys
+def _vis_counts(w, causal=True):
+    """Visible keys of every (token) row: [T]."""
+    cu = w["cu_q_lens_cpu"].numpy()
+    seq = w["seq_lens_cpu"].numpy()
+    out = np.zeros(w["T"], dtype=np.int64)
+    for b in range(w["B"]):
+        qb = cu[b + 1] - cu[b]
+        for i in range(qb):
+            out[cu[b] + i] = seq[b] if not causal else min(seq[b], max(0, seq[b] - qb + i + 1))
+    return out
+
+
+@pytest.mark.parametrize("kind", ["one_stage", "two_stage", "decode_kernel", "d256", "d64",
+                                  "decode_fp8"])
+def test_few_key_rows_are_correctly_rounded(kind):
+    """Rows that see fewer than 64 keys in total take the compensated P V
+    (P_hi + P_lo, both 16-bit): their outputs equal the oracle's exact result
+    correctly rounded to bf16, up to fp32 slack of 2^-14 max(|O|, 1) (the
+    fp32 sums run over terms P_j V_j of magnitude up to max |V|, so the slack
+    does not shrink with |O|) -- far inside the 2^-9 sum_j P_j |V_j| that
+    rounding P alone would leave.  Rows with more keys meet the usual bar."""
+    if kind in ("decode_kernel", "decode_fp8"):
+        kv = [2, 3, 4, 5, 7, 8, 13, 31, 63, 64, 2, 3, 9]
+        spec = W.custom_spec("few_dec", 16, 4, 128, 16, [1] * len(kv), kv, decode_only=True)
+    elif kind == "d256":
+        spec = W.custom_spec("few256", 8, 2, 256, 32, [40, 70, 3], [40, 70, 90])
+    elif kind == "d64":
+        spec = W.custom_spec("few64", 16, 2, 64, 16, [64, 100, 33], [64, 100, 50])
+    else:
+        spec = W.custom_spec("few", 16, 4, 128, 16, [64] * 6 + [150], [64] * 6 + [150])
+    w = gen(spec, 60 + len(kind))
+    plan = make_plan(w)
+    use_cu = not spec.decode_only
+    if kind == "two_stage":
+        plan.set_two_stage_prefill(True)
+    if kind == "decode_fp8":
+        k8 = (w["k_pool"].float() * 4).to(torch.float8_e4m3fn)
+        v8 = (w["v_pool"].float() * 4).to(torch.float8_e4m3fn)
+        plan.set_kv_fp8(True, 0.25, 0.25)
+        out, lse = plan.run(w["q"], k8.view(torch.uint8), v8.view(torch.uint8),
+                            w["page_table"], w["seq_lens"], None)
+        torch.cuda.synchronize()
+        o_ref, l_ref = O.paged_attention_fp8(
+            W.bf16_bits(w["q"]), k8.view(torch.uint8).cpu().numpy(),
+            v8.view(torch.uint8).cpu().numpy(), 0.25, 0.25, w["page_table_cpu"].numpy(),
+            w["seq_lens_cpu"].numpy(), w["cu_q_lens_cpu"].numpy(), w["scale"])
+    else:
+        out, lse, _ = gpu_run(w, plan, use_cu=use_cu)
+        o_ref, l_ref = oracle_all(w)
+    assert plan.status() == 0
+    compare(out, lse, o_ref, l_ref)
+    few = _vis_counts(w) < 64
+    o = out.float().cpu().numpy().astype(np.float64)[few]
+    x = o_ref[few]
+    rounded = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    slack = 2.0 ** -14 * np.maximum(np.abs(x), 1.0)
+    excess = np.abs(o - x) - (np.abs(rounded - x) + slack)
+    assert np.all(excess <= 0), "few-key row off its correctly rounded value by %g" % excess.max()
+
+
 # ------------------------------------------------------------------ full-size configs, every element
 # Each of the five workloads at its full size, in the launch configuration
 # bench.py times (default plan), and the opt-in two-stage kernel where it
