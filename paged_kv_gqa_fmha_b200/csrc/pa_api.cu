@@ -105,7 +105,7 @@ struct pa_plan {
   int tstride;                 // page-table row stride in int32 entries (default C)
   int o_tma;                   // tm_o is used (G divides 32)
   CUtensorMap tm_k2, tm_v2;   // page boxes of box_h2 rows
-  int kv_fp8;                  // 1: the pools hold E4M3 codes (decode kernel only)
+  int kv_fp8;                  // 1: the pools hold E4M3 codes
   float k_scale, v_scale;      // their per-tensor descales
   int tm_fp8;                  // the pool maps were encoded for E4M3 pools
 };
@@ -215,9 +215,15 @@ cudaError_t set_decode_smem_attr() {
 
 template <int D>
 cudaError_t set_smem_attr() {
-  cudaError_t e = cudaFuncSetAttribute(pa::pa_attention_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(pa::pa_attention_kernel<D, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       pa::TileCfg<D>::SMEM_BYTES);
+                                       pa::TileCfg<D, false>::SMEM_BYTES);
+  if constexpr (D >= 128) {
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(pa::pa_attention_kernel<D, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               pa::TileCfg<D, true>::SMEM_BYTES);
+  }
   if constexpr (D <= 128) {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(pa::pa_pair_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -288,30 +294,34 @@ cudaError_t launch_pairs(int n_sm, cudaStream_t st, const CUtensorMap& tq, const
 // The attention kernel and the merge are programmatic dependents of the
 // kernel launched before them on the stream (their prologues overlap it; each
 // waits with griddepcontrol.wait before reading its results).
-template <int D>
+template <int D, bool F8>
 cudaError_t launch_attention(int n_sm, cudaStream_t st, const CUtensorMap& tq,
                              const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& to, const pa::AttnParams& ap) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pa::TileCfg<D>::CTAS * n_sm);
+  cfg.gridDim = dim3(pa::TileCfg<D, F8>::CTAS * n_sm);
   cfg.blockDim = dim3(pa::kThreads);
-  cfg.dynamicSmemBytes = pa::TileCfg<D>::SMEM_BYTES;
+  cfg.dynamicSmemBytes = pa::TileCfg<D, F8>::SMEM_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, pa::pa_attention_kernel<D>, tq, tk, tv, to, ap);
+  return cudaLaunchKernelEx(&cfg, pa::pa_attention_kernel<D, F8>, tq, tk, tv, to, ap);
 }
 
-cudaError_t launch_attention_d(int D, int n_sm, cudaStream_t st, const CUtensorMap& tq,
+// fp8: E4M3 pools (head_dim 128 or 256; pa_set_kv_fp8 refuses 64)
+cudaError_t launch_attention_d(int D, bool fp8, int n_sm, cudaStream_t st, const CUtensorMap& tq,
                                const CUtensorMap& tk, const CUtensorMap& tv,
                                const CUtensorMap& to, const pa::AttnParams& ap) {
+  if (fp8)
+    return D == 128 ? launch_attention<128, true>(n_sm, st, tq, tk, tv, to, ap)
+                    : launch_attention<256, true>(n_sm, st, tq, tk, tv, to, ap);
   switch (D) {
-    case 64: return launch_attention<64>(n_sm, st, tq, tk, tv, to, ap);
-    case 128: return launch_attention<128>(n_sm, st, tq, tk, tv, to, ap);
-    default: return launch_attention<256>(n_sm, st, tq, tk, tv, to, ap);
+    case 64: return launch_attention<64, false>(n_sm, st, tq, tk, tv, to, ap);
+    case 128: return launch_attention<128, false>(n_sm, st, tq, tk, tv, to, ap);
+    default: return launch_attention<256, false>(n_sm, st, tq, tk, tv, to, ap);
   }
 }
 
@@ -614,10 +624,6 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     set_err("pa_run: current device %d is not the plan's device %d", dev, p->device);
     return PA_ERR_INVALID;
   }
-  if (p->kv_fp8 && cu_q_lens != nullptr) {
-    set_err("pa_run: E4M3 pools are read by the decode kernel only (cu_q_lens must be NULL)");
-    return PA_ERR_UNSUPPORTED;
-  }
   int rc = build_maps(p, q, k_pool, v_pool, out);
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -632,8 +638,9 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.req_aux = bufs.req_aux;
   sp.unit_off = bufs.unit_off;
   sp.split_list = bufs.split_list;
-  // without cu_q_lens every request is one decode token: no query-block pairs
-  const bool pairs = p->use_pairs && cu_q_lens != nullptr;
+  // without cu_q_lens every request is one decode token: no query-block pairs;
+  // the two-stage kernel reads bf16 pools only, so E4M3 pools skip it too
+  const bool pairs = p->use_pairs && cu_q_lens != nullptr && !p->kv_fp8;
   sp.items2 = pairs ? bufs.items2 : nullptr;
   sp.unit_off2 = bufs.unit_off2;
   sp.max_items2 = p->max_items2;
@@ -694,7 +701,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   }
   if (le == cudaSuccess)
     le = dec ? launch_decode(p->D, p->G, p->kv_fp8 != 0, p->n_sm, st, p->tm_k, p->tm_v, ap)
-             : launch_attention_d(p->D, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v, p->tm_o, ap);
+             : launch_attention_d(p->D, p->kv_fp8 != 0, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v,
+                                  p->tm_o, ap);
   if (prof) {
     cudaEventRecord(p->prof_ev[2 * p->prof_n + 1], st);
     ++p->prof_n;
@@ -838,7 +846,7 @@ int pa_set_kv_fp8(pa_plan* p, int on, float k_scale, float v_scale) {
     return PA_ERR_INVALID;
   }
   if (p->D != 128 && p->D != 256) {
-    set_err("pa_set_kv_fp8: head_dim %d has no E4M3 decode kernel (128 and 256 only)", p->D);
+    set_err("pa_set_kv_fp8: head_dim %d has no E4M3 kernels (128 and 256 only)", p->D);
     return PA_ERR_UNSUPPORTED;
   }
   p->kv_fp8 = 1;
@@ -1155,7 +1163,7 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
   ap.scale_log2 = sc * 1.4426950408889634f;
   CUtensorMap tm_none;
   memset(&tm_none, 0, sizeof(tm_none));
-  e = launch_attention_d(head_dim, nd->n_sm, st, tm_q, tm_k, tm_v, tm_none, ap);
+  e = launch_attention_d(head_dim, false, nd->n_sm, st, tm_q, tm_k, tm_v, tm_none, ap);
   if (e != cudaSuccess) {
     set_err("pa_run_noalloc: launch failed: %s", cudaGetErrorString(e));
     return PA_ERR_CUDA;

@@ -133,8 +133,12 @@ constexpr int kCompKeys = 64;
 // (64-key tiles, 256 TMEM columns, ~100 KB of shared memory each): two
 // independent load -> S -> softmax -> P V chains per SM hide each other's
 // latencies, which one CTA per SM cannot.  D = 256 needs the whole SM.
-template <int D>
+// F8: E4M3 pools.  The producer's TMA boxes land in NST fp8 staging tiles and
+// a converter warp widens them to fp16 in the 16-bit slots the MMAs read (one
+// slot fewer for D = 128, so the shared memory per CTA stays the same).
+template <int D, bool F8 = false>
 struct TileCfg {
+  static_assert(!F8 || D >= 128, "E4M3 pools: head_dim 128 or 256");
   static constexpr int CTAS = (D == 256) ? 1 : 2;      // CTAs per SM
   // 16 warps on 4 sub-partitions: 4 warps x 32 lanes x 128 = 16 K registers each
   static constexpr int MAXREG = (CTAS == 2) ? 128 : 255;
@@ -145,23 +149,26 @@ struct TileCfg {
   static constexpr int SLOT_CHUNK = BN * 128;         // bytes of one K/V column chunk
   static constexpr int SLOT_BYTES = BN * D * 2;
   static constexpr int QBUF = (D == 64) ? 2 : 1;      // Q tiles in flight
-  static constexpr int NSLOT = (D == 64) ? 8 : (D == 128 ? 4 : 5);
+  static constexpr int NSLOT = F8 ? (D == 128 ? 3 : 4) : ((D == 64) ? 8 : (D == 128 ? 4 : 5));
+  static constexpr int NST = F8 ? 2 : 0;              // fp8 staging tiles
+  static constexpr int STAGE_BYTES = BN * D;          // D / 128 chunks of BN rows x 128 bytes
   static constexpr int O_COL = 2 * BN;                // TMEM: S0 [0,BN), S1 [BN,2BN), O
   static constexpr int TMEM_COLS = (O_COL + D <= 256) ? 256 : 512;
   static constexpr int OCH = (CTAS == 2) ? 1 : 2;     // 32-column O chunks per TMEM wait
   // barriers: q_full[QBUF], q_empty[QBUF], kv_full[NSLOT], kv_empty[NSLOT], s_full[2],
-  //           p_full[2], pv_done[2], o_empty, drain
+  //           p_full[2], pv_done[2], o_empty, drain, st_full[NST], st_empty[NST]
   static constexpr int B_QFULL = 0, B_QEMPTY = QBUF, B_KVFULL = 2 * QBUF,
                        B_KVEMPTY = 2 * QBUF + NSLOT, B_SFULL = 2 * QBUF + 2 * NSLOT,
                        B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2, B_OEMPTY = B_PVDONE + 2,
-                       B_DRAIN = B_OEMPTY + 1, NBAR = B_DRAIN + 1;
+                       B_DRAIN = B_OEMPTY + 1, B_STFULL = B_DRAIN + 1,
+                       B_STEMPTY = B_STFULL + NST, NBAR = B_STEMPTY + NST;
   static constexpr int BAR_BYTES = 512;
   // epilogue staging: per softmax warp 32 rows x 32 columns of bf16 (64-byte
-  // swizzle); D = 256 has no room for it next to its five K/V slots
+  // swizzle); D = 256 has no room for it next to its K/V slots
   static constexpr int EPI_WARP_BYTES = 32 * 64;
   static constexpr int EPI_BYTES = (D == 256) ? 0 : 4 * EPI_WARP_BYTES;
-  static constexpr int SMEM_BYTES =
-      1024 + QBUF * Q_BYTES + NSLOT * SLOT_BYTES + EPI_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + QBUF * Q_BYTES + NSLOT * SLOT_BYTES +
+                                    NST * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
   static_assert(NBAR * 8 + 16 <= BAR_BYTES, "barrier area");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(CTAS == 1 || 2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
@@ -694,12 +701,14 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
 // inside [0, T) use one TMA box per 64-column chunk; partial blocks (decode,
 // last block of a request) use plain 16-byte loads of the live rows only,
 // stored with the same 128-byte swizzle the TMA applies (16-byte unit u of
-// row r lands at unit u ^ (r % 8) of that row).
-template <int D>
+// row r lands at unit u ^ (r % 8) of that row).  With E4M3 pools (F8) the MMAs
+// run in fp16: every block takes the plain-load path and is rounded to fp16
+// (magnitudes past 65504 saturate) on the way to shared memory.
+template <int D, bool F8>
 __device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const AttnParams& p,
                                               uint32_t sQ, uint32_t bar0, int n_items,
                                               volatile int* abort) {
-  using C = TileCfg<D>;
+  using C = TileCfg<D, F8>;
   const int lane = threadIdx.x & 31;
   const int G = p.G;
   const int T = p.cu_q_lens ? p.cu_q_lens[p.B] : p.B;
@@ -713,7 +722,7 @@ __device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const Att
     const uint32_t qfull = bar0 + 8 * (C::B_QFULL + qb);
     if (!warp_wait(bar0 + 8 * (C::B_QEMPTY + qb), ((q_cnt / C::QBUF) & 1) ^ 1, abort)) break;
     const int t0 = w.t_base + w.q_tok0;
-    if (w.n_tok == p.tpb && t0 + p.tpb <= T) {
+    if (!F8 && w.n_tok == p.tpb && t0 + p.tpb <= T) {
       if (lane == 0) {
         mbar_arrive_expect_tx(qfull, C::DCH * p.tpb * G * 128);
         for (int c = 0; c < C::DCH; ++c)
@@ -740,6 +749,12 @@ __device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const Att
             const int r = u / (D / 8), c16 = u % (D / 8);
             const uint32_t dst =
                 sQb + (c16 >> 3) * C::Q_CHUNK + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+            if constexpr (F8) {
+              v[k].x = bf16x2_to_f16x2_sat(v[k].x);
+              v[k].y = bf16x2_to_f16x2_sat(v[k].y);
+              v[k].z = bf16x2_to_f16x2_sat(v[k].z);
+              v[k].w = bf16x2_to_f16x2_sat(v[k].w);
+            }
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[k].x),
                          "r"(v[k].y), "r"(v[k].z), "r"(v[k].w)
                          : "memory");
@@ -754,7 +769,7 @@ __device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const Att
     // Q is read once, so it always comes from DRAM: pull the next item's Q
     // tile into L2 now so that its load is short when its turn comes.
     WorkItem nw;
-    if (lane == 0 && items.peek(nw) && item_tiles(nw, C::BN) > 0 && nw.n_tok == p.tpb) {
+    if (!F8 && lane == 0 && items.peek(nw) && item_tiles(nw, C::BN) > 0 && nw.n_tok == p.tpb) {
       const int tn = nw.t_base + nw.q_tok0;
       if (tn + p.tpb <= T)
         for (int c = 0; c < C::DCH; ++c) tma_prefetch_l2_3d(tm_q, c * 64, nw.kvh * G, tn);
@@ -768,15 +783,23 @@ __device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const Att
 
 // KV producer warp: K and V tiles in the MMA's consumption order into the slot
 // ring.  One TMA box is one page (or the part of a page inside the tile) of
-// one KV head; lane k issues box k.  Both producers walk the order; this one
-// issues the loads whose index has parity `which` and skips the others.  Each
-// lane reads its page id from the table right before its box (a loop-carried
-// look-ahead of the ids made every producer wait on every load's table read).
-template <int D>
+// one KV head; lane k issues box k.  With bf16 pools both producers walk the
+// order; this one issues the loads whose index has parity `which` and skips
+// the others.  With E4M3 pools (F8) one producer (which = 2) issues every
+// load, into the fp8 staging ring the converter warp drains.  Each lane reads
+// its page id from the table right before its box (a loop-carried look-ahead
+// of the ids made every producer wait on every load's table read).
+template <int D, bool F8>
 __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const AttnParams& p, uint32_t sKV, uint32_t bar0,
                                               int n_items, uint32_t which, volatile int* abort) {
-  using C = TileCfg<D>;
+  using C = TileCfg<D, F8>;
+  constexpr int RING = F8 ? C::NST : C::NSLOT;
+  constexpr int B_FULL = F8 ? C::B_STFULL : C::B_KVFULL;
+  constexpr int B_EMPTY = F8 ? C::B_STEMPTY : C::B_KVEMPTY;
+  constexpr int RING_BYTES = F8 ? C::STAGE_BYTES : C::SLOT_BYTES;
+  constexpr int NCH = F8 ? D / 128 : C::DCH;   // boxes (128-byte column chunks) per page part
+  constexpr int CH_ELEMS = F8 ? 128 : 64;      // elements of one chunk
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
@@ -785,12 +808,12 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
   while (ok && items.next(w)) {
     const int n = item_tiles(w, C::BN);
     for (int s = 0; s < 2 * n; ++s, ++ld_idx) {
-      if ((ld_idx & 1u) != which) continue;
+      if (which < 2 && (ld_idx & 1u) != which) continue;
       int j;
       bool is_v;
       kv_sequence(s, n, j, is_v);
-      const uint32_t slot = ld_idx % C::NSLOT;
-      if (!warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
+      const uint32_t slot = ld_idx % RING;
+      if (!warp_wait(bar0 + 8 * (B_EMPTY + slot), ((ld_idx / RING) & 1) ^ 1, abort)) {
         ok = false;
         break;
       }
@@ -799,8 +822,8 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
       // included) so that no stale shared memory meets P * V
       const int live = min(w.kv_len - n0, C::BN);
       const int nbox = (live + p.box_h - 1) >> p.box_log2;
-      const uint32_t full = bar0 + 8 * (C::B_KVFULL + slot);
-      if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * C::DCH);
+      const uint32_t full = bar0 + 8 * (B_FULL + slot);
+      if (lane == 0) mbar_arrive_expect_tx(full, nbox * p.box_h * 128 * NCH);
       __syncwarp();
       if (lane < nbox) {
         const int r = n0 + lane * p.box_h;     // < kv_len <= C * ps
@@ -810,29 +833,119 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
           page = -1;   // out of the tensor map: the box reads as zeros
         }
         const CUtensorMap* tm = is_v ? tm_v : tm_k;
-        const uint32_t dst = sKV + slot * C::SLOT_BYTES + lane * p.box_h * 128;
-        for (int c = 0; c < C::DCH; ++c)
-          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * 64, w.kvh, r & (p.ps - 1), page);
+        const uint32_t dst = sKV + slot * RING_BYTES + lane * p.box_h * 128;
+        for (int c = 0; c < NCH; ++c)
+          tma_load_4d(dst + c * C::SLOT_CHUNK, tm, full, c * CH_ELEMS, w.kvh, r & (p.ps - 1),
+                      page);
       }
     }
   }
   if (!ok || *abort) {
     // wait (bounded) for our copies still in flight before the CTA exits
     if (lane == 0) {
-      const uint32_t first = ld_idx > (uint32_t)C::NSLOT ? ld_idx - C::NSLOT : 0;
+      const uint32_t first = ld_idx > (uint32_t)RING ? ld_idx - RING : 0;
       for (uint32_t k = first; k < ld_idx; ++k)
-        if ((k & 1u) == which) mbar_drain(bar0 + 8 * (C::B_KVFULL + k % C::NSLOT), (k / C::NSLOT) & 1);
+        if (which > 1 || (k & 1u) == which)
+          mbar_drain(bar0 + 8 * (B_FULL + k % RING), (k / RING) & 1);
     }
   }
 }
 
+// E4M3 converter warp (F8).  Walks the producer's load order; staging tile
+// i % NST holds load i as D / 128 chunks of 64 rows x 128 bytes (16-byte unit
+// x of row r at x ^ (r & 7), the TMA 128-byte swizzle).  Each code is widened
+// to fp16 with cvt.rn.f16x2.e4m3x2 (exact: every E4M3 value is an fp16 value)
+// into 16-bit slot i % NSLOT, laid out as a TMA-loaded bf16 tile would be
+// (64-column chunks, 128-byte swizzle), so the MMAs read it unchanged.  The 8
+// lanes of a store phase take one 16-byte unit of 8 consecutive rows, whose
+// swizzled places in the staging tile and in the slot fall in 8 distinct bank
+// groups.  V rows at and past the request's end are written as zeros (P is 0
+// there, but 0 * NaN is not); K rows there only meet masked scores.
 template <int D>
+__device__ __forceinline__ void convert_role(const AttnParams& p, uint32_t sKV, uint32_t sST,
+                                             uint32_t bar0, int n_items, volatile int* abort) {
+  using C = TileCfg<D, true>;
+  constexpr int UPR = D / 16;                        // 16-byte fp8 units per row
+  constexpr int UNITS = C::BN * UPR;
+  const int lane = threadIdx.x & 31;
+  uint32_t ld_idx = 0;
+  bool ok = true;
+  ItemStream items(p.items, n_items, p.tpb);
+  WorkItem w;
+  while (ok && items.next(w)) {
+    const int n = item_tiles(w, C::BN);
+    for (int s = 0; s < 2 * n; ++s, ++ld_idx) {
+      int j;
+      bool is_v;
+      kv_sequence(s, n, j, is_v);
+      const uint32_t st = ld_idx % C::NST, slot = ld_idx % C::NSLOT;
+      if (!warp_wait(bar0 + 8 * (C::B_STFULL + st), (ld_idx / C::NST) & 1, abort) ||
+          !warp_wait(bar0 + 8 * (C::B_KVEMPTY + slot), ((ld_idx / C::NSLOT) & 1) ^ 1, abort)) {
+        ok = false;
+        break;
+      }
+      const int n0 = w.kv_lo + j * C::BN;
+      const int zero_from = is_v ? max(0, min(C::BN, w.kv_len - n0)) : C::BN;
+      const uint32_t src0 = sST + st * C::STAGE_BYTES;
+      const uint32_t dst0 = sKV + slot * C::SLOT_BYTES;
+#pragma unroll 1
+      for (int u0 = 0; u0 < UNITS; u0 += 8 * 32) {
+        uint32_t x[8][4];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {                 // all loads of the pass first
+          const int u = u0 + e * 32 + lane;
+          const int row = (u & 7) + 8 * (u / (8 * UPR)), k = (u >> 3) % UPR;
+          if (row < zero_from) {
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(x[e][0]), "=r"(x[e][1]), "=r"(x[e][2]), "=r"(x[e][3])
+                         : "r"(src0 + (k >> 3) * C::SLOT_CHUNK + row * 128 +
+                               (((k & 7) ^ (row & 7)) << 4)));
+          } else {
+            x[e][0] = x[e][1] = x[e][2] = x[e][3] = 0u;   // E4M3 code 0 is +0
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int u = u0 + e * 32 + lane;
+          const int row = (u & 7) + 8 * (u / (8 * UPR)), k = (u >> 3) % UPR;
+          uint32_t h[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) e4m3x4_to_f16x4(x[e][q], h[2 * q], h[2 * q + 1]);
+          // halves 0-7 go to 16-byte unit 2 (k & 3) of the 64-column chunk
+          // k / 4, halves 8-15 to the next unit (unit y stored at y ^ (row & 7))
+          const uint32_t rbase = dst0 + (k >> 2) * C::SLOT_CHUNK + row * 128;
+          const uint32_t y0 = 2 * (k & 3);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           rbase + ((y0 ^ (row & 7)) << 4)),
+                       "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           rbase + (((y0 + 1) ^ (row & 7)) << 4)),
+                       "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar0 + 8 * (C::B_KVFULL + slot));
+        mbar_arrive(bar0 + 8 * (C::B_STEMPTY + st));
+      }
+    }
+  }
+}
+
+// MMA issuer.  bf16 operands, or fp16 ones with E4M3 pools (F8: Q rounded to
+// fp16 by the Q loader, K and V widened by the converter, P written as fp16).
+template <int D, bool F8>
 __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint32_t sKV,
                                          uint32_t bar0, uint32_t tmem, int n_items,
                                          volatile int* abort) {
-  using C = TileCfg<D>;
-  constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, C::BN, false, false);
-  constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, false, true);
+  using C = TileCfg<D, F8>;
+  constexpr uint32_t kIdescS = F8 ? idesc_f16_f32(kBM, C::BN, false, false)
+                                  : idesc_bf16_f32(kBM, C::BN, false, false);
+  constexpr uint32_t kIdescPV = F8 ? idesc_f16_f32(kBM, D, false, true)
+                                   : idesc_bf16_f32(kBM, D, false, true);
   uint32_t ld_idx = 0, g_base = 0, q_cnt = 0;
   bool ok = true;
   ItemStream items(p.items, n_items, p.tpb);
@@ -908,10 +1021,10 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
 }
 
 // P = exp2(s * scale_log2 - m) of one row of a BN-key tile, packed as bf16
-// pairs into TMEM columns [taddr, taddr + BN/2); with COMP the rounding
-// remainder P_lo = bf16(P - P_hi) goes to [taddr + BN/2, taddr + BN).  Returns
-// the row sum of the fp32 P.  (The caller waits for the stores.)
-template <int BN, bool COMP>
+// pairs (fp16 with F16) into TMEM columns [taddr, taddr + BN/2); with COMP the
+// rounding remainder P_lo = 16-bit(P - P_hi) goes to [taddr + BN/2, taddr + BN).
+// Returns the row sum of the fp32 P.  (The caller waits for the stores.)
+template <int BN, bool COMP, bool F16 = false>
 __device__ __forceinline__ float write_p(float (&s)[BN], float scale_log2, float m_use,
                                          uint32_t taddr) {
   float rowsum = 0.f;
@@ -921,7 +1034,7 @@ __device__ __forceinline__ float write_p(float (&s)[BN], float scale_log2, float
     const float p0 = ex2_approx(fmaf(s[c], scale_log2, -m_use));
     const float p1 = ex2_approx(fmaf(s[c + 1], scale_log2, -m_use));
     rowsum += p0 + p1;
-    pk[c >> 1] = pack_bf16x2(p0, p1);
+    pk[c >> 1] = F16 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
     if constexpr (COMP) {
       s[c] = p0;
       s[c + 1] = p1;
@@ -931,20 +1044,25 @@ __device__ __forceinline__ float write_p(float (&s)[BN], float scale_log2, float
   for (int c = 0; c < BN / 32; ++c) tmem_st16(taddr + c * 16, pk + c * 16);
   if constexpr (COMP) {
 #pragma unroll
-    for (int c = 0; c < BN; c += 2)
-      pk[c >> 1] = pack_bf16x2(s[c] - bf16_to_f32(pk[c >> 1] & 0xffffu),
-                               s[c + 1] - bf16_to_f32(pk[c >> 1] >> 16));
+    for (int c = 0; c < BN; c += 2) {
+      if constexpr (F16)
+        pk[c >> 1] = pack_f16x2(s[c] - f16_to_f32((unsigned short)(pk[c >> 1] & 0xffffu)),
+                                s[c + 1] - f16_to_f32((unsigned short)(pk[c >> 1] >> 16)));
+      else
+        pk[c >> 1] = pack_bf16x2(s[c] - bf16_to_f32(pk[c >> 1] & 0xffffu),
+                                 s[c + 1] - bf16_to_f32(pk[c >> 1] >> 16));
+    }
 #pragma unroll
     for (int c = 0; c < BN / 32; ++c) tmem_st16(taddr + BN / 2 + c * 16, pk + c * 16);
   }
   return rowsum;
 }
 
-template <int D>
+template <int D, bool F8>
 __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const AttnParams& p,
                                              uint32_t sKV, uint32_t sEpi, uint32_t bar0,
                                              uint32_t tmem, int n_items, volatile int* abort) {
-  using C = TileCfg<D>;
+  using C = TileCfg<D, F8>;
   constexpr int BN = C::BN;
   const int r = threadIdx.x;          // query row of the tile, 0..127
   const int warp = r >> 5, lane = r & 31;
@@ -1051,15 +1169,16 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
         // P overwrites the first BN/2 columns of the S buffer it came from
         // (compensated items: P_lo the other BN/2); item-uniform branch, each
         // side its own instance so the common one stays as lean as before
-        l_run += comp ? write_p<BN, true>(s, p.scale_log2, m_use, trow + sb * BN)
-                      : write_p<BN, false>(s, p.scale_log2, m_use, trow + sb * BN);
+        l_run += comp ? write_p<BN, true, F8>(s, p.scale_log2, m_use, trow + sb * BN)
+                      : write_p<BN, false, F8>(s, p.scale_log2, m_use, trow + sb * BN);
         tmem_st_wait();
       }
       if (j == n - 1) {
-        if (n0 + BN > w.kv_len) {
+        if (!F8 && n0 + BN > w.kv_len) {
           // Last tile of the request: rows at and past kv_len in the V tile are
           // tail slots or rows never loaded; zero them so that 0 * garbage
-          // cannot reach O (P is 0 there, but 0 * NaN is NaN).
+          // cannot reach O (P is 0 there, but 0 * NaN is NaN).  (The E4M3
+          // converter writes those rows as zeros itself.)
           const uint32_t ldv = ld_base + 2 * n - 1;
           const uint32_t slot = ldv % C::NSLOT;
           if (!warp_wait(bar0 + 8 * (C::B_KVFULL + slot), (ldv / C::NSLOT) & 1, abort)) {
@@ -1095,7 +1214,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
     if (!warp_wait(bar0 + 8 * (C::B_PVDONE + (gl & 1)), (gl >> 1) & 1, abort)) { ok = false; break; }
     tc_fence_after();
     if (warp_active) {
-      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+      const float inv_l = l_run > 0.f ? p.v_scale / l_run : 0.f;   // V descale (1 for bf16)
       const float lse_v = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
       // whole blocks of 32 / G tokens per warp go out through TMA stores
       const bool o_tma = C::EPI_BYTES > 0 && !split && p.o_tma && w.n_tok == p.tpb &&
@@ -1175,22 +1294,23 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
   if (lane == 0) bulk_wait_all();   // O stores complete before the CTA exits
 }
 
-template <int D>
-__global__ void __maxnreg__(TileCfg<D>::MAXREG)
+template <int D, bool F8 = false>
+__global__ void __maxnreg__((TileCfg<D, F8>::MAXREG))
     pa_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_o, const AttnParams p) {
-  using C = TileCfg<D>;
+  using C = TileCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;             // 1024-B aligned for SW128
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t sQ = base;
   const uint32_t sKV = base + C::QBUF * C::Q_BYTES;
-  const uint32_t sEpi = sKV + C::NSLOT * C::SLOT_BYTES;
+  const uint32_t sST = sKV + C::NSLOT * C::SLOT_BYTES;     // fp8 staging (F8 only)
+  const uint32_t sEpi = sST + C::NST * C::STAGE_BYTES;
   const uint32_t bar0 = sEpi + C::EPI_BYTES;
-  uint8_t* bar_ptr = smem + C::QBUF * C::Q_BYTES + C::NSLOT * C::SLOT_BYTES + C::EPI_BYTES;
+  uint8_t* bar_ptr = smem + (bar0 - base);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NBAR);
   volatile int* abort = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 4);
 
@@ -1201,8 +1321,13 @@ __global__ void __maxnreg__(TileCfg<D>::MAXREG)
       mbar_init(bar0 + 8 * (C::B_QEMPTY + i), 1);
     }
     for (int i = 0; i < C::NSLOT; ++i) {
+      // filled by TMA (one expect_tx arrival) or by the converter warp (F8)
       mbar_init(bar0 + 8 * (C::B_KVFULL + i), 1);
       mbar_init(bar0 + 8 * (C::B_KVEMPTY + i), 1);
+    }
+    for (int i = 0; i < C::NST; ++i) {
+      mbar_init(bar0 + 8 * (C::B_STFULL + i), 1);
+      mbar_init(bar0 + 8 * (C::B_STEMPTY + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar0 + 8 * (C::B_SFULL + i), 1);
@@ -1218,11 +1343,11 @@ __global__ void __maxnreg__(TileCfg<D>::MAXREG)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if ((warp == kProducerWarp || warp == kProducer2Warp) && (threadIdx.x & 31) == 0) {
+  if ((warp == kProducerWarp || (!F8 && warp == kProducer2Warp)) && (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == kQWarp && (threadIdx.x & 31) == 0) tma_prefetch_desc(&tm_q);
+  if (!F8 && warp == kQWarp && (threadIdx.x & 31) == 0) tma_prefetch_desc(&tm_q);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1233,13 +1358,21 @@ __global__ void __maxnreg__(TileCfg<D>::MAXREG)
   const int n_items = p.hdr->n_items;
 
   if (warp == kProducerWarp || warp == kProducer2Warp) {
-    producer_role<D>(&tm_k, &tm_v, p, sKV, bar0, n_items, warp == kProducerWarp ? 0u : 1u, abort);
+    if constexpr (F8) {
+      // one producer issues every load into the staging ring; the other warp
+      // widens the staged tiles into the 16-bit slots
+      if (warp == kProducerWarp) producer_role<D, true>(&tm_k, &tm_v, p, sST, bar0, n_items, 2u, abort);
+      else convert_role<D>(p, sKV, sST, bar0, n_items, abort);
+    } else {
+      producer_role<D, false>(&tm_k, &tm_v, p, sKV, bar0, n_items,
+                              warp == kProducerWarp ? 0u : 1u, abort);
+    }
   } else if (warp == kQWarp) {
-    q_loader_role<D>(&tm_q, p, sQ, bar0, n_items, abort);
+    q_loader_role<D, F8>(&tm_q, p, sQ, bar0, n_items, abort);
   } else if (warp == kMmaWarp) {
-    mma_role<D>(p, sQ, sKV, bar0, tmem, n_items, abort);   // all 32 lanes
+    mma_role<D, F8>(p, sQ, sKV, bar0, tmem, n_items, abort);   // all 32 lanes
   } else {
-    softmax_role<D>(&tm_o, p, sKV, sEpi, bar0, tmem, n_items, abort);
+    softmax_role<D, F8>(&tm_o, p, sKV, sEpi, bar0, tmem, n_items, abort);
   }
 
   tc_fence_before();

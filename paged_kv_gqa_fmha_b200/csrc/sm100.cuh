@@ -373,6 +373,12 @@ __device__ __forceinline__ float f16_to_f32(unsigned short h) {
   asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
   return f;
 }
+// Two fp32 -> packed fp16x2, round to nearest even; `lo` goes to the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 // fp32 -> fp16 bits, round to nearest even.
 __device__ __forceinline__ unsigned short f16_bits(float x) {
   unsigned short h;

@@ -1,5 +1,7 @@
-"""GPU parity of the E4M3 (FP8) KV decode path (pa_set_kv_fp8 + pa_run,
-through the C ABI) with the oracle's attention over fp8 pools.
+"""GPU parity of the E4M3 (FP8) KV paths (pa_set_kv_fp8 + pa_run, through
+the C ABI) with the oracle's attention over fp8 pools: decode-only runs on the
+keys-as-M decode kernel, prefill, chunked prefill and mixed batches on the
+one-stage kernel (codes widened to fp16 in shared memory).
 
 The pools hold E4M3 codes of N(0,1) * 4 values (torch's round-to-nearest
 quantisation); the descales are arbitrary non-powers of two so that a missing
@@ -59,8 +61,9 @@ def _oracle(w, k8, v8):
                                  w["scale"])
 
 
-def _run(plan, w, k8, v8):
-    out, lse = plan.run(w["q"], k8, v8, w["page_table"], w["seq_lens"], None)
+def _run(plan, w, k8, v8, use_cu=False):
+    out, lse = plan.run(w["q"], k8, v8, w["page_table"], w["seq_lens"],
+                        w["cu_q_lens"] if use_cu else None)
     torch.cuda.synchronize()
     assert plan.status() == 0
     return out, lse
@@ -126,15 +129,78 @@ def test_fp8_rejections():
     w, k8, v8 = _fp8_workload(spec, 3)
     plan = _plan(w)
     with pytest.raises(binding.PAError) as e:
-        plan.run(w["q"], k8, v8, w["page_table"], w["seq_lens"], w["cu_q_lens"])
-    assert e.value.code == binding.PA_ERR_UNSUPPORTED
-    with pytest.raises(binding.PAError) as e:
         plan.set_kv_fp8(True, 0.0, 1.0)
     assert e.value.code == binding.PA_ERR_INVALID
     p64 = binding.Plan(2, 8, 2, 64, 16, 8)
     with pytest.raises(binding.PAError) as e:
         p64.set_kv_fp8(True, 1.0, 1.0)
     assert e.value.code == binding.PA_ERR_UNSUPPORTED
+
+
+PREFILL_GEOMS = [  # seed, D, G, ps, Hkv, q_lens, kv_lens
+    (11, 128, 4, 16, 2, [300, 1, 77, 129, 1], [300, 900, 500, 129, 64]),
+    (12, 128, 8, 64, 1, [64, 200, 1], [64, 1000, 40]),
+    (13, 128, 1, 128, 2, [100, 31], [700, 31]),
+    (14, 128, 32, 32, 1, [9, 4, 1], [9, 300, 800]),
+    (15, 256, 4, 32, 2, [90, 1, 40], [90, 500, 300]),
+    (16, 256, 2, 128, 1, [130, 3], [400, 3]),
+    (17, 128, 3, 16, 2, [50, 1, 2], [50, 60, 500]),
+]
+
+
+@pytest.mark.parametrize("seed,D,G,ps,Hkv,q_lens,kv_lens", PREFILL_GEOMS)
+def test_fp8_prefill_and_mixed_match_oracle(seed, D, G, ps, Hkv, q_lens, kv_lens):
+    """Causal prefill, chunked prefill (kv > q) and decode rows in one batch
+    over E4M3 pools, on the one-stage kernel, against the oracle; NaN codes
+    in every request's tail slots must not reach O."""
+    spec = W.custom_spec("fp8_pf", G * Hkv, Hkv, D, ps, q_lens, kv_lens)
+    w, k8, v8 = _fp8_workload(spec, 700 + seed)
+    out, lse = _run(_plan(w), w, k8, v8, use_cu=True)
+    compare(out, lse, *_oracle(w, k8, v8))
+
+
+@pytest.mark.parametrize("splits,fused,two_stage", [(0, False, False), (3, False, False),
+                                                    (3, True, False), (0, False, True)])
+def test_fp8_mixed_batch_options(splits, fused, two_stage):
+    """A mixed batch over E4M3 pools with KV splits for its single-token
+    requests (separate or fused merge), and with the two-stage prefill option
+    on (E4M3 runs stay on the one-stage kernel)."""
+    spec = W.custom_spec("fp8_mix", 32, 8, 128, 16, [200, 1, 1, 64, 1], [200, 1500, 90, 700, 3000])
+    w, k8, v8 = _fp8_workload(spec, 41)
+    plan = _plan(w, num_splits=splits)
+    plan.set_fused_merge(fused)
+    if two_stage:
+        plan.set_two_stage_prefill(True)
+    out, lse = _run(plan, w, k8, v8, use_cu=True)
+    compare(out, lse, *_oracle(w, k8, v8))
+
+
+def test_fp8_prefill_non_causal_and_descales():
+    """Non-causal mode and a second pair of descales on the same codes."""
+    spec = W.custom_spec("fp8_nc", 16, 4, 128, 32, [100, 1, 37], [300, 200, 37])
+    w, k8, v8 = _fp8_workload(spec, 43)
+    plan = _plan(w)
+    plan.set_causal(False)
+    for ks, vs in ((K_SCALE, V_SCALE), (0.05, 0.9)):
+        plan.set_kv_fp8(True, ks, vs)
+        out, lse = _run(plan, w, k8, v8, use_cu=True)
+        compare(out, lse, *_oracle_nc(w, k8, v8, ks, vs))
+
+
+def _oracle_nc(w, k8, v8, ks, vs):
+    """Non-causal reference over E4M3 pools: every query token becomes a
+    one-token request with its own request's page-table row and KV length, so
+    the oracle's (end-aligned causal) fp8 entry lets it see all of its keys."""
+    cu = w["cu_q_lens_cpu"].numpy()
+    seq = w["seq_lens_cpu"].numpy()
+    table = w["page_table_cpu"].numpy()
+    q = W.bf16_bits(w["q"])
+    T = w["T"]
+    rows_req = np.concatenate([np.full(cu[b + 1] - cu[b], b, dtype=np.int64) for b in range(w["B"])])
+    o, l = O.paged_attention_fp8(q, k8.cpu().numpy(), v8.cpu().numpy(), ks, vs,
+                                 table[rows_req], seq[rows_req], np.arange(T + 1, dtype=np.int32),
+                                 w["scale"])
+    return o, l
 
 
 @pytest.mark.slow
@@ -152,3 +218,20 @@ def test_fp8_full_size_llama_decode_every_element():
     err_o, err_l = compare(out, lse, o_ref, l_ref)
     print("llama8b_decode/fp8: %d elements, max|O-oracle| %.3e, max|LSE-oracle| %.3e"
           % (out.numel(), err_o, err_l))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["llama8b_causal_prefill", "unified_mixed"])
+def test_fp8_full_size_prefill_and_mixed_every_element(name):
+    """The causal-prefill and mixed-batch workloads at full size over E4M3 pools
+    (quantised on the device): every element of O and LSE against the oracle."""
+    w = W.generate(W.CONFIGS[name], W.default_seed(name), device="cuda")
+    k8 = (w["k_pool"].float() * 4).to(torch.float8_e4m3fn).view(torch.uint8)
+    v8 = (w["v_pool"].float() * 4).to(torch.float8_e4m3fn).view(torch.uint8)
+    del w["k_pool"], w["v_pool"]
+    plan = _plan(w)
+    out, lse = _run(plan, w, k8, v8, use_cu=True)
+    o_ref, l_ref = _oracle(w, k8, v8)
+    err_o, err_l = compare(out, lse, o_ref, l_ref)
+    print("%s/fp8: %d elements, max|O-oracle| %.3e, max|LSE-oracle| %.3e"
+          % (name, out.numel(), err_o, err_l))
