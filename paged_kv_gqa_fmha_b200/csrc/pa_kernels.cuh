@@ -1027,13 +1027,18 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
 template <int BN, bool COMP, bool F16 = false>
 __device__ __forceinline__ float write_p(float (&s)[BN], float scale_log2, float m_use,
                                          uint32_t taddr) {
-  float rowsum = 0.f;
+  // s * scale_log2 - m and the row sum in packed fp32 pairs (half the
+  // instructions); the sum runs in two independent pair accumulators
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_use, -m_use);
+  uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
   uint32_t pk[BN / 2];
 #pragma unroll
   for (int c = 0; c < BN; c += 2) {
-    const float p0 = ex2_approx(fmaf(s[c], scale_log2, -m_use));
-    const float p1 = ex2_approx(fmaf(s[c + 1], scale_log2, -m_use));
-    rowsum += p0 + p1;
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nm2), x0, x1);
+    const float p0 = ex2_approx(x0);
+    const float p1 = ex2_approx(x1);
+    rs2[(c >> 1) & 1] = f2_add(rs2[(c >> 1) & 1], f2_pack(p0, p1));
     pk[c >> 1] = F16 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
     if constexpr (COMP) {
       s[c] = p0;
@@ -1055,7 +1060,10 @@ __device__ __forceinline__ float write_p(float (&s)[BN], float scale_log2, float
 #pragma unroll
     for (int c = 0; c < BN / 32; ++c) tmem_st16(taddr + BN / 2 + c * 16, pk + c * 16);
   }
-  return rowsum;
+  float a0, a1, b0, b1;
+  f2_unpack(rs2[0], a0, a1);
+  f2_unpack(rs2[1], b0, b1);
+  return (a0 + b0) + (a1 + b1);
 }
 
 template <int D, bool F8>
@@ -1129,9 +1137,14 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
           for (int c = 0; c < BN; ++c)
             if (c >= nvis) s[c] = -INFINITY;   // mask by select, never by add
         }
-        float mx = -INFINITY;
+        // row maximum: four independent chains of three-input maxima
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < BN; c += 8) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) mx4[k] = fmax3(mx4[k], s[c + 2 * k], s[c + 2 * k + 1]);
+        }
+        const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
         const float m_new = fmaxf(m_run, mx * p.scale_log2);
         const bool need = real && (m_new > m_run + kRescaleThreshold);
         if (j > 0 && __any_sync(0xffffffffu, need && m_run != -INFINITY)) {
