@@ -201,6 +201,32 @@ int alloc_workspace(pa_plan* p) {
   return PA_OK;
 }
 
+// The E4M3 decode kernel splits its launch registers between warpgroups with
+// setmaxnreg (see DecCfg): a build whose kernel uses another launch count
+// would leave the softmax warpgroup's increase unsatisfiable, so it is
+// refused before any launch.
+template <int D, int RR>
+bool decode_f8_regs_ok(int* got) {
+  cudaFuncAttributes a;
+  if (cudaFuncGetAttributes(&a, pa::pa_decode_kernel<D, RR, true>) != cudaSuccess) return false;
+  *got = a.numRegs;
+  return a.numRegs == pa::DecCfg<D, pa::DecRows<RR>::NR, true>::LAUNCH_REGS;
+}
+
+template <int D>
+int check_decode_f8_regs(const char* who) {
+  int got = -1;
+  const bool ok = decode_f8_regs_ok<D, 4>(&got) && decode_f8_regs_ok<D, 8>(&got) &&
+                  decode_f8_regs_ok<D, 16>(&got) && decode_f8_regs_ok<D, 32>(&got);
+  if (!ok) {
+    set_err("%s: the E4M3 decode kernel for head_dim %d was built with %d registers per "
+            "thread; its warpgroup register split needs exactly %d", who, D, got,
+            pa::DecCfg<D, 16, true>::LAUNCH_REGS);
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
 template <int D, int RR>
 cudaError_t set_decode_smem_attr() {
   cudaError_t e = cudaFuncSetAttribute(pa::pa_decode_kernel<D, RR, false>,
@@ -503,6 +529,9 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
     set_err("pa_create_plan: cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
     return nullptr;
   }
+  if ((head_dim == 128 && check_decode_f8_regs<128>("pa_create_plan") != PA_OK) ||
+      (head_dim == 256 && check_decode_f8_regs<256>("pa_create_plan") != PA_OK))
+    return nullptr;
   pa_plan* p = new pa_plan();
   p->B = batch; p->Hq = heads_q; p->Hkv = heads_kv; p->D = head_dim; p->ps = page_size;
   p->C = capacity; p->G = G; p->device = dev; p->n_sm = n_sm;

@@ -71,6 +71,16 @@ struct DecCfg {
   static constexpr int TMEM_COLS =
       TMEM_USED <= 32 ? 32 : (TMEM_USED <= 64 ? 64 : (TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512)));
   static constexpr int THREADS = F8 ? 384 : 256;
+  // E4M3 variant: launched with LAUNCH_REGS per thread (384 threads, one CTA
+  // per SM); the softmax warpgroup then takes SOFTMAX_REGS (up to 32 rows of
+  // running maxima, sums, scores and scale factors per thread), the producer /
+  // MMA / Q warpgroup and the widening warpgroup give registers back.  The
+  // budgets sum to at most the launch pool (the host checks the compiled
+  // launch count before any launch).
+  static constexpr int LAUNCH_REGS = 168;
+  static constexpr int SOFTMAX_REGS = 224, WG1_REGS = 80, CONV_REGS = 128;
+  static_assert(!F8 || 128 * (SOFTMAX_REGS + WG1_REGS + CONV_REGS) <= THREADS * LAUNCH_REGS,
+                "warpgroup register budgets exceed the launch pool");
   static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5, Q_WARP = 6, PRODUCER2_WARP = 7;
   static constexpr int CONV_WARP0 = 8;                // E4M3 widening warps 8-11
   // barriers: q_full[2], q_empty[2], kv_full[NSLOT], kv_empty[NSLOT], s_full[2],
@@ -805,6 +815,7 @@ struct DecRows {
 
 template <int D, int RR, bool F8 = false>
 __global__ void __launch_bounds__(DecCfg<D, DecRows<RR>::NR, F8>::THREADS, 1)
+    __maxnreg__((F8 ? DecCfg<D, DecRows<RR>::NR, F8>::LAUNCH_REGS : 255))
     pa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   constexpr int NR = DecRows<RR>::NR;
@@ -873,18 +884,35 @@ __global__ void __launch_bounds__(DecCfg<D, DecRows<RR>::NR, F8>::THREADS, 1)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int n_items = p.hdr->n_items;
 
-  if (warp == C::PRODUCER_WARP || warp == C::PRODUCER2_WARP) {
-    dec_producer<D, NR, F8>(&tm_k, &tm_v, p, F8 ? sST : sKV, bar0, n_items,
-                            warp == C::PRODUCER_WARP ? 0u : 1u, abort);
-  } else if (warp == C::Q_WARP) {
-    dec_q_loader<D, NR, F8>(p, sQ, bar0, n_items, abort);
-  } else if (warp == C::MMA_WARP) {
-    if constexpr (F8) dec_mma_f8<D, NR>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
-    else dec_mma<D, NR>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
-  } else if (warp < kSoftmaxWarps) {
-    dec_softmax<D, NR, RR, F8>(p, sKV, sP, red, bar0, tmem, n_items, abort);
+  if constexpr (F8) {
+    // per-warpgroup register budgets first, then the roles
+    if (warp < kSoftmaxWarps) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
+      dec_softmax<D, NR, RR, F8>(p, sKV, sP, red, bar0, tmem, n_items, abort);
+    } else if (warp < C::CONV_WARP0) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::WG1_REGS));
+      if (warp == C::PRODUCER_WARP || warp == C::PRODUCER2_WARP)
+        dec_producer<D, NR, F8>(&tm_k, &tm_v, p, sST, bar0, n_items,
+                                warp == C::PRODUCER_WARP ? 0u : 1u, abort);
+      else if (warp == C::Q_WARP)
+        dec_q_loader<D, NR, F8>(p, sQ, bar0, n_items, abort);
+      else
+        dec_mma_f8<D, NR>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
+    } else {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONV_REGS));
+      dec_convert<D, NR>(p, sKV, sST, bar0, tmem, n_items, abort);
+    }
   } else {
-    if constexpr (F8) dec_convert<D, NR>(p, sKV, sST, bar0, tmem, n_items, abort);
+    if (warp == C::PRODUCER_WARP || warp == C::PRODUCER2_WARP) {
+      dec_producer<D, NR, F8>(&tm_k, &tm_v, p, sKV, bar0, n_items,
+                              warp == C::PRODUCER_WARP ? 0u : 1u, abort);
+    } else if (warp == C::Q_WARP) {
+      dec_q_loader<D, NR, F8>(p, sQ, bar0, n_items, abort);
+    } else if (warp == C::MMA_WARP) {
+      dec_mma<D, NR>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
+    } else if (warp < kSoftmaxWarps) {
+      dec_softmax<D, NR, RR, F8>(p, sKV, sP, red, bar0, tmem, n_items, abort);
+    }
   }
 
   tc_fence_before();
