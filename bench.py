@@ -404,7 +404,7 @@ def attention_kernel_name(w, decode_only: bool) -> str:
         while rr < G:
             rr *= 2
         return "pa_decode_kernel<128, %d, false>" % rr
-    return "pa_attention_kernel<%d>" % w["D"]
+    return "pa_attention_kernel<%d, false>" % w["D"]
 
 
 def main():
@@ -417,8 +417,8 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(W.CONFIGS),
                     help="workload of the timed steps (default: the headline decode)")
     ap.add_argument("--kv-fp8", action="store_true",
-                    help="E4M3 pools (decode workloads; implies --no-extra): the metric "
-                         "then counts one byte per K/V element")
+                    help="E4M3 pools (implies --no-extra): the metric then counts one byte "
+                         "per K/V element")
     args = ap.parse_args()
     if args.kv_fp8:
         args.no_extra = True
@@ -477,14 +477,13 @@ def main():
     plan = make_plan(w)
     kernel = attention_kernel_name(w, spec.decode_only)
     if args.kv_fp8:
-        if not spec.decode_only:
-            raise SystemExit("--kv-fp8: E4M3 pools are read by the decode kernel only")
         to_fp8_pools(w)
         plan.set_kv_fp8(True, FP8_DESCALE, FP8_DESCALE)
         counts["bytes"] -= counts["kv_bytes"] // 2
         counts["kv_bytes"] //= 2
-        kernel = "pa_decode_kernel<%d, %d, true>" % (
+        kernel = ("pa_decode_kernel<%d, %d, true>" % (
             w["D"], max(4, 1 << (w["Hq"] // w["Hkv"] - 1).bit_length()))
+            if spec.decode_only else "pa_attention_kernel<%d, true>" % w["D"])
     clocks = ClockSampler(local)
     clocks.start()
     ms, attn_ms, per_run, status = time_headline(w, plan, args.steps, args.warmup, dist_on)
@@ -568,7 +567,7 @@ def per_config(peaks, cpu=True):
         del w
         torch.cuda.empty_cache()
     res["kv_append"] = kv_append_rates(bw)
-    res["kv_fp8_decode"] = kv_fp8_decode_rates(bw)
+    res["kv_fp8"] = kv_fp8_rates(bw, tf)
     return res
 
 
@@ -591,34 +590,43 @@ def to_fp8_pools(w):
     torch.cuda.empty_cache()
 
 
-def kv_fp8_decode_rates(bw):
-    """Decode over E4M3 pools (pa_set_kv_fp8) on the decode workloads: the
-    bf16 pools are quantised on the device (x4, round to nearest E4M3) and
-    read back with descales 0.25.  Bytes per launch = the bf16 formula with K
-    and V at one byte per element; per-launch CUDA events (the plan's profile
-    pairs) over 20 launches after 5 warm-up launches (pools larger than L2)."""
+def kv_fp8_rates(bw, tf):
+    """Every non-tiny workload over E4M3 pools (pa_set_kv_fp8): the bf16 pools
+    are quantised on the device (x4, round to nearest E4M3) and read back with
+    descales 0.25.  Decode-only workloads run on the E4M3 decode kernel,
+    prefill and mixed batches on the one-stage kernel's E4M3 variant.  Bytes
+    per launch = the bf16 formula with K and V at one byte per element;
+    per-launch CUDA events (the plan's profile pairs) over 20 launches, each
+    synchronised, after 5 warm-up launches (pools larger than L2)."""
     out = {}
-    for name in ("llama8b_decode", "long_gqa32_decode"):
-        w = W.generate(W.CONFIGS[name], W.default_seed(name), device="cuda")
+    for name in ("llama8b_decode", "llama8b_causal_prefill", "unified_mixed",
+                 "long_gqa32_decode"):
+        spec = W.CONFIGS[name]
+        w = W.generate(spec, W.default_seed(name), device="cuda")
         c = work_counts(w)
         to_fp8_pools(w)
         plan = make_plan(w)
         plan.set_kv_fp8(True, FP8_DESCALE, FP8_DESCALE)
-        args = (w["q"], w["k_pool"], w["v_pool"], w["page_table"], w["seq_lens"], None)
+        args = (w["q"], w["k_pool"], w["v_pool"], w["page_table"], w["seq_lens"],
+                None if spec.decode_only else w["cu_q_lens"])
         for _ in range(5):
             plan.run(*args)
         torch.cuda.synchronize()
         plan.profile_start(20)
         for _ in range(20):
             plan.run(*args)
+            torch.cuda.synchronize()
         attn_ms, n_rec, _ = plan.profile_read()
         ms = attn_ms / max(1, n_rec)
         nbytes = c["bytes"] - c["kv_bytes"] // 2
         gbs = nbytes / (ms * 1e-3) / 1e9
-        out[name] = {"attn_kernel_ms": ms, "algorithmic_bytes": nbytes, "kernel_GBps": gbs,
-                     "hbm_frac": gbs / bw, "status_word": plan.status(),
-                     "kernel": "pa_decode_kernel<%d, %d, true>" % (
-                         w["D"], max(4, 1 << (w["Hq"] // w["Hkv"] - 1).bit_length()))}
+        tfs = c["flops"] / (ms * 1e-3) / 1e12
+        G = w["Hq"] // w["Hkv"]
+        kernel = ("pa_decode_kernel<%d, %d, true>" % (w["D"], max(4, 1 << (G - 1).bit_length()))
+                  if spec.decode_only else "pa_attention_kernel<%d, true>" % w["D"])
+        out[name] = {"attn_kernel_ms": ms, "algorithmic_bytes": nbytes, "flops": c["flops"],
+                     "kernel_GBps": gbs, "kernel_TFLOPs": tfs, "hbm_frac": gbs / bw,
+                     "tensor_frac": tfs / tf, "status_word": plan.status(), "kernel": kernel}
         plan.close()
         del w
         torch.cuda.empty_cache()
