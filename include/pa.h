@@ -250,8 +250,10 @@ PA_API int pa_selftest_wait_timeout(uint32_t limit_us, uint32_t *status_out,
  * k_scale * decode(code) and v_scale * decode(code); q stays bf16, out stays
  * bf16, lse is the log-sum-exp of the descaled logits.  The codes are widened
  * to fp16 on chip (exact); q and the softmax weights P are rounded to fp16 for
- * the MMAs (q magnitudes past 65504 saturate).  Decode only: pa_run returns
- * PA_ERR_UNSUPPORTED when cu_q_lens is not NULL while this is on.  on = 0
+ * the MMAs (q magnitudes past 65504 saturate).  Decode-only runs (cu_q_lens
+ * NULL) use the E4M3 decode kernel; runs with cu_q_lens (prefill, chunked
+ * prefill, mixed batches) use the one-stage kernel's E4M3 variant, also when
+ * pa_set_two_stage_prefill is on (that kernel reads bf16 pools only).  on = 0
  * restores bf16 pools (descales ignored).  Returns PA_ERR_INVALID for a NULL
  * plan or a descale that is not finite and > 0, PA_ERR_UNSUPPORTED for a
  * head_dim other than 128 or 256. */
