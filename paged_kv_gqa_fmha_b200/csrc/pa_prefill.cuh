@@ -17,10 +17,11 @@
 // so S_X(g) is always issued after P_X(g-2) V, which keeps the phases of the
 // per-buffer barriers unambiguous.
 //
-// Roles (11 warps, one CTA per SM):
+// Roles (12 warps, one CTA per SM):
 //   warps 0-3   stage A: softmax, correction, epilogue (thread r = query row r)
 //   warps 4-7   the same for stage B
-//   warp  8     K/V producer (page-table-driven TMA, order K0 K1 V0 K2 V1 ...)
+//   warps 8, 11 K/V producers (page-table-driven TMA; each issues the loads of
+//               one parity of the order K0 K1 V0 K2 V1 ...)
 //   warp  9     MMA issuer (warp-collective issue, one elected lane)
 //   warp  10    Q loader (Q_A and Q_B buffers in shared memory)
 // TMEM (512 columns): S_A0 S_A1 S_B0 S_B1 (BN each), O_A, O_B (D each).
@@ -46,8 +47,8 @@ struct PairCfg {
   static constexpr int S_COL = 0;                      // + (2 * stage + buffer) * BN
   static constexpr int O_COL = 4 * BN;                 // + stage * D
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 352;
-  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, Q_WARP = 10;
+  static constexpr int THREADS = 384;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, Q_WARP = 10, PRODUCER2_WARP = 11;
   // barriers: q_full[2], q_empty[2], kv_full[NSLOT], kv_empty[NSLOT],
   //           s_full[2][2], p_full[2][2], pv_done[2][2], o_empty[2], drain
   static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NSLOT,
@@ -173,7 +174,7 @@ __device__ __forceinline__ void pair_q_loader(const CUtensorMap* tm_q, const Att
 template <int D>
 __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const AttnParams& p, uint32_t sKV, uint32_t bar0,
-                                              int n_items, volatile int* abort) {
+                                              int n_items, uint32_t which, volatile int* abort) {
   using C = PairCfg<D>;
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
@@ -183,6 +184,7 @@ __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUt
   while (ok && items.next(w)) {
     const int n = pair_shape(w, p.tpb, C::BN, p.causal).n;
     for (int s = 0; s < 2 * n; ++s, ++ld_idx) {
+      if ((ld_idx & 1u) != which) continue;
       int j;
       bool is_v;
       kv_sequence(s, n, j, is_v);
@@ -215,7 +217,7 @@ __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUt
     if (lane == 0) {
       const uint32_t first = ld_idx > (uint32_t)C::NSLOT ? ld_idx - C::NSLOT : 0;
       for (uint32_t k = first; k < ld_idx; ++k)
-        mbar_drain(bar0 + 8 * (C::B_KVFULL + k % C::NSLOT), (k / C::NSLOT) & 1);
+        if ((k & 1u) == which) mbar_drain(bar0 + 8 * (C::B_KVFULL + k % C::NSLOT), (k / C::NSLOT) & 1);
     }
   }
 }
@@ -415,8 +417,11 @@ __device__ __forceinline__ void pair_softmax(const CUtensorMap* tm_o, const Attn
         }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], sc[c]);
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        for (int c = 0; c < BN; c += 8) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) mx4[k] = fmax3(mx4[k], sc[c + 2 * k], sc[c + 2 * k + 1]);
+        }
+        const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
         const float m_new = fmaxf(m_run, mx * p.scale_log2);
         const bool need = real && (m_new > m_run + kRescaleThreshold);
         if (j > 0 && __any_sync(0xffffffffu, need && m_run != -INFINITY)) {
@@ -444,16 +449,19 @@ __device__ __forceinline__ void pair_softmax(const CUtensorMap* tm_o, const Attn
           m_run = m_new;
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        float rs0 = 0.f, rs1 = 0.f;
+        // s * scale_log2 - m and the row sum in packed fp32 pairs
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-m_use, -m_use);
+        uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2_approx(fmaf(sc[c * 32 + e], p.scale_log2, -m_use));
-            const float p1 = ex2_approx(fmaf(sc[c * 32 + e + 1], p.scale_log2, -m_use));
-            rs0 += p0;
-            rs1 += p1;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(sc[c * 32 + e], sc[c * 32 + e + 1]), sc2, nm2), x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            rs2[(e >> 1) & 1] = f2_add(rs2[(e >> 1) & 1], f2_pack(p0, p1));
             pk[e >> 1] = pack_bf16x2(p0, p1);
             sc[c * 32 + e] = p0;
             sc[c * 32 + e + 1] = p1;
@@ -469,7 +477,12 @@ __device__ __forceinline__ void pair_softmax(const CUtensorMap* tm_o, const Attn
             tmem_st16(trow + s_col + BN / 2 + c * 16, pk);
           }
         }
-        l_run += rs0 + rs1;
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(rs2[0], a0, a1);
+          f2_unpack(rs2[1], b0, b1);
+          l_run += (a0 + b0) + (a1 + b1);
+        }
         tmem_st_wait();
       }
       if (j == n - 1 && zero_v) {
@@ -602,7 +615,7 @@ __global__ void __maxnreg__(168)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == C::PRODUCER_WARP && (threadIdx.x & 31) == 0) {
+  if ((warp == C::PRODUCER_WARP || warp == C::PRODUCER2_WARP) && (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
@@ -615,8 +628,9 @@ __global__ void __maxnreg__(168)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int n_items = p.hdr->n_items2;
 
-  if (warp == C::PRODUCER_WARP) {
-    pair_producer<D>(&tm_k, &tm_v, p, sKV, bar0, n_items, abort);
+  if (warp == C::PRODUCER_WARP || warp == C::PRODUCER2_WARP) {
+    pair_producer<D>(&tm_k, &tm_v, p, sKV, bar0, n_items,
+                     warp == C::PRODUCER_WARP ? 0u : 1u, abort);
   } else if (warp == C::Q_WARP) {
     pair_q_loader<D>(&tm_q, p, sQ, bar0, n_items, abort);
   } else if (warp == C::MMA_WARP) {
