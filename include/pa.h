@@ -183,17 +183,18 @@ PA_API int pa_max_splits(const pa_plan *plan);
 PA_API int pa_set_two_stage_prefill(pa_plan *plan, int on);
 
 /* Split-KV merge.  0 (default): a separate merge kernel runs after the
- * attention kernel.  1: fused -- every softmax warp of a split item counts
- * itself in a per-(request, KV head) counter after writing its partial state,
- * and the warp that arrives last merges all splits of that (request, KV head)
- * (the fused split reduction with a per-run counter that "integrate PrimTS
- * FMHA kernels", section "Planning, preprocessing, and workspace ownership",
- * names; here the scheduler zeroes the counters every run and no warp waits
- * for another).  The fused form saves the merge launch but leaves one warp
- * to merge up to 128 rows, so it is slower when a (request, KV head) has many
- * rows and splits (0.85 against 0.30 ms per step with G = 32, D = 256).  Both
- * compute L = ln sum_s exp(L_s), O = sum_s exp(L_s - L) O_s.  Takes effect at
- * the next pa_run.  PA_ERR_INVALID for a NULL plan. */
+ * attention kernel.  1: fused -- the softmax warps of a split item write its
+ * partial state, and the CTA counts itself in a per-(request, KV head)
+ * counter; the CTA that arrives last merges all splits of that (request, KV
+ * head) on its four softmax warps (the fused split reduction with a per-run
+ * counter that "integrate PrimTS FMHA kernels", section "Planning,
+ * preprocessing, and workspace ownership", names; here the scheduler zeroes
+ * the counters every run and no CTA waits for another).  The fused form saves
+ * the merge launch but runs each (request, KV head)'s merge on one CTA after
+ * its last split, so it is slower when few (request, KV head) units carry many
+ * rows and splits (0.34 against 0.28 ms per step with G = 32, D = 256, 16
+ * units).  Both compute L = ln sum_s exp(L_s), O = sum_s exp(L_s - L) O_s.
+ * Takes effect at the next pa_run.  PA_ERR_INVALID for a NULL plan. */
 PA_API int pa_set_fused_merge(pa_plan *plan, int on);
 
 /* Mask mode.  1 (default): causal, aligned to the end of each request's KV

@@ -92,7 +92,7 @@ struct DecCfg {
                        B_OEMPTY = B_PVDONE + 2, B_DRAIN = B_OEMPTY + 1, B_RED = B_DRAIN + 1,
                        B_REDSUM = B_RED + 2, B_STFULL = B_REDSUM + 1, B_STEMPTY = B_STFULL + NST,
                        B_KFULL = B_STEMPTY + NST, B_KEMPTY = B_KFULL + NKB,
-                       NBAR = B_KFULL + (F8 ? 2 * NKB : 0);
+                       B_MERGE = B_KFULL + (F8 ? 2 * NKB : 0), NBAR = B_MERGE + 1;
   static constexpr int BAR_BYTES = F8 ? 384 : 256;
   static constexpr int SMEM_BYTES = 1024 + NSLOT * SLOT_BYTES + NST * STAGE_BYTES +
                                     QBUF * Q_BYTES + 2 * P_BYTES + RED_BYTES + BAR_BYTES;
@@ -621,7 +621,8 @@ __device__ __forceinline__ bool block_reduce_rows(float (&v)[RR], float* red, ui
 template <int D, int NR, int RR, bool F8>
 __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, uint32_t sP,
                                             float* red, uint32_t bar0, uint32_t tmem,
-                                            int n_items, volatile int* abort) {
+                                            int n_items, volatile int* merge_flag,
+                                            volatile int* abort) {
   using C = DecCfg<D, NR, F8>;
   constexpr int BN = C::BN;
   const int t = threadIdx.x;
@@ -654,7 +655,8 @@ __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, u
           else if (p.lse) p.lse[orow0 + r] = -INFINITY;
         }
       }
-      if (split && p.fused_merge) split_arrive_and_merge(p, w, D);
+      if (split && p.fused_merge)
+        split_arrive_and_merge(p, w, D, bar0 + 8 * C::B_MERGE, merge_flag, abort);
       continue;
     }
     float m_run[RR], l_part[RR];
@@ -800,7 +802,8 @@ __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, u
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar0 + 8 * C::B_OEMPTY);
-    if (split && p.fused_merge) split_arrive_and_merge(p, w, D);
+    if (split && p.fused_merge)
+        split_arrive_and_merge(p, w, D, bar0 + 8 * C::B_MERGE, merge_flag, abort);
     ++q_cnt;
   }
 }
@@ -835,9 +838,11 @@ __global__ void __launch_bounds__(DecCfg<D, DecRows<RR>::NR, F8>::THREADS, 1)
   uint8_t* bar_ptr = smem + off_red + C::RED_BYTES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NBAR);
   volatile int* abort = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 4);
+  volatile int* merge_flag = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 8);
 
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
+    mbar_init(bar0 + 8 * C::B_MERGE, kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar0 + 8 * (C::B_QFULL + i), 1);
       mbar_init(bar0 + 8 * (C::B_QEMPTY + i), 1);
@@ -888,7 +893,7 @@ __global__ void __launch_bounds__(DecCfg<D, DecRows<RR>::NR, F8>::THREADS, 1)
     // per-warpgroup register budgets first, then the roles
     if (warp < kSoftmaxWarps) {
       asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
-      dec_softmax<D, NR, RR, F8>(p, sKV, sP, red, bar0, tmem, n_items, abort);
+      dec_softmax<D, NR, RR, F8>(p, sKV, sP, red, bar0, tmem, n_items, merge_flag, abort);
     } else if (warp < C::CONV_WARP0) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::WG1_REGS));
       if (warp == C::PRODUCER_WARP || warp == C::PRODUCER2_WARP)
@@ -911,7 +916,7 @@ __global__ void __launch_bounds__(DecCfg<D, DecRows<RR>::NR, F8>::THREADS, 1)
     } else if (warp == C::MMA_WARP) {
       dec_mma<D, NR>(p, sQ, sKV, sP, bar0, tmem, n_items, abort);
     } else if (warp < kSoftmaxWarps) {
-      dec_softmax<D, NR, RR, F8>(p, sKV, sP, red, bar0, tmem, n_items, abort);
+      dec_softmax<D, NR, RR, F8>(p, sKV, sP, red, bar0, tmem, n_items, merge_flag, abort);
     }
   }
 

@@ -156,12 +156,14 @@ struct TileCfg {
   static constexpr int TMEM_COLS = (O_COL + D <= 256) ? 256 : 512;
   static constexpr int OCH = (CTAS == 2) ? 1 : 2;     // 32-column O chunks per TMEM wait
   // barriers: q_full[QBUF], q_empty[QBUF], kv_full[NSLOT], kv_empty[NSLOT], s_full[2],
-  //           p_full[2], pv_done[2], o_empty, drain, st_full[NST], st_empty[NST]
+  //           p_full[2], pv_done[2], o_empty, drain, st_full[NST], st_empty[NST],
+  //           merge (the softmax warps' fused split-merge hand-shake)
   static constexpr int B_QFULL = 0, B_QEMPTY = QBUF, B_KVFULL = 2 * QBUF,
                        B_KVEMPTY = 2 * QBUF + NSLOT, B_SFULL = 2 * QBUF + 2 * NSLOT,
                        B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2, B_OEMPTY = B_PVDONE + 2,
                        B_DRAIN = B_OEMPTY + 1, B_STFULL = B_DRAIN + 1,
-                       B_STEMPTY = B_STFULL + NST, NBAR = B_STEMPTY + NST;
+                       B_STEMPTY = B_STFULL + NST, B_MERGE = B_STEMPTY + NST,
+                       NBAR = B_MERGE + 1;
   static constexpr int BAR_BYTES = 512;
   // epilogue staging: per softmax warp 32 rows x 32 columns of bf16 (64-byte
   // swizzle); D = 256 has no room for it next to its K/V slots
@@ -259,26 +261,36 @@ __device__ __forceinline__ void merge_one_row(const float* part_o, const float* 
   if (lane == 0 && lse_out) *lse_out = L;
 }
 
-// Fused split-KV reduction.  Called by every softmax warp of a CTA after it
-// wrote its share of a split item's partials (or nothing, for rows it does not
-// own): each warp publishes its writes (__threadfence) and counts itself in
-// the (request, KV head) counter; the warp that brings the count to
-// kSoftmaxWarps * n_splits has every split's partials visible and merges all
-// rows of the item into out and lse.  No warp waits for another.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort);
+
+// Fused split-KV reduction.  Called by all four softmax warps of a CTA after
+// they wrote their share of a split item's partials (or nothing, for rows they
+// do not own).  The CTA, not the warp, counts itself in the (request, KV head)
+// counter: every warp publishes its writes (__threadfence) and arrives on the
+// CTA's merge barrier `mbar` (count 4); once all four have, warp 0 takes a
+// ticket and tells the others through `flag` (a second phase of the same
+// barrier) whether this CTA brought the count to n_splits.  If so, every
+// split's partials are visible and the four warps merge the item's rows
+// between them (row r by warp r % 4).  Each call uses two phases of the
+// barrier (parities 0 and 1); the waits are bounded, so a warp that gave up
+// elsewhere cannot hang the others.  No CTA waits for another CTA.
 __device__ __forceinline__ void split_arrive_and_merge(const AttnParams& p, const WorkItem& w,
-                                                       int D) {
-  const int lane = threadIdx.x & 31;
+                                                       int D, uint32_t mbar, volatile int* flag,
+                                                       volatile int* abort) {
+  const int warp = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
   __threadfence();
   __syncwarp();
-  int last = 0;
-  if (lane == 0)
-    last = atomicAdd(p.split_cnt + (size_t)w.b * p.Hkv + w.kvh, 1) ==
-           kSoftmaxWarps * w.n_splits - 1;
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last) return;
+  if (lane == 0) mbar_arrive(mbar);
+  if (!warp_wait(mbar, 0, abort)) return;
+  if (warp == 0 && lane == 0)
+    *flag = atomicAdd(p.split_cnt + (size_t)w.b * p.Hkv + w.kvh, 1) == w.n_splits - 1;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(mbar);
+  if (!warp_wait(mbar, 1, abort)) return;
+  if (!*flag) return;
   __threadfence();
   const int n_rows = w.n_tok * p.G;
-  for (int r = 0; r < n_rows; ++r) {
+  for (int r = warp; r < n_rows; r += kSoftmaxWarps) {
     const size_t base = ((size_t)w.b * p.Hkv + w.kvh) * p.S_max * kBM + r;
     const size_t orow = (size_t)(w.t_base + w.q_tok0 + r / p.G) * p.Hq + w.kvh * p.G + r % p.G;
     merge_one_row(p.part_o, p.part_lse, base, w.n_splits, D, p.out + orow * D,
@@ -1069,7 +1081,8 @@ __device__ __forceinline__ float write_p(float (&s)[BN], float scale_log2, float
 template <int D, bool F8>
 __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const AttnParams& p,
                                              uint32_t sKV, uint32_t sEpi, uint32_t bar0,
-                                             uint32_t tmem, int n_items, volatile int* abort) {
+                                             uint32_t tmem, int n_items, volatile int* merge_flag,
+                                             volatile int* abort) {
   using C = TileCfg<D, F8>;
   constexpr int BN = C::BN;
   const int r = threadIdx.x;          // query row of the tile, 0..127
@@ -1105,7 +1118,8 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
           if (p.lse) p.lse[(size_t)t * p.Hq + h] = -INFINITY;
         }
       }
-      if (split && p.fused_merge) split_arrive_and_merge(p, w, D);
+      if (split && p.fused_merge)
+        split_arrive_and_merge(p, w, D, bar0 + 8 * C::B_MERGE, merge_flag, abort);
       continue;
     }
     // keys visible to this row: [kv_lo, lim)
@@ -1300,7 +1314,8 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar0 + 8 * C::B_OEMPTY);
-    if (split && p.fused_merge) split_arrive_and_merge(p, w, D);
+    if (split && p.fused_merge)
+        split_arrive_and_merge(p, w, D, bar0 + 8 * C::B_MERGE, merge_flag, abort);
     g_base += n;
     ld_base += 2 * n;
   }
@@ -1326,9 +1341,11 @@ __global__ void __maxnreg__((TileCfg<D, F8>::MAXREG))
   uint8_t* bar_ptr = smem + (bar0 - base);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NBAR);
   volatile int* abort = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 4);
+  volatile int* merge_flag = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NBAR + 8);
 
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
+    mbar_init(bar0 + 8 * C::B_MERGE, kSoftmaxWarps);
     for (int i = 0; i < C::QBUF; ++i) {
       mbar_init(bar0 + 8 * (C::B_QFULL + i), 1);
       mbar_init(bar0 + 8 * (C::B_QEMPTY + i), 1);
@@ -1385,7 +1402,7 @@ __global__ void __maxnreg__((TileCfg<D, F8>::MAXREG))
   } else if (warp == kMmaWarp) {
     mma_role<D, F8>(p, sQ, sKV, bar0, tmem, n_items, abort);   // all 32 lanes
   } else {
-    softmax_role<D, F8>(&tm_o, p, sKV, sEpi, bar0, tmem, n_items, abort);
+    softmax_role<D, F8>(&tm_o, p, sKV, sEpi, bar0, tmem, n_items, merge_flag, abort);
   }
 
   tc_fence_before();
