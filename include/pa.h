@@ -249,16 +249,40 @@ PA_API int pa_selftest_wait_timeout(uint32_t limit_us, uint32_t *status_out,
  * v_pool of the following pa_run calls are uint8 [P, ps, Hkv, D] arrays of
  * E4M3 codes, and attention is computed as if the pools held
  * k_scale * decode(code) and v_scale * decode(code); q stays bf16, out stays
- * bf16, lse is the log-sum-exp of the descaled logits.  The codes are widened
- * to fp16 on chip (exact); q and the softmax weights P are rounded to fp16 for
- * the MMAs (q magnitudes past 65504 saturate).  Decode-only runs (cu_q_lens
- * NULL) use the E4M3 decode kernel; runs with cu_q_lens (prefill, chunked
- * prefill, mixed batches) use the one-stage kernel's E4M3 variant, also when
- * pa_set_two_stage_prefill is on (that kernel reads bf16 pools only).  on = 0
- * restores bf16 pools (descales ignored).  Returns PA_ERR_INVALID for a NULL
- * plan or a descale that is not finite and > 0, PA_ERR_UNSUPPORTED for a
- * head_dim other than 128 or 256. */
+ * bf16, lse is the log-sum-exp of the descaled logits.  Decode-only runs
+ * (cu_q_lens NULL) use the E4M3 decode kernel, which widens the codes to fp16
+ * on chip (exact) and rounds q and the softmax weights P to fp16 for the MMAs
+ * (q magnitudes past 65504 saturate).  Runs with cu_q_lens (prefill, chunked
+ * prefill, mixed batches) take two paths in the same run:
+ *   - a request with two or more query blocks (q_len > 128 / G) reads each
+ *     K/V tile once per block, so its pages are widened once per run into a
+ *     scratch pool of bf16 values (exact: every E4M3 value is a bf16 value)
+ *     and its blocks run on the bf16 one-stage kernel, q in bf16 and P in bf16
+ *     as for bf16 pools (pa_set_kv_fp8_widen sizes the scratch pool);
+ *   - every other request (decode rows, short chunks) runs on the one-stage
+ *     kernel's E4M3 variant, which widens each tile to fp16 on chip with q and
+ *     P in fp16 as above.
+ * Neither path uses the two-stage kernel (pa_set_two_stage_prefill reads bf16
+ * pools only).  on = 0 restores bf16 pools (descales ignored).  Turning the
+ * mode on or off resizes the plan's work-list workspace (synchronous).
+ * Returns PA_ERR_INVALID for a NULL plan or a descale that is not finite and
+ * > 0, PA_ERR_UNSUPPORTED for a head_dim other than 128 or 256, PA_ERR_CUDA
+ * if the workspace cannot be reallocated (the plan is then unchanged). */
 PA_API int pa_set_kv_fp8(pa_plan *plan, int on, float k_scale, float v_scale);
+
+/* Scratch capacity, in pages, for widened E4M3 requests (see pa_set_kv_fp8).
+ * The scratch pool holds bf16 K and V pages [max_pages, ps, Hkv, D] plus a
+ * page table [B, C]; the first pa_run over E4M3 pools with cu_q_lens allocates
+ * it (cudaMalloc; PA_ERR_CUDA from that pa_run if the allocation fails), and
+ * it lives until the plan is destroyed or the capacity changes.  Requests of
+ * two or more query blocks are widened in request order while their pages
+ * (ceil(kv_len / ps) each) fit; the rest run on the E4M3 one-stage kernel, so
+ * every capacity gives the same results within the stated tolerances.
+ * max_pages = -1 (default): every page the batch can hold (B * C), at most
+ * 512 MiB of K and V; 0: never widen; n > 0: n pages (at most B * C).  A new
+ * value frees the current scratch pool (cudaFree synchronises the device).
+ * Returns PA_ERR_INVALID for a NULL plan or max_pages < -1. */
+PA_API int pa_set_kv_fp8_widen(pa_plan *plan, int max_pages);
 
 /* Paged KV append: write this step's new K and V rows into the pools before
  * attention ("integrate PrimTS FMHA kernels", section "Planning,

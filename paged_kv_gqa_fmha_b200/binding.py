@@ -29,7 +29,7 @@ EXPORTS = ("pa_create_plan", "pa_run", "pa_destroy", "pa_last_error", "pa_set_sc
            "pa_max_splits", "pa_profile_start", "pa_profile_read", "pa_run_noalloc",
            "pa_set_two_stage_prefill", "pa_set_decode_kernel", "pa_append_kv",
            "pa_set_causal", "pa_set_page_table_stride", "pa_set_fused_merge", "pa_set_kv_fp8",
-           "pa_selftest_wait_timeout", "pa_noalloc_get_status")
+           "pa_selftest_wait_timeout", "pa_noalloc_get_status", "pa_set_kv_fp8_widen")
 
 # Size of the library's static scratch array used by pa_run_noalloc.
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -91,6 +91,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_set_page_table_stride.restype = I
     lib.pa_set_kv_fp8.argtypes = [P, I, F, F]
     lib.pa_set_kv_fp8.restype = I
+    lib.pa_set_kv_fp8_widen.argtypes = [P, I]
+    lib.pa_set_kv_fp8_widen.restype = I
     lib.pa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.POINTER(ctypes.c_uint32),
                                              ctypes.POINTER(ctypes.c_uint32)]
     lib.pa_selftest_wait_timeout.restype = I
@@ -160,10 +162,16 @@ class Plan:
 
     def set_kv_fp8(self, on: bool, k_scale: float = 1.0, v_scale: float = 1.0):
         """True: the pools of later ``run`` calls are uint8 tensors of E4M3
-        codes, read as ``k_scale * code`` and ``v_scale * code`` (decode only:
-        cu_q_lens must be None).  False: bf16 pools."""
+        codes, read as ``k_scale * code`` and ``v_scale * code`` (decode runs,
+        prefill and mixed batches).  False: bf16 pools."""
         _check(self._lib.pa_set_kv_fp8(self._h, 1 if on else 0, float(k_scale), float(v_scale)))
         self._kv_dtype = torch.uint8 if on else torch.bfloat16
+
+    def set_kv_fp8_widen(self, max_pages: int):
+        """Scratch capacity in pages for E4M3 requests of two or more query
+        blocks, which are widened once per run and read as bf16 pages
+        (-1 automatic, 0 never)."""
+        _check(self._lib.pa_set_kv_fp8_widen(self._h, int(max_pages)))
 
     def set_causal(self, causal: bool):
         """True (default): causal mask aligned to the end of KV; False: every

@@ -20,6 +20,7 @@
 #include "pa_prefill.cuh"
 #include "pa_decode.cuh"
 #include "pa_append.cuh"
+#include "pa_widen.cuh"
 
 namespace {
 
@@ -68,6 +69,7 @@ struct SchedBufs {
   int* unit_off2;
   pa::PackedItem* items2;
   int* split_cnt;             // [B * Hkv] fused-merge counters (plans with splits)
+  int* wpre;                  // [B + 1] first scratch page per widened request (E4M3 pools)
 };
 
 struct pa_plan {
@@ -108,6 +110,16 @@ struct pa_plan {
   int kv_fp8;                  // 1: the pools hold E4M3 codes
   float k_scale, v_scale;      // their per-tensor descales
   int tm_fp8;                  // the pool maps were encoded for E4M3 pools
+  // E4M3 pools: requests with two or more query blocks are widened once per run
+  // into a bf16 scratch pool of widen_cap pages (pa_widen_kernel) and run on
+  // the bf16 one-stage kernel; allocated on the first run that needs it
+  int widen_req;               // -1 automatic capacity (default), 0 never widen, n pages
+  int widen_cap;               // pages of the allocated scratch pool (0: none yet)
+  void* widen_buf;             // K pool, V pool, page table [B, C]
+  void* kw;
+  void* vw;
+  int* spt;
+  CUtensorMap tm_kw, tm_vw;    // the scratch pools, bf16 page boxes of box_h rows
 };
 
 namespace {
@@ -143,11 +155,15 @@ int alloc_workspace(pa_plan* p) {
     return PA_ERR_UNSUPPORTED;
   }
   (void)G;
-  const long max_items2 = p->use_pairs ? (long)p->B * p->Hkv * ((blocks_per_req + 1) / 2) : 0;
+  // second list: query-block pairs (two-stage prefill) or the blocks of widened
+  // requests (E4M3 pools)
+  // (E4M3 pools never use pairs, and their list is the longer one)
+  const long max_items2 = p->kv_fp8 ? (long)p->B * p->Hkv * blocks_per_req
+                          : (p->use_pairs ? (long)p->B * p->Hkv * ((blocks_per_req + 1) / 2) : 0);
   const size_t n_part_rows = p->S_max > 1 ? (size_t)p->B * p->Hkv * p->S_max * pa::kBM : 0;
   size_t off = 0;
   size_t o_hdr[2], o_req[2], o_aux[2], o_uoff[2], o_split[2], o_items[2], o_uoff2[2],
-      o_items2[2], o_cnt[2];
+      o_items2[2], o_cnt[2], o_wpre[2];
   o_hdr[0] = off; off = align_up(off + sizeof(pa::WsHeader), 256);
   o_hdr[1] = off; off = align_up(off + sizeof(pa::WsHeader), 256);
   const size_t zero_bytes = off;   // both headers start zeroed
@@ -161,6 +177,7 @@ int alloc_workspace(pa_plan* p) {
     o_items2[k] = off; off = align_up(off + sizeof(pa::PackedItem) * (size_t)max_items2, 256);
     o_cnt[k] = off;
     off = align_up(off + (p->S_max > 1 ? sizeof(int) * (size_t)p->B * p->Hkv : 0), 256);
+    o_wpre[k] = off; off = align_up(off + sizeof(int) * (size_t)(p->B + 1), 256);
   }
   const size_t o_plse = off; off = align_up(off + sizeof(float) * n_part_rows, 256);
   const size_t o_po = off; off = align_up(off + sizeof(float) * n_part_rows * p->D, 256);
@@ -191,6 +208,7 @@ int alloc_workspace(pa_plan* p) {
     b.unit_off2 = reinterpret_cast<int*>(c + o_uoff2[k]);
     b.items2 = reinterpret_cast<pa::PackedItem*>(c + o_items2[k]);
     b.split_cnt = p->S_max > 1 ? reinterpret_cast<int*>(c + o_cnt[k]) : nullptr;
+    b.wpre = reinterpret_cast<int*>(c + o_wpre[k]);
   }
   p->hdr = p->sb[0].hdr;
   p->run_par = 0;
@@ -471,6 +489,70 @@ int build_maps(pa_plan* p, const void* q, const void* k, const void* v, void* ou
 
 bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
 
+// Automatic scratch capacity for widened E4M3 requests: every page the batch
+// can hold, up to 512 MiB of bf16 K and V.
+constexpr size_t kWidenAutoBytes = size_t(512) << 20;
+
+void free_widen(pa_plan* p) {
+  if (p->widen_buf) cudaFree(p->widen_buf);
+  p->widen_buf = p->kw = p->vw = nullptr;
+  p->spt = nullptr;
+  p->widen_cap = 0;
+}
+
+// Allocate the scratch pools and page table of widened requests and encode
+// their tensor maps ([cap, ps, Hkv, D] bf16, the bf16 pools' page boxes).
+int alloc_widen(pa_plan* p) {
+  const size_t part = (size_t)p->ps * p->Hkv * p->D * 2;   // bytes of one bf16 page part
+  const long all = (long)p->B * p->C;
+  long cap = p->widen_req > 0 ? p->widen_req : (long)(kWidenAutoBytes / (2 * part));
+  if (cap > all) cap = all;
+  if (cap < 1) cap = 1;
+  const size_t o_v = align_up(part * (size_t)cap, 256);
+  const size_t o_t = o_v + align_up(part * (size_t)cap, 256);
+  const size_t bytes = o_t + sizeof(int) * (size_t)all;
+  void* buf = nullptr;
+  cudaError_t e = cudaMalloc(&buf, bytes);
+  if (e != cudaSuccess) {
+    set_err("pa_run: cudaMalloc of %zu bytes for the widened E4M3 pages failed: %s "
+            "(pa_set_kv_fp8_widen sets a smaller capacity, or 0 for none)",
+            bytes, cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  free_widen(p);
+  p->widen_buf = buf;
+  p->kw = buf;
+  p->vw = static_cast<char*>(buf) + o_v;
+  p->spt = reinterpret_cast<int*>(static_cast<char*>(buf) + o_t);
+  const cuuint64_t e2 = 2;
+  cuuint64_t dims[4] = {(cuuint64_t)p->D, (cuuint64_t)p->Hkv, (cuuint64_t)p->ps, (cuuint64_t)cap};
+  cuuint64_t str[3] = {(cuuint64_t)p->D * e2, (cuuint64_t)p->Hkv * p->D * e2,
+                       (cuuint64_t)p->ps * p->Hkv * p->D * e2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)p->box_h, 1};
+  int rc = encode(&p->tm_kw, p->kw, 4, dims, str, box, "widened k");
+  if (rc == PA_OK) rc = encode(&p->tm_vw, p->vw, 4, dims, str, box, "widened v");
+  if (rc != PA_OK) {
+    free_widen(p);
+    return rc;
+  }
+  p->widen_cap = (int)cap;
+  return PA_OK;
+}
+
+cudaError_t launch_widen(int n_sm, cudaStream_t st, const pa::WidenParams& wp) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(4 * n_sm);
+  cfg.blockDim = dim3(pa::kWidenThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pa::pa_widen_kernel, wp);
+}
+
 }  // namespace
 
 extern "C" {
@@ -558,6 +640,10 @@ pa_plan* pa_create_plan(int batch, int heads_q, int heads_kv, int head_dim, int 
   p->k_scale = p->v_scale = 1.0f;
   p->tm_fp8 = 0;
   p->tm_num_pages = -1;
+  p->widen_req = -1;
+  p->widen_cap = 0;
+  p->widen_buf = p->kw = p->vw = nullptr;
+  p->spt = nullptr;
   if (alloc_workspace(p) != PA_OK) {
     delete p;
     return nullptr;
@@ -577,6 +663,7 @@ static void free_profile_events(pa_plan* p) {
 void pa_destroy(pa_plan* p) {
   if (!p) return;
   free_profile_events(p);
+  free_widen(p);
   if (p->ws) cudaFree(p->ws);
   delete p;
 }
@@ -659,7 +746,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
 
   // this run's set of scheduler outputs (the previous run may still read the other)
   const SchedBufs& bufs = p->sb[p->run_par & 1u];
-  pa::SchedParams sp;
+  pa::SchedParams sp = {};
   sp.seq_lens = seq_lens;
   sp.cu_q_lens = cu_q_lens;
   sp.items = bufs.items;
@@ -670,7 +757,16 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   // without cu_q_lens every request is one decode token: no query-block pairs;
   // the two-stage kernel reads bf16 pools only, so E4M3 pools skip it too
   const bool pairs = p->use_pairs && cu_q_lens != nullptr && !p->kv_fp8;
-  sp.items2 = pairs ? bufs.items2 : nullptr;
+  // E4M3 pools with query blocks: requests of two or more blocks are widened
+  // once (pa_widen_kernel) and run on the bf16 kernel from the second list
+  const bool wide = p->kv_fp8 && cu_q_lens != nullptr && p->widen_req != 0;
+  if (wide && p->widen_buf == nullptr) {
+    rc = alloc_widen(p);
+    if (rc) return rc;
+  }
+  sp.items2 = (pairs || wide) ? bufs.items2 : nullptr;
+  sp.wide_cap = wide ? p->widen_cap : 0;
+  sp.wpre = bufs.wpre;
   sp.unit_off2 = bufs.unit_off2;
   sp.max_items2 = p->max_items2;
   sp.hdr = bufs.hdr;
@@ -728,6 +824,32 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     le = p->D == 64 ? launch_pairs<64>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, p->tm_o, ap2)
                     : launch_pairs<128>(p->n_sm, st, p->tm_q, p->tm_k2, p->tm_v2, p->tm_o, ap2);
   }
+  if (le == cudaSuccess && wide) {
+    // widen the chosen requests' pages, then run their blocks over the
+    // scratch pools as a bf16 batch (descales still in scale_log2 and v_scale)
+    pa::WidenParams wp;
+    wp.k8 = static_cast<const uint4*>(k_pool);
+    wp.v8 = static_cast<const uint4*>(v_pool);
+    wp.k16 = static_cast<uint4*>(p->kw);
+    wp.v16 = static_cast<uint4*>(p->vw);
+    wp.spt = p->spt;
+    wp.page_table = page_table;
+    wp.wpre = bufs.wpre;
+    wp.hdr = bufs.hdr;
+    wp.status = &p->hdr->status;
+    wp.B = p->B; wp.C = p->C; wp.tstride = p->tstride; wp.num_pages = p->num_pages;
+    wp.part_u4 = p->ps * p->Hkv * p->D / 16;
+    le = launch_widen(p->n_sm, st, wp);
+    if (le == cudaSuccess) {
+      pa::AttnParams aw = ap;
+      aw.items = bufs.items2;
+      aw.list2 = 1;
+      aw.page_table = p->spt;
+      aw.tstride = p->C;
+      aw.num_pages = p->widen_cap;
+      le = launch_attention_d(p->D, false, p->n_sm, st, p->tm_q, p->tm_kw, p->tm_vw, p->tm_o, aw);
+    }
+  }
   if (le == cudaSuccess)
     le = dec ? launch_decode(p->D, p->G, p->kv_fp8 != 0, p->n_sm, st, p->tm_k, p->tm_v, ap)
              : launch_attention_d(p->D, p->kv_fp8 != 0, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v,
@@ -752,7 +874,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     set_err("pa_run: launch failed: %s", cudaGetErrorString(le));
     return PA_ERR_CUDA;
   }
-  p->last_launches = 2 + (pairs ? 1 : 0) + (sp.S_max > 1 && !fused ? 1 : 0);
+  p->last_launches = 2 + (pairs ? 1 : 0) + (wide ? 2 : 0) + (sp.S_max > 1 && !fused ? 1 : 0);
   p->run_par ^= 1u;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -865,7 +987,11 @@ int pa_selftest_wait_timeout(uint32_t limit_us, uint32_t* status_out,
 int pa_set_kv_fp8(pa_plan* p, int on, float k_scale, float v_scale) {
   if (!p) { set_err("pa_set_kv_fp8: NULL plan"); return PA_ERR_INVALID; }
   if (!on) {
-    p->kv_fp8 = 0;
+    if (p->kv_fp8) {
+      p->kv_fp8 = 0;
+      int rc = alloc_workspace(p);   // the second list shrinks back
+      if (rc != PA_OK) { p->kv_fp8 = 1; return rc; }
+    }
     p->k_scale = p->v_scale = 1.0f;
     return PA_OK;
   }
@@ -878,9 +1004,26 @@ int pa_set_kv_fp8(pa_plan* p, int on, float k_scale, float v_scale) {
     set_err("pa_set_kv_fp8: head_dim %d has no E4M3 kernels (128 and 256 only)", p->D);
     return PA_ERR_UNSUPPORTED;
   }
-  p->kv_fp8 = 1;
+  if (!p->kv_fp8) {
+    p->kv_fp8 = 1;
+    int rc = alloc_workspace(p);     // room for the blocks of widened requests
+    if (rc != PA_OK) { p->kv_fp8 = 0; return rc; }
+  }
   p->k_scale = k_scale;
   p->v_scale = v_scale;
+  return PA_OK;
+}
+
+int pa_set_kv_fp8_widen(pa_plan* p, int max_pages) {
+  if (!p) { set_err("pa_set_kv_fp8_widen: NULL plan"); return PA_ERR_INVALID; }
+  if (max_pages < -1) {
+    set_err("pa_set_kv_fp8_widen: max_pages %d (use -1, 0 or a page count)", max_pages);
+    return PA_ERR_INVALID;
+  }
+  if (max_pages != p->widen_req) {
+    free_widen(p);     // the next run that needs it allocates the new capacity
+    p->widen_req = max_pages;
+  }
   return PA_OK;
 }
 
@@ -1141,7 +1284,7 @@ int pa_run_noalloc(int batch, int heads_q, int heads_kv, int head_dim, int page_
     return PA_ERR_CUDA;
   }
 
-  pa::SchedParams sp;
+  pa::SchedParams sp = {};
   sp.seq_lens = seq_lens;
   sp.cu_q_lens = cu_q_lens;
   sp.items = reinterpret_cast<pa::PackedItem*>(base + o_items);

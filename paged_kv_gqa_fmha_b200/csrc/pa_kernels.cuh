@@ -102,8 +102,9 @@ struct WsHeader {
   unsigned status;
   int n_items;
   int n_split_reqs;   // requests split over KV (entries of the split list)
-  int n_items2;       // items of the query-block-pair list (two-stage prefill kernel)
-  int pad[60];
+  int n_items2;       // items of the second list (query-block pairs, or widened requests)
+  int n_wide_pages;   // pages of the widened requests (E4M3 pools, second list)
+  int pad[59];
 };
 
 constexpr int kBM = 128;              // query rows per tile (tcgen05 M)
@@ -197,6 +198,7 @@ struct AttnParams {
   int fused_merge;            // 1: the last split warp of a (request, KV head) merges
   float scale_log2;           // softmax scale * log2(e) (times the K descale for E4M3 pools)
   float v_scale;              // V descale of E4M3 pools (1 for bf16 pools)
+  int list2;                  // 1: items is the second list (its count is hdr->n_items2)
 };
 
 constexpr int kSoftmaxWarps = 4;      // softmax warps per CTA in every attention kernel
@@ -342,9 +344,16 @@ struct SchedParams {
   const int* seq_lens;
   const int* cu_q_lens;
   PackedItem* items;
-  PackedItem* items2;  // pairs of query blocks, or nullptr when pairs are not used
-  int* unit_off2;      // [B + 1] exclusive prefix sum of pair units
+  PackedItem* items2;  // second list (pairs or widened requests), or nullptr
+  int* unit_off2;      // [B + 1] exclusive prefix sum of second-list units
   int max_items2;
+  // E4M3 pools: requests with two or more query blocks are widened once into a
+  // 16-bit scratch pool of wide_cap pages, in request order while they fit,
+  // and their blocks go to the second list (one unit per block).  wide_cap = 0:
+  // no widening.  wpre[b] = first scratch page of request b ([B + 1] entries,
+  // non-decreasing; requests that are not widened own no pages).
+  int wide_cap;
+  int* wpre;
   int* split_list;     // [B] requests with more than one split
   int4* req_info;      // [B] {n_splits, q_len, t_base, kv_len}
   int4* req_aux;       // [B] {units, tiles per split, KV tiles of the single block, 0}
@@ -518,21 +527,33 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
   __syncthreads();
   const int chunk = s_chunk;
 
-  // 2.  A request with two or more query blocks goes to the pair list when the
-  // two-stage prefill kernel is in use (items2 != nullptr): one unit per pair of
-  // consecutive blocks.  Every other request goes to the main list.
+  // 2.  A request with two or more query blocks goes to the second list when
+  // items2 != nullptr: with the two-stage prefill kernel one unit per pair of
+  // consecutive blocks; with E4M3 pools (wide_cap > 0) one unit per block, if
+  // its pages still fit the scratch pool (the request is then widened once
+  // and read as 16-bit tiles).  Every other request goes to the main list.
   __shared__ int s_nsplit;
+  __shared__ int s_wide_pages;
   __shared__ int s_uoff[kSchedSmemReqs + 1];
   __shared__ int s_uoff2[kSchedSmemReqs + 1];
-  if (tid == 0) s_nsplit = 0;
+  if (tid == 0) { s_nsplit = 0; s_wide_pages = 0; }
   __syncthreads();
-  int running = 0, running2 = 0;
+  const bool wide_mode = p.items2 != nullptr && p.wide_cap > 0;
+  int running = 0, running2 = 0, running_pg = 0;
   for (int b0 = 0; b0 < p.B; b0 += blockDim.x) {
     const int b = b0 + tid;
-    int units = 0, units2 = 0;
+    int units = 0, units2 = 0, pages = 0, nb = 0;
+    ReqInfo r = {0, 0, 0, 0u};
     if (b < p.B) {
-      const ReqInfo r = read_request(p, b);
-      const int nb = n_qblocks(r.q_len, p.tpb);
+      r = read_request(p, b);
+      nb = n_qblocks(r.q_len, p.tpb);
+      if (wide_mode && nb >= 2) pages = ceil_div(r.kv_len, p.ps);
+    }
+    // scratch pages: the candidates' exclusive prefix, in request order
+    int total_pg;
+    const int pg0 = running_pg + block_scan_1024(pages, warp_sums, &total_pg);
+    const bool wide = pages > 0 && pg0 + pages <= p.wide_cap;
+    if (b < p.B) {
       const int tiles = ceil_div(block_kv_hi(r.q_len, r.kv_len, 0, r.q_len, p.causal), p.BN);
       int ns = 1, per = tiles > 0 ? tiles : 1;
       if (nb == 1 && p.S_max > 1 && tiles > 1) {
@@ -542,12 +563,16 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
         per = ceil_div(tiles, sp);
         ns = ceil_div(tiles, per);
       }
-      if (p.items2 != nullptr && ns == 1 && nb >= 2) units2 = (nb + 1) / 2;
+      if (wide) units2 = nb;
+      else if (!wide_mode && p.items2 != nullptr && ns == 1 && nb >= 2) units2 = (nb + 1) / 2;
       else units = ns > 1 ? ns : nb;
       p.req_info[b] = make_int4(ns, r.q_len, r.t_base, r.kv_len);
       p.req_aux[b] = make_int4(units, per, tiles, 0);
       if (ns > 1) p.split_list[atomicAdd(&s_nsplit, 1)] = b;
+      if (wide_mode) p.wpre[b] = pg0;
+      if (wide) atomicMax(&s_wide_pages, pg0 + pages);
     }
+    running_pg += total_pg;
     int total, total2;
     const int off = block_scan_1024(units, warp_sums, &total);
     const int off2 = block_scan_1024(units2, warp_sums, &total2);
@@ -572,6 +597,8 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
     p.hdr->n_split_reqs = s_nsplit;
     const int n2 = running2 * p.Hkv;
     p.hdr->n_items2 = n2 < p.max_items2 ? n2 : p.max_items2;
+    p.hdr->n_wide_pages = s_wide_pages;
+    if (wide_mode) p.wpre[p.B] = running_pg;
   }
   __syncthreads();
   const int U = running;
@@ -579,8 +606,10 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
   const int U2 = running2;
   const int* uoff2 = p.B <= kSchedSmemReqs ? s_uoff2 : p.unit_off2;
 
-  // 2b.  Pair list: each request's pairs stay together, last pair (most keys)
-  // first; a unit writes its Hkv items (one per KV head) at consecutive places.
+  // 2b.  Second list: each request's units (pairs, or single blocks of a
+  // widened request) stay together, last unit (most keys) first; a unit writes
+  // its Hkv items (one per KV head) at consecutive places.
+  const int bpu = wide_mode ? 1 : 2;   // query blocks per unit
   for (int u0 = 0; u0 < U2; u0 += blockDim.x) {
     const int u = u0 + tid;
     if (u < U2) {
@@ -593,9 +622,9 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
       const int4 ri = p.req_info[b];
       const int k = u - uoff2[b];
       const int units2 = uoff2[b + 1] - uoff2[b];
-      const int pair = units2 - 1 - k;
-      const int q0 = 2 * pair * p.tpb;
-      const int ntok = min(2 * p.tpb, ri.y - q0);
+      const int unit = units2 - 1 - k;
+      const int q0 = bpu * unit * p.tpb;
+      const int ntok = min(bpu * p.tpb, ri.y - q0);
       const int hi_kv = block_kv_hi(ri.y, ri.w, q0, ntok, p.causal);
       const int pos = u * p.Hkv;
       for (int g = 0; g < p.Hkv; ++g) {
@@ -1385,7 +1414,7 @@ __global__ void __maxnreg__((TileCfg<D, F8>::MAXREG))
   // everything above overlaps the scheduler kernel; its work list is read below
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int n_items = p.hdr->n_items;
+  const int n_items = p.list2 ? p.hdr->n_items2 : p.hdr->n_items;
 
   if (warp == kProducerWarp || warp == kProducer2Warp) {
     if constexpr (F8) {

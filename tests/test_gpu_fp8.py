@@ -235,3 +235,71 @@ def test_fp8_full_size_prefill_and_mixed_every_element(name):
     err_o, err_l = compare(out, lse, o_ref, l_ref)
     print("%s/fp8: %d elements, max|O-oracle| %.3e, max|LSE-oracle| %.3e"
           % (name, out.numel(), err_o, err_l))
+
+
+# q_lens / kv_lens of a batch with three multi-block requests (G = 4: 32 tokens
+# per block) and two decode rows; page size 16, so the multi-block requests
+# own 19, 32 and 10 pages
+WIDE_Q = [300, 1, 200, 150, 1]
+WIDE_KV = [300, 900, 500, 150, 2000]
+
+
+@pytest.mark.parametrize("max_pages,launches", [(-1, 4), (0, 2), (19, 4), (20, 4), (61, 4)])
+def test_fp8_widened_requests_match_oracle(max_pages, launches):
+    """Requests of two or more query blocks over E4M3 pools are widened once
+    into the bf16 scratch pool (in request order while their pages fit) and
+    run on the bf16 kernel; the rest stay on the E4M3 one-stage kernel.  Every
+    capacity -- all widened (-1, 61), none (0), only the first request (19:
+    its pages exactly; 20: one spare page, the next request does not fit) --
+    matches the oracle, and the run enqueues the widening pass and the bf16
+    launch only when the capacity is not 0."""
+    spec = W.custom_spec("fp8_wide", 16, 4, 128, 16, WIDE_Q, WIDE_KV)
+    w, k8, v8 = _fp8_workload(spec, 47)
+    o_ref, l_ref = _oracle(w, k8, v8)
+    plan = _plan(w, num_splits=1)
+    plan.set_kv_fp8_widen(max_pages)
+    for _ in range(2):      # the second run reuses the scratch pool
+        plan.profile_start(1)
+        out, lse = _run(plan, w, k8, v8, use_cu=True)
+        _, n, per_run = plan.profile_read()
+        assert n == 1 and per_run == launches
+        compare(out, lse, o_ref, l_ref)
+
+
+def test_fp8_widen_paths_agree_and_d256():
+    """head_dim 256 over E4M3 pools with and without widening: both match the
+    oracle (the two paths round q and P differently, so they agree only
+    within the tolerances)."""
+    spec = W.custom_spec("fp8_wide256", 8, 2, 256, 32, [70, 1, 9], [300, 400, 9])
+    w, k8, v8 = _fp8_workload(spec, 53)
+    o_ref, l_ref = _oracle(w, k8, v8)
+    for max_pages in (-1, 0):
+        plan = _plan(w)
+        plan.set_kv_fp8_widen(max_pages)
+        out, lse = _run(plan, w, k8, v8, use_cu=True)
+        compare(out, lse, o_ref, l_ref)
+
+
+def test_fp8_widened_bad_page_is_reported():
+    """A page id outside [0, num_pages) inside a widened request's pages is
+    reported as PA_STATUS_BAD_PAGE (the page reads as zeros), and the plan
+    keeps working: the next run with a valid table matches the oracle."""
+    spec = W.custom_spec("fp8_wide_bad", 16, 4, 128, 16, WIDE_Q, WIDE_KV)
+    w, k8, v8 = _fp8_workload(spec, 59)
+    plan = _plan(w)
+    bad = w["page_table"].clone()
+    bad[0, 3] = w["P"] + 5
+    plan.run(w["q"], k8, v8, bad, w["seq_lens"], w["cu_q_lens"])
+    torch.cuda.synchronize()
+    assert plan.status() & binding.STATUS_BAD_PAGE
+    out, lse = _run(plan, w, k8, v8, use_cu=True)
+    compare(out, lse, *_oracle(w, k8, v8))
+
+
+def test_fp8_widen_rejects_bad_capacity():
+    spec = W.custom_spec("fp8_wide_rej", 8, 2, 128, 16, [40], [40])
+    w, _, _ = _fp8_workload(spec, 61)
+    plan = _plan(w)
+    with pytest.raises(binding.PAError) as e:
+        plan.set_kv_fp8_widen(-2)
+    assert e.value.code == binding.PA_ERR_INVALID
