@@ -593,8 +593,12 @@ def to_fp8_pools(w):
 def kv_fp8_rates(bw, tf):
     """Every non-tiny workload over E4M3 pools (pa_set_kv_fp8): the bf16 pools
     are quantised on the device (x4, round to nearest E4M3) and read back with
-    descales 0.25.  Decode-only workloads run on the E4M3 decode kernel,
-    prefill and mixed batches on the one-stage kernel's E4M3 variant.  Bytes
+    descales 0.25.  Decode-only workloads run on the kernel a default plan
+    picks (the E4M3 decode kernel at head_dim 128, the one-stage kernel's E4M3
+    variant at 256); in prefill and mixed batches the requests of two or more
+    query blocks are widened once into bf16 scratch pages (pa_widen_kernel)
+    and run on the bf16 one-stage kernel, the rest on its E4M3 variant; the
+    time covers all of these launches.  Bytes
     per launch = the bf16 formula with K and V at one byte per element;
     per-launch CUDA events (the plan's profile pairs) over 20 launches, each
     synchronised, after 5 warm-up launches (pools larger than L2)."""
@@ -622,8 +626,12 @@ def kv_fp8_rates(bw, tf):
         gbs = nbytes / (ms * 1e-3) / 1e9
         tfs = c["flops"] / (ms * 1e-3) / 1e12
         G = w["Hq"] // w["Hkv"]
-        kernel = ("pa_decode_kernel<%d, %d, true>" % (w["D"], max(4, 1 << (G - 1).bit_length()))
-                  if spec.decode_only else "pa_attention_kernel<%d, true>" % w["D"])
+        if spec.decode_only:
+            kernel = ("pa_decode_kernel<%d, %d, true>" % (w["D"], max(4, 1 << (G - 1).bit_length()))
+                      if w["D"] == 128 else "pa_attention_kernel<%d, true>" % w["D"])
+        else:
+            kernel = ("pa_widen_kernel + pa_attention_kernel<{0}, false> (widened requests) + "
+                      "pa_attention_kernel<{0}, true>".format(w["D"]))
         out[name] = {"attn_kernel_ms": ms, "algorithmic_bytes": nbytes, "flops": c["flops"],
                      "kernel_GBps": gbs, "kernel_TFLOPs": tfs, "hbm_frac": gbs / bw,
                      "tensor_frac": tfs / tf, "status_word": plan.status(), "kernel": kernel}

@@ -221,8 +221,8 @@ PA_API int pa_set_page_table_stride(pa_plan *plan, int row_stride);
  * S^T = K Q^T and O^T = V^T P^T with the 128 keys of a tile as the MMA's M
  * dimension and the G query rows (padded to 16 or 32) as N -- the same online
  * softmax ("FlashAttention", Dao et al., Algorithm 1) with 1/8 to 1/4 of the
- * tensor work of 128-row query tiles.  Default: head_dim 128 runs on it,
- * head_dim 256 on the one-stage kernel.  on = 1: head_dim 128 and 256 run on
+ * tensor work of 128-row query tiles.  Default (bf16 and E4M3 pools alike):
+ * head_dim 128 runs on it, head_dim 256 on the one-stage kernel.  on = 1: head_dim 128 and 256 run on
  * it.  on = 0: every such run uses the one-stage kernel.  The two paths agree
  * within the stated tolerances, not bit for bit.  Takes effect at the next
  * pa_run; no reallocation.  PA_ERR_INVALID for a NULL plan. */
@@ -250,9 +250,10 @@ PA_API int pa_selftest_wait_timeout(uint32_t limit_us, uint32_t *status_out,
  * E4M3 codes, and attention is computed as if the pools held
  * k_scale * decode(code) and v_scale * decode(code); q stays bf16, out stays
  * bf16, lse is the log-sum-exp of the descaled logits.  Decode-only runs
- * (cu_q_lens NULL) use the E4M3 decode kernel, which widens the codes to fp16
- * on chip (exact) and rounds q and the softmax weights P to fp16 for the MMAs
- * (q magnitudes past 65504 saturate).  Runs with cu_q_lens (prefill, chunked
+ * (cu_q_lens NULL) pick their kernel as for bf16 pools (pa_set_decode_kernel):
+ * the E4M3 decode kernel, or the one-stage kernel's E4M3 variant; both widen
+ * the codes to fp16 on chip (exact) and round q and the softmax weights P to
+ * fp16 for the MMAs (q magnitudes past 65504 saturate).  Runs with cu_q_lens (prefill, chunked
  * prefill, mixed batches) take two paths in the same run:
  *   - a request with two or more query blocks (q_len > 128 / G) reads each
  *     K/V tile once per block, so its pages are widened once per run into a

@@ -780,11 +780,10 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   sp.split_cnt = fused ? bufs.split_cnt : nullptr;
   sp.forced_splits = p->num_splits > 1 ? p->num_splits : 0;
   // decode-only runs (one query token per request) with up to 32 query heads
-  // per KV head go to the keys-as-M decode kernel (one CTA per SM)
-  // (E4M3 pools always take it: pa_set_kv_fp8 checked head_dim)
+  // per KV head go to the keys-as-M decode kernel (one CTA per SM): by default
+  // at head_dim 128, on request at 256 too; the same rule for E4M3 pools
   const bool dec = cu_q_lens == nullptr && p->G <= 32 &&
-                   (p->kv_fp8 || (p->use_dec == -1 && p->D == 128) ||
-                    (p->use_dec == 1 && p->D >= 128));
+                   ((p->use_dec == -1 && p->D == 128) || (p->use_dec == 1 && p->D >= 128));
   sp.n_ctas = dec ? p->n_sm : attn_grid(p->D, p->n_sm);
   cudaError_t le = launch_schedule(st, sp);
 

@@ -81,12 +81,19 @@ GEOMS = [  # seed, D, G, ps, Hkv, B, max_kv
 ]
 
 
+@pytest.mark.parametrize("other_kernel", [False, True])
 @pytest.mark.parametrize("seed,D,G,ps,Hkv,B,max_kv", GEOMS)
-def test_fp8_decode_matches_oracle(seed, D, G, ps, Hkv, B, max_kv):
+def test_fp8_decode_matches_oracle(seed, D, G, ps, Hkv, B, max_kv, other_kernel):
+    """Decode-only runs over E4M3 pools on the default kernel (the decode
+    kernel at head_dim 128, the one-stage kernel at 256) and on the other one
+    (pa_set_decode_kernel)."""
     rng = np.random.default_rng(seed)
     spec = W.random_small(rng, D=D, ps=ps, G=G, Hkv=Hkv, B=B, max_kv=max_kv, prefill=False)
     w, k8, v8 = _fp8_workload(spec, 500 + seed)
-    out, lse = _run(_plan(w), w, k8, v8)
+    plan = _plan(w)
+    if other_kernel:
+        plan.set_decode_kernel(D == 256)
+    out, lse = _run(plan, w, k8, v8)
     o_ref, l_ref = _oracle(w, k8, v8)
     compare(out, lse, o_ref, l_ref)
 
