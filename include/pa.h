@@ -125,9 +125,14 @@ PA_API pa_plan *pa_create_plan(int batch, int heads_q, int heads_kv, int head_di
  * the request's KV; decode sees every key).  Query head h reads KV head
  * h / G.  All pointers must be 16-byte aligned.
  *
- * Enqueues at most four kernels (scheduler, two-stage prefill when enabled,
- * attention, split merge); does not allocate, does not synchronise and reads
- * no device data on the host, so it can be captured in a CUDA graph.  The
+ * Enqueues at most five kernels (scheduler; the two-stage prefill kernel when
+ * enabled, or with E4M3 pools and cu_q_lens the widening pass and the bf16
+ * attention kernel over the widened requests; attention; split merge); does
+ * not synchronise and reads no device data on the host, so it can be captured
+ * in a CUDA graph.  It does not allocate, with one exception: the first run
+ * over E4M3 pools with cu_q_lens allocates the widening scratch pool
+ * (pa_set_kv_fp8_widen), so such a run must happen once before capture (or
+ * the capacity be set to 0).  The
  * scheduler may start while the previous pa_run on the same plan and stream
  * is still finishing (it writes the other of two work-list buffers) and ends
  * only after that run, so consecutive runs keep stream order.  Returns PA_OK, PA_ERR_INVALID
@@ -265,7 +270,8 @@ PA_API int pa_selftest_wait_timeout(uint32_t limit_us, uint32_t *status_out,
  *     P in fp16 as above.
  * Neither path uses the two-stage kernel (pa_set_two_stage_prefill reads bf16
  * pools only).  on = 0 restores bf16 pools (descales ignored).  Turning the
- * mode on or off resizes the plan's work-list workspace (synchronous).
+ * mode on or off resizes the plan's work-list workspace (synchronous; call it
+ * outside graph capture).
  * Returns PA_ERR_INVALID for a NULL plan or a descale that is not finite and
  * > 0, PA_ERR_UNSUPPORTED for a head_dim other than 128 or 256, PA_ERR_CUDA
  * if the workspace cannot be reallocated (the plan is then unchanged). */
