@@ -344,7 +344,7 @@ cudaError_t launch_attention(int n_sm, cudaStream_t st, const CUtensorMap& tq,
                              const CUtensorMap& to, const pa::AttnParams& ap) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pa::TileCfg<D, F8>::CTAS * n_sm);
-  cfg.blockDim = dim3(pa::kThreads);
+  cfg.blockDim = dim3(pa::TileCfg<D, F8>::THREADS);
   cfg.dynamicSmemBytes = pa::TileCfg<D, F8>::SMEM_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -782,8 +782,16 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   // decode-only runs (one query token per request) with up to 32 query heads
   // per KV head go to the keys-as-M decode kernel (one CTA per SM): by default
   // at head_dim 128, on request at 256 too; the same rule for E4M3 pools
-  const bool dec = cu_q_lens == nullptr && p->G <= 32 &&
-                   ((p->use_dec == -1 && p->D == 128) || (p->use_dec == 1 && p->D >= 128));
+  const bool dec_shape = p->G <= 32 &&
+                         ((p->use_dec == -1 && p->D == 128) || (p->use_dec == 1 && p->D >= 128));
+  const bool dec = cu_q_lens == nullptr && dec_shape;
+  // E4M3 pools with cu_q_lens: rows of one query token (the decode rows of a
+  // mixed batch) run on the E4M3 decode kernel from a second segment of the
+  // main list; on the one-stage kernel each would widen its tiles through one
+  // warp (bf16 pools keep one launch: there the one-stage kernel overlaps the
+  // decode rows' HBM streaming with the prefill blocks' tensor work)
+  const bool dec_seg = p->kv_fp8 && cu_q_lens != nullptr && dec_shape;
+  sp.split_decode = dec_seg ? 1 : 0;
   sp.n_ctas = dec ? p->n_sm : attn_grid(p->D, p->n_sm);
   cudaError_t le = launch_schedule(st, sp);
 
@@ -842,7 +850,7 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     if (le == cudaSuccess) {
       pa::AttnParams aw = ap;
       aw.items = bufs.items2;
-      aw.list2 = 1;
+      aw.list = 1;
       aw.page_table = p->spt;
       aw.tstride = p->C;
       aw.num_pages = p->widen_cap;
@@ -853,6 +861,11 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     le = dec ? launch_decode(p->D, p->G, p->kv_fp8 != 0, p->n_sm, st, p->tm_k, p->tm_v, ap)
              : launch_attention_d(p->D, p->kv_fp8 != 0, p->n_sm, st, p->tm_q, p->tm_k, p->tm_v,
                                   p->tm_o, ap);
+  if (le == cudaSuccess && dec_seg) {
+    pa::AttnParams ad = ap;
+    ad.list = 2;
+    le = launch_decode(p->D, p->G, true, p->n_sm, st, p->tm_k, p->tm_v, ad);
+  }
   if (prof) {
     cudaEventRecord(p->prof_ev[2 * p->prof_n + 1], st);
     ++p->prof_n;
@@ -873,7 +886,8 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
     set_err("pa_run: launch failed: %s", cudaGetErrorString(le));
     return PA_ERR_CUDA;
   }
-  p->last_launches = 2 + (pairs ? 1 : 0) + (wide ? 2 : 0) + (sp.S_max > 1 && !fused ? 1 : 0);
+  p->last_launches = 2 + (pairs ? 1 : 0) + (wide ? 2 : 0) + (dec_seg ? 1 : 0) +
+                     (sp.S_max > 1 && !fused ? 1 : 0);
   p->run_par ^= 1u;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

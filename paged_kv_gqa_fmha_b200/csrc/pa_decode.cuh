@@ -111,7 +111,7 @@ __device__ __forceinline__ void dec_q_loader(const AttnParams& p, uint32_t sQ, u
   const int lane = threadIdx.x & 31;
   const int G = p.G;
   uint32_t q_cnt = 0;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (items.next(w)) {
     if (w.kv_hi <= w.kv_lo) continue;
@@ -181,7 +181,7 @@ __device__ __forceinline__ void dec_producer(const CUtensorMap* tm_k, const CUte
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = item_tiles(w, C::BN);
@@ -252,7 +252,7 @@ __device__ __forceinline__ void dec_convert(const AttnParams& p, uint32_t sKV, u
   const uint32_t tl = tmem + (static_cast<uint32_t>((ct >> 5) * 32) << 16);
   uint32_t ld_idx = 0, g = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = item_tiles(w, C::BN);
@@ -403,7 +403,7 @@ __device__ __forceinline__ void dec_mma(const AttnParams& p, uint32_t sQ, uint32
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, NR, true, false);
   uint32_t ld_idx = 0, g = 0, q_cnt = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
 
   auto kv_wait = [&](uint32_t idx) -> bool {
@@ -492,7 +492,7 @@ __device__ __forceinline__ void dec_mma_f8(const AttnParams& p, uint32_t sQ, uin
   constexpr uint32_t kIdescO = idesc_f16_f32(128, NR, true, false);
   uint32_t g = 0, q_cnt = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
 
   // S^T(gs) = K Q^T: A = widened K in TMEM (128 lanes = keys, 8 columns per
@@ -634,7 +634,7 @@ __device__ __forceinline__ void dec_softmax(const AttnParams& p, uint32_t sKV, u
   const int p_unit = (t & 63) >> 3;
   uint32_t g = 0, ld_base = 0, q_cnt = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = item_tiles(w, BN);
@@ -887,7 +887,7 @@ __global__ void __launch_bounds__(DecCfg<D, DecRows<RR>::NR, F8>::THREADS, 1)
   // everything above overlaps the scheduler kernel; its work list is read below
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int n_items = p.hdr->n_items;
+  const int n_items = list_count(p);
 
   if constexpr (F8) {
     // per-warpgroup register budgets first, then the roles

@@ -104,7 +104,8 @@ struct WsHeader {
   int n_split_reqs;   // requests split over KV (entries of the split list)
   int n_items2;       // items of the second list (query-block pairs, or widened requests)
   int n_wide_pages;   // pages of the widened requests (E4M3 pools, second list)
-  int pad[59];
+  int n_items_b;      // one-token segment after the main list's n_items (split_decode)
+  int pad[58];
 };
 
 constexpr int kBM = 128;              // query rows per tile (tcgen05 M)
@@ -115,7 +116,7 @@ constexpr int kQWarp = 6;
 constexpr int kProducer2Warp = 7;     // second K/V producer: one issuing warp per CTA
                                       // cannot keep HBM busy with page-sized boxes
 constexpr int kCostBuckets = 1024;
-constexpr int kSchedSmemReqs = 4096;  // unit offsets of up to this many requests live in smem
+constexpr int kSchedSmemReqs = 3072;  // unit offsets of up to this many requests live in smem
 constexpr int kMaxSplits = 64;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows > 2^8
 // Compensated P * V.  The softmax weights feed the P V product as 16-bit
@@ -134,15 +135,25 @@ constexpr int kCompKeys = 64;
 // (64-key tiles, 256 TMEM columns, ~100 KB of shared memory each): two
 // independent load -> S -> softmax -> P V chains per SM hide each other's
 // latencies, which one CTA per SM cannot.  D = 256 needs the whole SM.
-// F8: E4M3 pools.  The producer's TMA boxes land in NST fp8 staging tiles and
-// a converter warp widens them to fp16 in the 16-bit slots the MMAs read (one
-// slot fewer for D = 128, so the shared memory per CTA stays the same).
+// F8: E4M3 pools.  The producers' TMA boxes land in NST fp8 staging tiles and
+// the widening warp(s) turn them into fp16 in the 16-bit slots the MMAs read.
+// The loads in flight are what hides HBM latency, so F8 trades 16-bit slots
+// for staging tiles in the same shared memory: four staging tiles, and two
+// slots for D = 128 or three for D = 256 (the widening is quick next to a load;
+// two staging tiles with four or three slots was 7 % / 5 % slower).
 template <int D, bool F8 = false>
 struct TileCfg {
   static_assert(!F8 || D >= 128, "E4M3 pools: head_dim 128 or 256");
   static constexpr int CTAS = (D == 256) ? 1 : 2;      // CTAs per SM
-  // 16 warps on 4 sub-partitions: 4 warps x 32 lanes x 128 = 16 K registers each
-  static constexpr int MAXREG = (CTAS == 2) ? 128 : 255;
+  // E4M3 widening warps.  D = 256 (one CTA per SM): a warpgroup of four that
+  // shares every tile (one warp widened ~8 codes per clock, a third of the
+  // HBM rate), with a second producer; D = 128 (two CTAs per SM, every
+  // register taken): one.
+  static constexpr int NCONV = (F8 && D == 256) ? 4 : 1;
+  static constexpr int THREADS = (NCONV > 1) ? 384 : 256;
+  // two CTAs: 16 warps on 4 sub-partitions, 4 warps x 32 lanes x 128 = 16 K
+  // registers each; 384 threads: 168 (65 536 / 384, rounded down to 8)
+  static constexpr int MAXREG = (CTAS == 2) ? 128 : (THREADS == 384 ? 168 : 255);
   static constexpr int BN = 64;                       // keys per KV tile
   static constexpr int DCH = D / 64;                  // 128-byte column chunks per row
   static constexpr int Q_CHUNK = kBM * 128;           // bytes of one Q column chunk
@@ -150,8 +161,8 @@ struct TileCfg {
   static constexpr int SLOT_CHUNK = BN * 128;         // bytes of one K/V column chunk
   static constexpr int SLOT_BYTES = BN * D * 2;
   static constexpr int QBUF = (D == 64) ? 2 : 1;      // Q tiles in flight
-  static constexpr int NSLOT = F8 ? (D == 128 ? 3 : 4) : ((D == 64) ? 8 : (D == 128 ? 4 : 5));
-  static constexpr int NST = F8 ? 2 : 0;              // fp8 staging tiles
+  static constexpr int NSLOT = F8 ? (D == 128 ? 2 : 3) : ((D == 64) ? 8 : (D == 128 ? 4 : 5));
+  static constexpr int NST = F8 ? 4 : 0;              // fp8 staging tiles
   static constexpr int STAGE_BYTES = BN * D;          // D / 128 chunks of BN rows x 128 bytes
   static constexpr int O_COL = 2 * BN;                // TMEM: S0 [0,BN), S1 [BN,2BN), O
   static constexpr int TMEM_COLS = (O_COL + D <= 256) ? 256 : 512;
@@ -198,8 +209,17 @@ struct AttnParams {
   int fused_merge;            // 1: the last split warp of a (request, KV head) merges
   float scale_log2;           // softmax scale * log2(e) (times the K descale for E4M3 pools)
   float v_scale;              // V descale of E4M3 pools (1 for bf16 pools)
-  int list2;                  // 1: items is the second list (its count is hdr->n_items2)
+  int list;                   // 0: the main list; 1: items is the second list (hdr->n_items2);
+                              // 2: the one-token segment after the main list (hdr->n_items_b)
 };
+
+// The work list a kernel walks (see AttnParams::list).
+__device__ __forceinline__ const PackedItem* list_items(const AttnParams& p) {
+  return p.list == 2 ? p.items + p.hdr->n_items : p.items;
+}
+__device__ __forceinline__ int list_count(const AttnParams& p) {
+  return p.list == 1 ? p.hdr->n_items2 : (p.list == 2 ? p.hdr->n_items_b : p.hdr->n_items);
+}
 
 constexpr int kSoftmaxWarps = 4;      // softmax warps per CTA in every attention kernel
 
@@ -354,6 +374,10 @@ struct SchedParams {
   // non-decreasing; requests that are not widened own no pages).
   int wide_cap;
   int* wpre;
+  // 1: requests of one query token form a second segment of the main list
+  // (items [n_items, n_items + n_items_b)), for the decode kernel; the rest
+  // stay in the first segment
+  int split_decode;
   int* split_list;     // [B] requests with more than one split
   int4* req_info;      // [B] {n_splits, q_len, t_base, kv_len}
   int4* req_aux;       // [B] {units, tiles per split, KV tiles of the single block, 0}
@@ -480,14 +504,16 @@ __device__ __forceinline__ Unit unit_of(const SchedParams& p, const int4& ri, co
 // Atomics on the histogram and the cursors are aggregated per warp.
 __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ int hist[kCostBuckets];
-  __shared__ int cursor[kCostBuckets];
+  // cost buckets of the main list's two segments (the second one only with
+  // split_decode): [0, kCostBuckets) and [kCostBuckets, 2 kCostBuckets)
+  __shared__ int hist[2 * kCostBuckets];
+  __shared__ int cursor[2 * kCostBuckets];
   __shared__ unsigned long long total_tiles;
   __shared__ int s_chunk;
   __shared__ unsigned s_flags;
   __shared__ int warp_sums[32];
   const int tid = threadIdx.x, lane = tid & 31;
-  for (int i = tid; i < kCostBuckets; i += blockDim.x) hist[i] = 0;
+  for (int i = tid; i < 2 * kCostBuckets; i += blockDim.x) hist[i] = 0;
   if (tid == 0) { total_tiles = 0; s_flags = 0; }
   if (p.split_cnt)
     for (int i = tid; i < p.B * p.Hkv; i += blockDim.x) p.split_cnt[i] = 0;
@@ -656,19 +682,28 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
         if (uoff[mid] <= u) lo = mid; else hi = mid - 1;
       }
       const int4 ri = p.req_info[lo], ra = p.req_aux[lo];
-      if (!(ri.x == 1 && ra.x > 1)) key = cost_bucket(unit_of(p, ri, ra, u - uoff[lo]).cost);
+      if (!(ri.x == 1 && ra.x > 1))
+        key = cost_bucket(unit_of(p, ri, ra, u - uoff[lo]).cost) +
+              ((p.split_decode && ri.y == 1) ? kCostBuckets : 0);
     }
     const unsigned grp = __match_any_sync(0xffffffffu, key);
     if (key >= 0 && lane == __ffs(grp) - 1) atomicAdd(&hist[key], __popc(grp) * p.Hkv);
   }
   __syncthreads();
   {
+    // each segment longest first; the one-token segment after the other
     const int bucket = kCostBuckets - 1 - tid;
-    const int v = hist[bucket];
-    int total;
-    const int before = block_scan_1024(v, warp_sums, &total);
-    cursor[bucket] = before;
-    if (tid == 0) p.hdr->n_items = total < p.max_items ? total : p.max_items;
+    int total_a, total_b;
+    const int before_a = block_scan_1024(hist[bucket], warp_sums, &total_a);
+    const int before_b = block_scan_1024(hist[kCostBuckets + bucket], warp_sums, &total_b);
+    cursor[bucket] = before_a;
+    cursor[kCostBuckets + bucket] = total_a + before_b;
+    if (tid == 0) {
+      const int na = total_a < p.max_items ? total_a : p.max_items;
+      const int nb = total_b < p.max_items - na ? total_b : p.max_items - na;
+      p.hdr->n_items = na;
+      p.hdr->n_items_b = nb;
+    }
   }
   __syncthreads();
   for (int b = tid; b < p.B; b += blockDim.x) {
@@ -703,7 +738,7 @@ __global__ void __launch_bounds__(1024) pa_schedule_kernel(SchedParams p) {
       const int k = u - uoff[b];
       un = unit_of(p, ri, ra, k);
       if (ri.x == 1 && ra.x > 1) pos = ra.w + (ra.x - 1 - k) * p.Hkv;   // grouped request
-      else key = cost_bucket(un.cost);
+      else key = cost_bucket(un.cost) + ((p.split_decode && ri.y == 1) ? kCostBuckets : 0);
     }
     const unsigned grp = __match_any_sync(0xffffffffu, key);
     const int leader = __ffs(grp) - 1;
@@ -754,7 +789,7 @@ __device__ __forceinline__ void q_loader_role(const CUtensorMap* tm_q, const Att
   const int G = p.G;
   const int T = p.cu_q_lens ? p.cu_q_lens[p.B] : p.B;
   uint32_t q_cnt = 0;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (items.next(w)) {
     if (item_tiles(w, C::BN) == 0) continue;
@@ -844,7 +879,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = item_tiles(w, C::BN);
@@ -904,14 +939,15 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tm_k, const CUt
 // there, but 0 * NaN is not); K rows there only meet masked scores.
 template <int D>
 __device__ __forceinline__ void convert_role(const AttnParams& p, uint32_t sKV, uint32_t sST,
-                                             uint32_t bar0, int n_items, volatile int* abort) {
+                                             uint32_t bar0, int n_items, int cw,
+                                             volatile int* abort) {
   using C = TileCfg<D, true>;
   constexpr int UPR = D / 16;                        // 16-byte fp8 units per row
   constexpr int UNITS = C::BN * UPR;
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = item_tiles(w, C::BN);
@@ -929,8 +965,9 @@ __device__ __forceinline__ void convert_role(const AttnParams& p, uint32_t sKV, 
       const int zero_from = is_v ? max(0, min(C::BN, w.kv_len - n0)) : C::BN;
       const uint32_t src0 = sST + st * C::STAGE_BYTES;
       const uint32_t dst0 = sKV + slot * C::SLOT_BYTES;
+      // passes of 8 x 32 units, dealt round-robin to the NCONV widening warps
 #pragma unroll 1
-      for (int u0 = 0; u0 < UNITS; u0 += 8 * 32) {
+      for (int u0 = cw * 8 * 32; u0 < UNITS; u0 += C::NCONV * 8 * 32) {
         uint32_t x[8][4];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {                 // all loads of the pass first
@@ -989,7 +1026,7 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, uint32_t sQ, uint3
                                    : idesc_bf16_f32(kBM, D, false, true);
   uint32_t ld_idx = 0, g_base = 0, q_cnt = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = item_tiles(w, C::BN);
@@ -1122,7 +1159,7 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tm_o, const Attn
   const uint32_t sEpiW = sEpi + warp * C::EPI_WARP_BYTES;
   uint32_t g_base = 0, ld_base = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = item_tiles(w, BN);
@@ -1380,13 +1417,13 @@ __global__ void __maxnreg__((TileCfg<D, F8>::MAXREG))
       mbar_init(bar0 + 8 * (C::B_QEMPTY + i), 1);
     }
     for (int i = 0; i < C::NSLOT; ++i) {
-      // filled by TMA (one expect_tx arrival) or by the converter warp (F8)
-      mbar_init(bar0 + 8 * (C::B_KVFULL + i), 1);
+      // filled by TMA (one expect_tx arrival) or by the NCONV widening warps (F8)
+      mbar_init(bar0 + 8 * (C::B_KVFULL + i), F8 ? C::NCONV : 1);
       mbar_init(bar0 + 8 * (C::B_KVEMPTY + i), 1);
     }
     for (int i = 0; i < C::NST; ++i) {
       mbar_init(bar0 + 8 * (C::B_STFULL + i), 1);
-      mbar_init(bar0 + 8 * (C::B_STEMPTY + i), 1);
+      mbar_init(bar0 + 8 * (C::B_STEMPTY + i), C::NCONV);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar0 + 8 * (C::B_SFULL + i), 1);
@@ -1402,7 +1439,9 @@ __global__ void __maxnreg__((TileCfg<D, F8>::MAXREG))
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if ((warp == kProducerWarp || (!F8 && warp == kProducer2Warp)) && (threadIdx.x & 31) == 0) {
+  constexpr bool two_producers = !F8 || C::NCONV > 1;
+  if ((warp == kProducerWarp || (two_producers && warp == kProducer2Warp)) &&
+      (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
@@ -1414,14 +1453,27 @@ __global__ void __maxnreg__((TileCfg<D, F8>::MAXREG))
   // everything above overlaps the scheduler kernel; its work list is read below
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int n_items = p.list2 ? p.hdr->n_items2 : p.hdr->n_items;
+  const int n_items = list_count(p);
 
-  if (warp == kProducerWarp || warp == kProducer2Warp) {
-    if constexpr (F8) {
+  bool widening_warp = false;
+  if constexpr (F8 && C::NCONV > 1) {
+    // E4M3, D = 256: warps 8-11 widen each staged tile together
+    if (warp >= 8) {
+      convert_role<D>(p, sKV, sST, bar0, n_items, warp - 8, abort);
+      widening_warp = true;
+    }
+  }
+  if (widening_warp) {
+  } else if (warp == kProducerWarp || warp == kProducer2Warp) {
+    if constexpr (F8 && C::NCONV > 1) {
+      // two producers, one parity of the loads (and one staging tile) each
+      producer_role<D, true>(&tm_k, &tm_v, p, sST, bar0, n_items,
+                             warp == kProducerWarp ? 0u : 1u, abort);
+    } else if constexpr (F8) {
       // one producer issues every load into the staging ring; the other warp
       // widens the staged tiles into the 16-bit slots
       if (warp == kProducerWarp) producer_role<D, true>(&tm_k, &tm_v, p, sST, bar0, n_items, 2u, abort);
-      else convert_role<D>(p, sKV, sST, bar0, n_items, abort);
+      else convert_role<D>(p, sKV, sST, bar0, n_items, 0, abort);
     } else {
       producer_role<D, false>(&tm_k, &tm_v, p, sKV, bar0, n_items,
                               warp == kProducerWarp ? 0u : 1u, abort);

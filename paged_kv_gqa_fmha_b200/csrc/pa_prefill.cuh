@@ -103,7 +103,7 @@ __device__ __forceinline__ void pair_q_loader(const CUtensorMap* tm_q, const Att
   const int T = p.cu_q_lens ? p.cu_q_lens[p.B] : p.B;
   uint32_t qc[2] = {0, 0};
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const PairShape ps = pair_shape(w, p.tpb, C::BN, p.causal);
@@ -179,7 +179,7 @@ __device__ __forceinline__ void pair_producer(const CUtensorMap* tm_k, const CUt
   const int lane = threadIdx.x & 31;
   uint32_t ld_idx = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const int n = pair_shape(w, p.tpb, C::BN, p.causal).n;
@@ -236,7 +236,7 @@ __device__ __forceinline__ void pair_mma(const AttnParams& p, uint32_t sQ, uint3
   uint32_t g[2] = {0, 0};     // tiles processed per stage
   uint32_t itc[2] = {0, 0};   // items per stage with tiles (q_full / o_empty phases)
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
 
   auto kv_wait = [&](uint32_t idx) -> bool {
@@ -357,7 +357,7 @@ __device__ __forceinline__ void pair_softmax(const CUtensorMap* tm_o, const Attn
   const uint32_t sEpiW = sEpi + (4 * x + warp) * C::EPI_WARP_BYTES;
   uint32_t g = 0, ld_base = 0;
   bool ok = true;
-  ItemStream items(p.items, n_items, p.tpb);
+  ItemStream items(list_items(p), n_items, p.tpb);
   WorkItem w;
   while (ok && items.next(w)) {
     const PairShape ps = pair_shape(w, p.tpb, BN, p.causal);

@@ -251,7 +251,9 @@ WIDE_Q = [300, 1, 200, 150, 1]
 WIDE_KV = [300, 900, 500, 150, 2000]
 
 
-@pytest.mark.parametrize("max_pages,launches", [(-1, 4), (0, 2), (19, 4), (20, 4), (61, 4)])
+# launches: the scheduler, [the widening pass and the bf16 kernel,] the E4M3
+# one-stage kernel and the decode kernel (the batch's two decode rows)
+@pytest.mark.parametrize("max_pages,launches", [(-1, 5), (0, 3), (19, 5), (20, 5), (61, 5)])
 def test_fp8_widened_requests_match_oracle(max_pages, launches):
     """Requests of two or more query blocks over E4M3 pools are widened once
     into the bf16 scratch pool (in request order while their pages fit) and
@@ -310,3 +312,43 @@ def test_fp8_widen_rejects_bad_capacity():
     with pytest.raises(binding.PAError) as e:
         plan.set_kv_fp8_widen(-2)
     assert e.value.code == binding.PA_ERR_INVALID
+
+
+def test_fp8_batch_larger_than_scheduler_cache():
+    """3 200 requests over E4M3 pools (more than the scheduler's 3 072 cached
+    unit offsets): widened multi-block requests, one-token rows on the decode
+    kernel's segment (some of them split) and the rest, against the oracle."""
+    rng = np.random.default_rng(3201)
+    B = 3200
+    q_lens = [1] * B
+    kv_lens = [int(x) for x in rng.integers(1, 120, size=B)]
+    for b in range(0, B, 97):
+        q_lens[b] = kv_lens[b] = int(rng.integers(40, 160))
+    for b in range(3, B, 211):         # one-block chunks (q_len 2..8) stay on the E4M3 kernel
+        q_lens[b] = int(rng.integers(2, 9))
+        kv_lens[b] = max(kv_lens[b], q_lens[b])
+    for b in range(5, B, 401):
+        kv_lens[b] = 3000
+    spec = W.custom_spec("fp8_big_batch", 8, 2, 128, 16, q_lens, kv_lens)
+    w, k8, v8 = _fp8_workload(spec, 3201)
+    out, lse = _run(_plan(w), w, k8, v8, use_cu=True)
+    compare(out, lse, *_oracle(w, k8, v8))
+
+
+@pytest.mark.parametrize("decode_kernel", [True, False])
+def test_fp8_mixed_decode_rows_on_either_kernel(decode_kernel):
+    """Decode rows of a mixed batch over E4M3 pools run on the decode kernel
+    (default at head_dim 128: a second segment of the work list) or, with
+    pa_set_decode_kernel(0), on the one-stage kernel; both match the oracle,
+    with KV splits and the launch count of each path."""
+    spec = W.custom_spec("fp8_segs", 32, 8, 128, 16, [300, 1, 1, 5, 1, 64],
+                         [300, 2500, 90, 700, 1, 64])
+    w, k8, v8 = _fp8_workload(spec, 67)
+    plan = _plan(w, num_splits=3)
+    plan.set_decode_kernel(decode_kernel)
+    plan.profile_start(1)
+    out, lse = _run(plan, w, k8, v8, use_cu=True)
+    _, n, per_run = plan.profile_read()
+    # scheduler, widening, bf16 kernel (widened), E4M3 one-stage, [decode kernel], merge
+    assert per_run == (6 if decode_kernel else 5)
+    compare(out, lse, *_oracle(w, k8, v8))

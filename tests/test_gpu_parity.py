@@ -505,3 +505,22 @@ def test_wait_timeout_sets_status_and_releases_other_roles(limit_us):
     out, lse, plan = gpu_run(w, use_cu=False)
     assert plan.status() == 0
     compare(out, lse, *oracle_all(w))
+
+
+def test_batch_larger_than_scheduler_cache():
+    """More requests (3 200) than the scheduler keeps unit offsets for in shared
+    memory (3 072), so its later requests' offsets come from global memory:
+    decode rows, multi-block prefill requests and a few long-KV rows that split,
+    every element against the oracle."""
+    rng = np.random.default_rng(3200)
+    B = 3200
+    q_lens = [1] * B
+    kv_lens = [int(x) for x in rng.integers(1, 120, size=B)]
+    for b in range(0, B, 97):          # prefill requests of two or more blocks
+        q_lens[b] = kv_lens[b] = int(rng.integers(40, 160))
+    for b in range(5, B, 401):         # long decode rows
+        kv_lens[b] = 3000
+    spec = W.custom_spec("big_batch", 8, 2, 128, 16, q_lens, kv_lens)
+    w = gen(spec, 3200)
+    out, lse, _ = gpu_run(w)
+    compare(out, lse, *oracle_all(w))
