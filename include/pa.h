@@ -355,10 +355,10 @@ PA_API int pa_profile_read(pa_plan *plan, float *attn_ms, int *n_runs, int *laun
  * its kernels run.  Calls whose work overlaps on the GPU (different streams,
  * or several threads) race on the array and must be serialised by the caller.
  *
- * The first call on a device performs a one-time set-up on that device (it
- * resolves the array's device address with cudaGetSymbolAddress and sets the
- * kernel's shared-memory limit); make that first call before any stream
- * capture.  Later calls only enqueue work.
+ * The first call on a device performs a one-time set-up on that device with
+ * synchronous runtime calls (it resolves the array's device address with
+ * cudaGetSymbolAddress and sets the kernel's shared-memory limit).  Later
+ * calls only enqueue work.
  *
  * Arguments are those of pa_create_plan followed by those of pa_run, plus
  *   num_pages  pool size P for page-id checks (0 = trust the table)

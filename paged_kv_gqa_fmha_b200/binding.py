@@ -336,8 +336,8 @@ def run_noalloc(q, k_pool, v_pool, page_table, seq_lens, cu_q_lens, out, lse, *,
     own allocator, a loop that must not stall on an allocation); the
     library's static scratch array replaces the plan's workspace.  Every
     output tensor is passed in; nothing is allocated here or in the library.
-    The first call on a device does a one-time set-up there, so make it
-    before any stream capture.  Calls that overlap on the GPU race on the
+    The first call on a device does a one-time set-up there with
+    synchronous runtime calls.  Calls that overlap on the GPU race on the
     shared scratch.  Pools are bf16 only.  Read the status word with
     ``noalloc_status`` before the next call, which clears it."""
     lib = load_library()
