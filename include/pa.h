@@ -128,11 +128,8 @@ PA_API pa_plan *pa_create_plan(int batch, int heads_q, int heads_kv, int head_di
  * Enqueues at most five kernels (scheduler; the two-stage prefill kernel when
  * enabled, or with E4M3 pools and cu_q_lens the widening pass and the bf16
  * attention kernel over the widened requests; attention; split merge); does
- * not synchronise and reads no device data on the host, so it can be captured
- * in a CUDA graph.  It does not allocate, with one exception: the first run
- * over E4M3 pools with cu_q_lens allocates the widening scratch pool
- * (pa_set_kv_fp8_widen), so such a run must happen once before capture (or
- * the capacity be set to 0).  The
+ * not allocate, does not synchronise and reads no device data on the host, so
+ * it can be captured in a CUDA graph.  The
  * scheduler may start while the previous pa_run on the same plan and stream
  * is still finishing (it writes the other of two work-list buffers) and ends
  * only after that run, so consecutive runs keep stream order.  Returns PA_OK, PA_ERR_INVALID
@@ -270,7 +267,9 @@ PA_API int pa_selftest_wait_timeout(uint32_t limit_us, uint32_t *status_out,
  *     P in fp16 as above.
  * Neither path uses the two-stage kernel (pa_set_two_stage_prefill reads bf16
  * pools only).  on = 0 restores bf16 pools (descales ignored).  Turning the
- * mode on or off resizes the plan's work-list workspace (synchronous; call it
+ * mode on or off resizes the plan's work-list workspace, and on allocates the
+ * scratch pool of widened requests (pa_set_kv_fp8_widen; set its capacity
+ * first to avoid a transient allocation), off frees it (synchronous; call it
  * outside graph capture).
  * Returns PA_ERR_INVALID for a NULL plan or a descale that is not finite and
  * > 0, PA_ERR_UNSUPPORTED for a head_dim other than 128 or 256, PA_ERR_CUDA
@@ -279,16 +278,18 @@ PA_API int pa_set_kv_fp8(pa_plan *plan, int on, float k_scale, float v_scale);
 
 /* Scratch capacity, in pages, for widened E4M3 requests (see pa_set_kv_fp8).
  * The scratch pool holds bf16 K and V pages [max_pages, ps, Hkv, D] plus a
- * page table [B, C]; the first pa_run over E4M3 pools with cu_q_lens allocates
- * it (cudaMalloc; PA_ERR_CUDA from that pa_run if the allocation fails), and
- * it lives until the plan is destroyed or the capacity changes.  Requests of
+ * page table [B, C]; pa_set_kv_fp8 (on) allocates it, and so does this call
+ * while E4M3 pools are on (cudaMalloc, synchronous: call it outside graph
+ * capture; PA_ERR_CUDA if the allocation fails, after which the plan widens
+ * nothing until a capacity is set that fits).  It lives until the plan is
+ * destroyed, E4M3 pools are turned off or the capacity changes.  Requests of
  * two or more query blocks are widened in request order while their pages
  * (ceil(kv_len / ps) each) fit; the rest run on the E4M3 one-stage kernel, so
  * every capacity gives the same results within the stated tolerances.
  * max_pages = -1 (default): every page the batch can hold (B * C), at most
  * 512 MiB of K and V; 0: never widen; n > 0: n pages (at most B * C).  A new
- * value frees the current scratch pool (cudaFree synchronises the device).
- * Returns PA_ERR_INVALID for a NULL plan or max_pages < -1. */
+ * value frees the current scratch pool first (cudaFree synchronises the
+ * device).  Returns PA_ERR_INVALID for a NULL plan or max_pages < -1. */
 PA_API int pa_set_kv_fp8_widen(pa_plan *plan, int max_pages);
 
 /* Paged KV append: write this step's new K and V rows into the pools before

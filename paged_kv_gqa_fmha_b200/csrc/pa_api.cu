@@ -514,7 +514,7 @@ int alloc_widen(pa_plan* p) {
   void* buf = nullptr;
   cudaError_t e = cudaMalloc(&buf, bytes);
   if (e != cudaSuccess) {
-    set_err("pa_run: cudaMalloc of %zu bytes for the widened E4M3 pages failed: %s "
+    set_err("cudaMalloc of %zu bytes for the widened E4M3 pages failed: %s "
             "(pa_set_kv_fp8_widen sets a smaller capacity, or 0 for none)",
             bytes, cudaGetErrorString(e));
     return PA_ERR_CUDA;
@@ -759,11 +759,9 @@ int pa_run(pa_plan* p, const void* q, const void* k_pool, const void* v_pool,
   const bool pairs = p->use_pairs && cu_q_lens != nullptr && !p->kv_fp8;
   // E4M3 pools with query blocks: requests of two or more blocks are widened
   // once (pa_widen_kernel) and run on the bf16 kernel from the second list
-  const bool wide = p->kv_fp8 && cu_q_lens != nullptr && p->widen_req != 0;
-  if (wide && p->widen_buf == nullptr) {
-    rc = alloc_widen(p);
-    if (rc) return rc;
-  }
+  // (the scratch pool is allocated by pa_set_kv_fp8 / pa_set_kv_fp8_widen;
+  // pa_run allocates nothing)
+  const bool wide = p->kv_fp8 && cu_q_lens != nullptr && p->widen_buf != nullptr;
   sp.items2 = (pairs || wide) ? bufs.items2 : nullptr;
   sp.wide_cap = wide ? p->widen_cap : 0;
   sp.wpre = bufs.wpre;
@@ -1004,6 +1002,7 @@ int pa_set_kv_fp8(pa_plan* p, int on, float k_scale, float v_scale) {
       p->kv_fp8 = 0;
       int rc = alloc_workspace(p);   // the second list shrinks back
       if (rc != PA_OK) { p->kv_fp8 = 1; return rc; }
+      free_widen(p);
     }
     p->k_scale = p->v_scale = 1.0f;
     return PA_OK;
@@ -1020,6 +1019,14 @@ int pa_set_kv_fp8(pa_plan* p, int on, float k_scale, float v_scale) {
   if (!p->kv_fp8) {
     p->kv_fp8 = 1;
     int rc = alloc_workspace(p);     // room for the blocks of widened requests
+    if (rc == PA_OK && p->widen_req != 0) {
+      rc = alloc_widen(p);           // the scratch pool of widened requests
+      if (rc != PA_OK) {
+        p->kv_fp8 = 0;
+        alloc_workspace(p);          // back to the bf16 sizes (smaller: cannot fail on memory)
+        return rc;
+      }
+    }
     if (rc != PA_OK) { p->kv_fp8 = 0; return rc; }
   }
   p->k_scale = k_scale;
@@ -1034,8 +1041,12 @@ int pa_set_kv_fp8_widen(pa_plan* p, int max_pages) {
     return PA_ERR_INVALID;
   }
   if (max_pages != p->widen_req) {
-    free_widen(p);     // the next run that needs it allocates the new capacity
+    free_widen(p);
     p->widen_req = max_pages;
+    if (p->kv_fp8 && max_pages != 0) {
+      int rc = alloc_widen(p);       // the new capacity, now
+      if (rc != PA_OK) return rc;    // (the plan then widens nothing)
+    }
   }
   return PA_OK;
 }

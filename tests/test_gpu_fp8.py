@@ -352,3 +352,24 @@ def test_fp8_mixed_decode_rows_on_either_kernel(decode_kernel):
     # scheduler, widening, bf16 kernel (widened), E4M3 one-stage, [decode kernel], merge
     assert per_run == (6 if decode_kernel else 5)
     compare(out, lse, *_oracle(w, k8, v8))
+
+
+def test_fp8_run_allocates_nothing():
+    """pa_set_kv_fp8 allocates the widening scratch pool; pa_run over E4M3
+    pools with cu_q_lens (widening pass included) then allocates no device
+    memory: free memory is unchanged across runs with preallocated outputs."""
+    spec = W.custom_spec("fp8_noalloc", 16, 4, 128, 16, WIDE_Q, WIDE_KV)
+    w, k8, v8 = _fp8_workload(spec, 71)
+    plan = _plan(w)
+    out = torch.empty_like(w["q"])
+    lse = torch.empty(w["T"], w["Hq"], device="cuda")
+    args = (w["q"], k8, v8, w["page_table"], w["seq_lens"], w["cu_q_lens"])
+    plan.run(*args, out=out, lse=lse)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        plan.run(*args, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert plan.status() == 0
+    compare(out, lse, *_oracle(w, k8, v8))
