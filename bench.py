@@ -597,8 +597,9 @@ def kv_fp8_rates(bw, tf):
     picks (the E4M3 decode kernel at head_dim 128, the one-stage kernel's E4M3
     variant at 256); in prefill and mixed batches the requests of two or more
     query blocks are widened once into bf16 scratch pages (pa_widen_kernel)
-    and run on the bf16 one-stage kernel, the rest on its E4M3 variant; the
-    time covers all of these launches.  Bytes
+    and run on the bf16 one-stage kernel, rows of one query token on the E4M3
+    decode kernel (head_dim 128) and the rest on the one-stage kernel's E4M3
+    variant; the time covers all of these launches.  Bytes
     per launch = the bf16 formula with K and V at one byte per element;
     per-launch CUDA events (the plan's profile pairs) over 20 launches, each
     synchronised, after 5 warm-up launches (pools larger than L2)."""
@@ -632,6 +633,9 @@ def kv_fp8_rates(bw, tf):
         else:
             kernel = ("pa_widen_kernel + pa_attention_kernel<{0}, false> (widened requests) + "
                       "pa_attention_kernel<{0}, true>".format(w["D"]))
+            if w["D"] == 128 and G <= 32:
+                kernel += " + pa_decode_kernel<128, %d, true> (one-token rows)" % max(
+                    4, 1 << (G - 1).bit_length())
         out[name] = {"attn_kernel_ms": ms, "algorithmic_bytes": nbytes, "flops": c["flops"],
                      "kernel_GBps": gbs, "kernel_TFLOPs": tfs, "hbm_frac": gbs / bw,
                      "tensor_frac": tfs / tf, "status_word": plan.status(), "kernel": kernel}
